@@ -1,0 +1,359 @@
+"""Pins for the fp64 oracle: checks against facts that do not come from the oracle.
+
+Each ``check_*`` returns ``(ok, message)`` so the same battery can (a) pass on
+the oracle the suite trusts and (b) be shown to fail on copies of the oracle
+with one planted mistake.  The facts used:
+
+* brute-force central finite differences of L = sum(dO * O) (pins the whole
+  backward against the forward);
+* an independent fp64 torch implementation (explicit mask + softmax + matmul,
+  gradients by autograd) -- the special case "library routine";
+* scipy's logsumexp over explicitly computed scores;
+* closed forms: constant V gives O = V; Q = 0 gives the mean of the allowed
+  values and LSE = log(#allowed); a causal row 0 sees only key 0; a single key
+  gives O = v_0; shifting every key of a segment by one vector leaves O
+  unchanged and moves LSE_i by scale * <q_i, shift>;
+* gradient identities: sum_j dK_j = 0 (each row of dS sums to zero) and
+  sum_j dV_j = sum over the group's rows of dO (each row of P sums to one);
+* structure: a packed varlen batch equals independent dense calls, and GQA
+  equals MHA with K/V repeated per group (dK/dV then sum over the group).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+from scipy.special import logsumexp
+
+import oracle
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _rand(shape, seed):
+    return _rng(seed).standard_normal(shape)
+
+
+def _cu(lengths):
+    cu = np.zeros(len(lengths) + 1, np.int32)
+    cu[1:] = np.cumsum(lengths)
+    return cu
+
+
+def _close(a, b, tol):
+    a, b = np.asarray(a), np.asarray(b)
+    fin = np.isfinite(b)
+    if not np.array_equal(np.isfinite(a), fin):
+        return False, "finite pattern differs"
+    if not np.array_equal(a[~fin], b[~fin]):
+        return False, "non-finite values differ"
+    if fin.sum() == 0:
+        return True, "ok"
+    err = float(np.max(np.abs(a[fin] - b[fin])))
+    scale = max(1.0, float(np.max(np.abs(b[fin]))))
+    return (err <= tol * scale), f"max err {err:.3e} (tol {tol:.1e} x {scale:.2e})"
+
+
+# --------------------------------------------------------------------------
+# independent torch fp64 implementation (explicit mask, autograd)
+# --------------------------------------------------------------------------
+def torch_reference(q, k, v, dout, lengths_q, lengths_k, scale, causal):
+    """Dense per-segment softmax(scale QK^T + mask) V with autograd (fp64 CPU)."""
+    tq = torch.tensor(q, dtype=torch.float64, requires_grad=True)
+    tk = torch.tensor(k, dtype=torch.float64, requires_grad=True)
+    tv = torch.tensor(v, dtype=torch.float64, requires_grad=True)
+    Hq, Hkv = q.shape[1], k.shape[1]
+    G = Hq // Hkv
+    outs, lses = [], []
+    oq = ok_ = 0
+    for sq, sk in zip(lengths_q, lengths_k):
+        qs = tq[oq:oq + sq].permute(1, 0, 2)                      # [Hq, sq, D]
+        ks = tk[ok_:ok_ + sk].permute(1, 0, 2).repeat_interleave(G, 0)
+        vs = tv[ok_:ok_ + sk].permute(1, 0, 2).repeat_interleave(G, 0)
+        s = scale * qs @ ks.transpose(1, 2)                       # [Hq, sq, sk]
+        i = torch.arange(sq).view(-1, 1)
+        j = torch.arange(sk).view(1, -1)
+        allowed = (j <= i + (sk - sq)) if causal else torch.ones(sq, sk, dtype=torch.bool)
+        s = s.masked_fill(~allowed, float("-inf"))
+        lse = torch.logsumexp(s, dim=-1)                          # [Hq, sq]
+        p = torch.exp(s - lse.unsqueeze(-1))
+        p = torch.nan_to_num(p, nan=0.0)
+        outs.append((p @ vs).permute(1, 0, 2))
+        lses.append(lse)
+        oq += sq
+        ok_ += sk
+    out = torch.cat(outs, 0)
+    lse = torch.cat(lses, 1)
+    grads = (None, None, None)
+    if dout is not None:
+        (out * torch.tensor(dout, dtype=torch.float64)).sum().backward()
+        grads = tuple(t.grad.numpy() if t.grad is not None else np.zeros(t.shape)
+                      for t in (tq, tk, tv))
+    return out.detach().numpy(), lse.detach().numpy(), grads
+
+
+# --------------------------------------------------------------------------
+# the battery
+# --------------------------------------------------------------------------
+CASES = [
+    # (lengths_q, lengths_k, Hq, Hkv, D, causal)
+    ([7], [7], 2, 1, 4, False),
+    ([7], [7], 2, 1, 4, True),
+    ([3, 5], [3, 5], 2, 2, 8, True),
+    ([4, 6], [6, 3], 4, 2, 4, True),      # s_q != s_k, bottom-right causal
+    ([5, 0, 4], [5, 0, 4], 2, 1, 4, False),  # a zero-length segment
+]
+
+
+def check_finite_differences(mutation=0, eps=1e-6, tol=1e-6):
+    for ci, (lq, lk, Hq, Hkv, D, causal) in enumerate(CASES):
+        Tq, Tk = sum(lq), sum(lk)
+        q = _rand((Tq, Hq, D), 10 + ci)
+        k = _rand((Tk, Hkv, D), 20 + ci)
+        v = _rand((Tk, Hkv, D), 30 + ci)
+        do = _rand((Tq, Hq, D), 40 + ci)
+        scale = 0.7
+        cq, ck = _cu(lq), _cu(lk)
+        dq, dk, dv = oracle.bwd(q, k, v, do, cq, ck, scale, causal, mutation=mutation)
+
+        def loss(q_, k_, v_):
+            o, _ = oracle.fwd(q_, k_, v_, cq, ck, scale, causal, mutation=mutation)
+            return float(np.sum(o * do))
+
+        for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            num = np.zeros_like(x)
+            flat = x.reshape(-1)
+            for t in range(flat.size):
+                old = flat[t]
+                flat[t] = old + eps
+                lp = loss(q, k, v)
+                flat[t] = old - eps
+                lm = loss(q, k, v)
+                flat[t] = old
+                num.reshape(-1)[t] = (lp - lm) / (2 * eps)
+            ok, msg = _close(g, num, tol)
+            if not ok:
+                return False, f"FD case {ci} d{name}: {msg}"
+    return True, "ok"
+
+
+def check_torch_reference(mutation=0, tol=1e-12):
+    for ci, (lq, lk, Hq, Hkv, D, causal) in enumerate(CASES):
+        Tq, Tk = sum(lq), sum(lk)
+        q = _rand((Tq, Hq, D), 50 + ci)
+        k = _rand((Tk, Hkv, D), 60 + ci)
+        v = _rand((Tk, Hkv, D), 70 + ci)
+        do = _rand((Tq, Hq, D), 80 + ci)
+        scale = D ** -0.5
+        cq, ck = _cu(lq), _cu(lk)
+        o, lse = oracle.fwd(q, k, v, cq, ck, scale, causal, mutation=mutation)
+        dq, dk, dv = oracle.bwd(q, k, v, do, cq, ck, scale, causal, mutation=mutation)
+        ro, rlse, (rdq, rdk, rdv) = torch_reference(q, k, v, do, lq, lk, scale, causal)
+        for name, a, b in (("O", o, ro), ("LSE", lse, rlse), ("dQ", dq, rdq),
+                           ("dK", dk, rdk), ("dV", dv, rdv)):
+            ok, msg = _close(a, b, tol)
+            if not ok:
+                return False, f"torch case {ci} {name}: {msg}"
+    return True, "ok"
+
+
+def check_lse_logsumexp(mutation=0):
+    lq = [9, 16]
+    Hq, Hkv, D = 4, 2, 8
+    q = 3 * _rand((25, Hq, D), 1)      # large scores: the max term matters
+    k = 3 * _rand((25, Hkv, D), 2)
+    v = _rand((25, Hkv, D), 3)
+    for causal in (False, True):
+        _, lse = oracle.fwd(q, k, v, _cu(lq), _cu(lq), 0.5, causal, mutation=mutation)
+        off = 0
+        for s in lq:
+            for h in range(Hq):
+                hk = h // (Hq // Hkv)
+                sc = 0.5 * q[off:off + s, h] @ k[off:off + s, hk].T
+                if causal:
+                    sc = np.where(np.tri(s, s, 0, dtype=bool), sc, -np.inf)
+                ref = logsumexp(sc, axis=1)
+                ok, msg = _close(lse[h, off:off + s], ref, 1e-12)
+                if not ok:
+                    return False, f"logsumexp causal={causal} h={h}: {msg}"
+            off += s
+    return True, "ok"
+
+
+def check_closed_forms(mutation=0):
+    Hq, Hkv, D = 4, 2, 8
+    lq = [6, 11]
+    cu = _cu(lq)
+    T = sum(lq)
+    q = _rand((T, Hq, D), 4)
+    k = _rand((T, Hkv, D), 5)
+    # constant V -> O = V
+    c = _rand((1, Hkv, D), 6)
+    vconst = np.repeat(c, T, axis=0)
+    for causal in (False, True):
+        o, _ = oracle.fwd(q, k, vconst, cu, cu, 0.9, causal, mutation=mutation)
+        G = Hq // Hkv
+        ref = np.repeat(c, G, axis=1).repeat(T, axis=0)
+        ok, msg = _close(o, ref, 1e-12)
+        if not ok:
+            return False, f"constant V causal={causal}: {msg}"
+    # causal row 0 sees only key 0: O_0 = v_0, LSE_0 = s_00
+    v = _rand((T, Hkv, D), 7)
+    o, lse = oracle.fwd(q, k, v, cu, cu, 0.9, True, mutation=mutation)
+    off = 0
+    for s in lq:
+        for h in range(Hq):
+            hk = h // (Hq // Hkv)
+            ok, msg = _close(o[off, h], v[off, hk], 1e-12)
+            if not ok:
+                return False, f"causal row 0 O: {msg}"
+            ok, msg = _close(lse[h, off], 0.9 * q[off, h] @ k[off, hk], 1e-12)
+            if not ok:
+                return False, f"causal row 0 LSE: {msg}"
+        off += s
+    # Q = 0 -> uniform weights over the allowed keys
+    qz = np.zeros_like(q)
+    for causal in (False, True):
+        o, lse = oracle.fwd(qz, k, v, cu, cu, 0.9, causal, mutation=mutation)
+        off = 0
+        for s in lq:
+            for h in range(Hq):
+                hk = h // (Hq // Hkv)
+                for i in range(s):
+                    n = (i + 1) if causal else s
+                    ok, msg = _close(o[off + i, h], v[off:off + n, hk].mean(0), 1e-12)
+                    if not ok:
+                        return False, f"Q=0 causal={causal} O: {msg}"
+                    ok, msg = _close(lse[h, off + i], np.log(n), 1e-12)
+                    if not ok:
+                        return False, f"Q=0 causal={causal} LSE: {msg}"
+            off += s
+    # a single key: O = v_0 for every query row, LSE = its score
+    q1 = _rand((5, 2, D), 8)
+    k1 = _rand((1, 1, D), 9)
+    v1 = _rand((1, 1, D), 10)
+    o, lse = oracle.fwd(q1, k1, v1, _cu([5]), _cu([1]), 0.3, False, mutation=mutation)
+    ok, msg = _close(o, np.broadcast_to(v1, o.shape), 1e-12)
+    if not ok:
+        return False, f"single key O: {msg}"
+    ok, msg = _close(lse, 0.3 * np.einsum("thd,d->ht", q1, k1[0, 0]), 1e-12)
+    if not ok:
+        return False, f"single key LSE: {msg}"
+    # shifting every key of a segment by one vector: O unchanged, LSE shifts
+    shift = _rand((1, Hkv, D), 11)
+    for causal in (False, True):
+        o0, l0 = oracle.fwd(q, k, v, cu, cu, 0.9, causal, mutation=mutation)
+        o1, l1 = oracle.fwd(q, k + shift, v, cu, cu, 0.9, causal, mutation=mutation)
+        ok, msg = _close(o1, o0, 1e-10)
+        if not ok:
+            return False, f"key shift O causal={causal}: {msg}"
+        G = Hq // Hkv
+        dl = 0.9 * np.einsum("thd,hd->ht", q, np.repeat(shift[0], G, axis=0))
+        ok, msg = _close(l1, l0 + dl, 1e-10)
+        if not ok:
+            return False, f"key shift LSE causal={causal}: {msg}"
+    return True, "ok"
+
+
+def check_gradient_identities(mutation=0):
+    Hq, Hkv, D = 4, 2, 8
+    lq = [13, 6]
+    cu = _cu(lq)
+    T = sum(lq)
+    q, k, v, do = (_rand((T, h, D), s) for h, s in ((Hq, 12), (Hkv, 13), (Hkv, 14), (Hq, 15)))
+    G = Hq // Hkv
+    for causal in (False, True):
+        dq, dk, dv = oracle.bwd(q, k, v, do, cu, cu, 0.6, causal, mutation=mutation)
+        off = 0
+        for s in lq:
+            ok, msg = _close(dk[off:off + s].sum(0), np.zeros((Hkv, D)), 1e-12)
+            if not ok:
+                return False, f"sum dK causal={causal}: {msg}"
+            ref = do[off:off + s].sum(0).reshape(Hkv, G, D).sum(1)
+            ok, msg = _close(dv[off:off + s].sum(0), ref, 1e-12)
+            if not ok:
+                return False, f"sum dV causal={causal}: {msg}"
+            off += s
+    return True, "ok"
+
+
+def check_structure(mutation=0):
+    Hq, Hkv, D = 4, 2, 8
+    lq = [5, 9, 1, 7]
+    cu = _cu(lq)
+    T = sum(lq)
+    q, k, v, do = (_rand((T, h, D), s) for h, s in ((Hq, 16), (Hkv, 17), (Hkv, 18), (Hq, 19)))
+    G = Hq // Hkv
+    for causal in (False, True):
+        o, lse = oracle.fwd(q, k, v, cu, cu, 0.4, causal, mutation=mutation)
+        dq, dk, dv = oracle.bwd(q, k, v, do, cu, cu, 0.4, causal, mutation=mutation)
+        # each segment alone gives bit-identical results
+        off = 0
+        for s in lq:
+            sl = slice(off, off + s)
+            c1 = _cu([s])
+            o1, l1 = oracle.fwd(q[sl], k[sl], v[sl], c1, c1, 0.4, causal, mutation=mutation)
+            d1 = oracle.bwd(q[sl], k[sl], v[sl], do[sl], c1, c1, 0.4, causal, mutation=mutation)
+            if not (np.array_equal(o1, o[sl]) and np.array_equal(l1, lse[:, sl])):
+                return False, f"varlen segment fwd differs (causal={causal})"
+            if not all(np.array_equal(a, b[sl]) for a, b in zip(d1, (dq, dk, dv))):
+                return False, f"varlen segment bwd differs (causal={causal})"
+            off += s
+        # GQA == MHA on K/V repeated per contiguous group
+        kr, vr = np.repeat(k, G, axis=1), np.repeat(v, G, axis=1)
+        om, lm = oracle.fwd(q, kr, vr, cu, cu, 0.4, causal, mutation=mutation)
+        dqm, dkm, dvm = oracle.bwd(q, kr, vr, do, cu, cu, 0.4, causal, mutation=mutation)
+        for name, a, b in (("O", o, om), ("LSE", lse, lm), ("dQ", dq, dqm),
+                           ("dK", dk, dkm.reshape(T, Hkv, G, D).sum(2)),
+                           ("dV", dv, dvm.reshape(T, Hkv, G, D).sum(2))):
+            ok, msg = _close(a, b, 1e-12)
+            if not ok:
+                return False, f"GQA vs repeated MHA {name} causal={causal}: {msg}"
+    return True, "ok"
+
+
+def check_rows_match_full(mutation=0):
+    Hq, Hkv, D = 4, 1, 8
+    lq = [10, 17]
+    cu = _cu(lq)
+    T = sum(lq)
+    q, k, v, do = (_rand((T, h, D), s) for h, s in ((Hq, 20), (Hkv, 21), (Hkv, 22), (Hq, 23)))
+    for causal in (False, True):
+        o, lse = oracle.fwd(q, k, v, cu, cu, 0.5, causal, mutation=mutation)
+        dq, _, _ = oracle.bwd(q, k, v, do, cu, cu, 0.5, causal, mutation=mutation)
+        heads = np.array([0, 3, 1, 2, 2], np.int32)
+        rows = np.array([0, 9, 10, 26, 13], np.int64)
+        ro, rl, rdq = oracle.rows(q, k, v, cu, cu, 0.5, causal, heads, rows, dout=do,
+                                  mutation=mutation)
+        if not (np.array_equal(ro, o[rows, heads]) and np.array_equal(rl, lse[heads, rows])
+                and np.array_equal(rdq, dq[rows, heads])):
+            return False, f"sampled rows differ from the full oracle (causal={causal})"
+    return True, "ok"
+
+
+def check_fully_masked_rows(mutation=0):
+    # causal with s_q > s_k: the first s_q - s_k rows see no key at all
+    q = _rand((6, 1, 4), 24)
+    k = _rand((3, 1, 4), 25)
+    v = _rand((3, 1, 4), 26)
+    do = _rand((6, 1, 4), 27)
+    o, lse = oracle.fwd(q, k, v, _cu([6]), _cu([3]), 1.0, True, mutation=mutation)
+    if not (np.all(o[:3] == 0) and np.all(np.isneginf(lse[0, :3])) and np.all(np.isfinite(lse[0, 3:]))):
+        return False, "fully masked rows are not O=0, LSE=-inf"
+    dq, dk, dv = oracle.bwd(q, k, v, do, _cu([6]), _cu([3]), 1.0, True, mutation=mutation)
+    if not (np.all(dq[:3] == 0) and np.all(np.isfinite(dk)) and np.all(np.isfinite(dv))):
+        return False, "fully masked rows leak into gradients"
+    return True, "ok"
+
+
+ALL_CHECKS = [
+    check_closed_forms,
+    check_lse_logsumexp,
+    check_gradient_identities,
+    check_structure,
+    check_rows_match_full,
+    check_fully_masked_rows,
+    check_torch_reference,
+    check_finite_differences,
+]
