@@ -1,0 +1,179 @@
+"""Exact attention on B200 (sm_100a): thin Python binding over libattn.so.
+
+Every step of the computation runs in the CUDA kernels behind the C ABI in
+``include/attn.h``; this module only marshals torch tensors (device memory,
+current stream) into that ABI.  There is no CPU fallback: if the library is
+missing or the tensors are not on a CUDA device, calls raise.
+
+Functions
+---------
+attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, ...)
+    -> (out, lse)
+attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, ...)
+    -> (dq, dk, dv)
+attention(...)  autograd-aware forward (backward through attn_bwd)
+last_device_error() -> (status, message)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["attn_fwd", "attn_bwd", "attention", "bwd_workspace_size", "last_device_error",
+           "library", "LIB_PATH", "AttnError", "STATUS"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
+STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED",
+          3: "ATTN_ERR_CUDA", 4: "ATTN_ERR_TIMEOUT"}
+EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_last_device_error",
+            "attn_version")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Load libattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m exact_attention_129_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+        lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                 f32, i32, i32, vp, vp, vp]
+        lib.attn_fwd.restype = ctypes.c_int
+        lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                 i32, i32, f32, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        lib.attn_bwd.restype = ctypes.c_int
+        lib.attn_bwd_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.attn_bwd_workspace_size.restype = ctypes.c_size_t
+        lib.attn_last_device_error.argtypes = [vp, ctypes.c_char_p, ctypes.c_size_t]
+        lib.attn_last_device_error.restype = ctypes.c_int
+        lib.attn_version.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("exact_attention_129_b200 runs on CUDA tensors only")
+
+
+def _check_layout(name, t, dtype):
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
+             scale=None, causal=False, return_lse=True, out=None, lse=None):
+    """Forward pass. q [Tq,Hq,D], k/v [Tk,Hkv,D] bf16; returns (out, lse or None)."""
+    _check_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k, out, lse)
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_layout(n, t, torch.bfloat16)
+    _check_layout("cu_seqlens_q", cu_seqlens_q, torch.int32)
+    _check_layout("cu_seqlens_k", cu_seqlens_k, torch.int32)
+    tq, hq, d = q.shape
+    tk, hkv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((hq, tq), device=q.device, dtype=torch.float32)
+    rc = library().attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+        cu_seqlens_q.numel() - 1, tq, tk, int(max_seqlen_q), int(max_seqlen_k), hq, hkv, d,
+        float(scale), int(bool(causal)), int(bool(return_lse)), _ptr(out),
+        _ptr(lse) if return_lse else None, _stream(q.device))
+    if rc != 0:
+        raise AttnError("attn_fwd", rc)
+    return out, (lse if return_lse else None)
+
+
+def bwd_workspace_size(batch, total_q, nheads_q, head_dim) -> int:
+    return int(library().attn_bwd_workspace_size(batch, total_q, nheads_q, head_dim))
+
+
+def attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+             *, scale=None, causal=False, dq=None, dk=None, dv=None, workspace=None):
+    """Backward pass; returns (dq, dk, dv) in the layouts of q, k, v."""
+    _check_cuda(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, dq, dk, dv, workspace)
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _check_layout(n, t, torch.bfloat16)
+    _check_layout("lse", lse, torch.float32)
+    tq, hq, d = q.shape
+    tk, hkv, _ = k.shape
+    batch = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = d ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_size(batch, tq, hq, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
+    rc = library().attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(cu_seqlens_q),
+        _ptr(cu_seqlens_k), batch, tq, tk, int(max_seqlen_q), int(max_seqlen_k), hq, hkv, d,
+        float(scale), int(bool(causal)), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(q.device))
+    if rc != 0:
+        raise AttnError("attn_bwd", rc)
+    return dq, dk, dv
+
+
+def last_device_error(stream=None):
+    """Synchronise the stream and read/clear the device error word."""
+    buf = ctypes.create_string_buffer(256)
+    s = ctypes.c_void_p(stream.cuda_stream) if stream is not None else \
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = library().attn_last_device_error(s, buf, 256)
+    return rc, buf.value.decode()
+
+
+class _Attention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, scale, causal):
+        out, lse = attn_fwd(q, k, v, cu_q, cu_k, max_q, max_k, scale=scale, causal=causal,
+                            return_lse=True)
+        ctx.save_for_backward(q, k, v, out, lse, cu_q, cu_k)
+        ctx.args = (max_q, max_k, scale, causal)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse, cu_q, cu_k = ctx.saved_tensors
+        max_q, max_k, scale, causal = ctx.args
+        dq, dk, dv = attn_bwd(q, k, v, out, lse, dout.contiguous(), cu_q, cu_k, max_q, max_k,
+                              scale=scale, causal=causal)
+        return dq, dk, dv, None, None, None, None, None, None
+
+
+def attention(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
+              scale=None, causal=False):
+    """Differentiable exact attention over packed variable-length segments."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    return _Attention.apply(q, k, v, cu_seqlens_q, cu_seqlens_k, int(max_seqlen_q),
+                            int(max_seqlen_k), float(scale), bool(causal))

@@ -1,0 +1,279 @@
+// api.cu -- the C ABI declared in include/attn.h: argument checks, TMA tensor
+// maps, kernel launches and the device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "bwd_kernels.cuh"
+#include "fwd_kernel.cuh"
+
+namespace attn {
+
+// One error word per device: kernels record a timed-out wait here.
+__device__ uint32_t g_device_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  std::once_flag once;
+  cudaError_t init_status = cudaSuccess;
+  uint32_t* err = nullptr;
+  int sm_major = 0, sm_minor = 0;
+  int smem_optin = 0;
+};
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+uint64_t wait_timeout_ns() {
+  static uint64_t v = [] {
+    const char* e = std::getenv("ATTN_WAIT_TIMEOUT_MS");
+    long ms = e ? std::atol(e) : 2000;
+    if (ms <= 0) ms = 2000;
+    return static_cast<uint64_t>(ms) * 1000000ull;
+  }();
+  return v;
+}
+
+// Per-device set-up, once: the error word's device address and the device's
+// compute capability.
+DeviceState* device_state(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceState& st = g_dev[dev];
+  std::call_once(st.once, [&st, dev] {
+    st.init_status = cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err), g_device_error);
+    if (st.init_status != cudaSuccess) return;
+    cudaDeviceGetAttribute(&st.sm_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&st.sm_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&st.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  });
+  if (st.init_status != cudaSuccess) return nullptr;
+  *dev_out = dev;
+  return &st;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// bf16 [rows][heads][D] viewed as a 3-D tensor (D, heads, rows); box of
+// 64 columns x 1 head x box_rows rows, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* ptr, int rows, int heads, int d, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(heads) * d * 2};
+  const cuuint32_t box[3] = {64u, 1u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+attn_status_t check_common(const void* q, const void* k, const void* v,
+                           const int32_t* cu_q, const int32_t* cu_k, int32_t batch,
+                           int32_t total_q, int32_t total_k, int32_t max_q, int32_t max_k,
+                           int32_t hq, int32_t hkv, int32_t d, float scale) {
+  if (!q || !k || !v || !cu_q || !cu_k) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return ATTN_ERR_INVALID_ARG;
+  if (batch < 1 || total_q < 0 || total_k < 0 || max_q < 0 || max_k < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (hq < 1 || hkv < 1 || hq % hkv != 0 || hq > 65535) return ATTN_ERR_INVALID_ARG;
+  if (batch > 65535) return ATTN_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  // index arithmetic inside the kernels is 32-bit per row offset
+  if (static_cast<int64_t>(total_q) * hq * d >= (int64_t(1) << 40)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+template <int D, bool CAUSAL>
+attn_status_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const FwdParams& p, int batch, int hq, int max_q,
+                         cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  static std::once_flag attr_once[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once[dev], [&] {
+    attr_err = cudaFuncSetAttribute(attn_fwd_kernel<D, CAUSAL>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+  const int m_tiles = (max_q + C::BM * C::NQ - 1) / (C::BM * C::NQ);
+  if (m_tiles == 0) return ATTN_OK;
+  dim3 grid(m_tiles, hq, batch);
+  attn_fwd_kernel<D, CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" attn_status_t attn_fwd(const void* q, const void* k, const void* v,
+                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                  int32_t batch, int32_t total_q, int32_t total_k,
+                                  int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t nheads_q,
+                                  int32_t nheads_kv, int32_t head_dim, float scale,
+                                  int32_t causal, int32_t return_lse, void* out, float* lse,
+                                  attn_stream_t stream) {
+  attn_status_t st = check_common(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                  max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim,
+                                  scale);
+  if (st != ATTN_OK) return st;
+  if (!out || !aligned16(out)) return ATTN_ERR_INVALID_ARG;
+  if (return_lse && (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u))) return ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  DeviceState* ds = device_state(&dev);
+  if (!ds) return ATTN_ERR_CUDA;
+  if (ds->sm_major != 10) return ATTN_ERR_UNSUPPORTED;
+  if (total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+
+  FwdParams p;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.out = out;
+  p.lse = lse;
+  p.err = ds->err;
+  p.total_q = total_q;
+  p.nheads_q = nheads_q;
+  p.nheads_kv = nheads_kv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.return_lse = return_lse ? 1 : 0;
+  p.timeout_ns = wait_timeout_ns();
+
+  CUtensorMap mq, mk, mv;
+  const int vrows = 8192 / head_dim;
+  if (!make_map(&mq, q, total_q, nheads_q, head_dim, 128) ||
+      !make_map(&mk, k, total_k, nheads_kv, head_dim, 128) ||
+      !make_map(&mv, v, total_k, nheads_kv, head_dim, vrows))
+    return ATTN_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool c = causal != 0;
+  switch (head_dim) {
+    case 64:
+      return c ? launch_fwd<64, true>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s)
+               : launch_fwd<64, false>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s);
+    case 128:
+      return c ? launch_fwd<128, true>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s)
+               : launch_fwd<128, false>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s);
+    default:
+      return c ? launch_fwd<256, true>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s)
+               : launch_fwd<256, false>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s);
+  }
+}
+
+extern "C" size_t attn_bwd_workspace_size(int32_t batch, int32_t total_q, int32_t nheads_q,
+                                          int32_t head_dim) {
+  if (batch < 1 || total_q < 0 || nheads_q < 1 || head_dim < 1) return 0;
+  return bwd_workspace_bytes(batch, total_q, nheads_q, head_dim);
+}
+
+extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                                  const float* lse, const void* dout,
+                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                  int32_t batch, int32_t total_q, int32_t total_k,
+                                  int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t nheads_q,
+                                  int32_t nheads_kv, int32_t head_dim, float scale,
+                                  int32_t causal, void* dq, void* dk, void* dv, void* workspace,
+                                  size_t workspace_bytes, attn_stream_t stream) {
+  attn_status_t st = check_common(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                  max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim,
+                                  scale);
+  if (st != ATTN_OK) return st;
+  if (!out || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < bwd_workspace_bytes(batch, total_q, nheads_q, head_dim))
+    return ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  DeviceState* ds = device_state(&dev);
+  if (!ds) return ATTN_ERR_CUDA;
+  if (ds->sm_major != 10) return ATTN_ERR_UNSUPPORTED;
+  BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse; a.dout = dout;
+  a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k;
+  a.batch = batch; a.total_q = total_q; a.total_k = total_k;
+  a.max_q = max_seqlen_q; a.max_k = max_seqlen_k;
+  a.hq = nheads_q; a.hkv = nheads_kv; a.d = head_dim;
+  a.scale = scale; a.causal = causal != 0;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.workspace = workspace;
+  a.err = ds->err;
+  a.timeout_ns = wait_timeout_ns();
+  return bwd_launch(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" attn_status_t attn_last_device_error(attn_stream_t stream, char* msg,
+                                                size_t msg_len) {
+  auto put = [&](const char* m) {
+    if (msg && msg_len) {
+      std::strncpy(msg, m, msg_len - 1);
+      msg[msg_len - 1] = '\0';
+    }
+  };
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    put(cudaGetErrorString(e));
+    return ATTN_ERR_CUDA;
+  }
+  int dev = 0;
+  DeviceState* ds = device_state(&dev);
+  if (!ds) {
+    put("device set-up failed");
+    return ATTN_ERR_CUDA;
+  }
+  uint32_t word = 0;
+  const uint32_t zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) {
+    put("could not read the device error word");
+    return ATTN_ERR_CUDA;
+  }
+  if (word == 0) {
+    put("ok");
+    return ATTN_OK;
+  }
+  static const char* kernels[] = {"?", "fwd load", "fwd mma", "fwd softmax", "bwd preprocess",
+                                  "bwd load", "bwd mma", "bwd softmax", "bwd dq convert"};
+  const uint32_t kid = (word >> 8) & 0xff;
+  char buf[128];
+  std::snprintf(buf, sizeof(buf), "timed-out wait in %s (wait %u)",
+                kid < sizeof(kernels) / sizeof(kernels[0]) ? kernels[kid] : "?", word & 0xffu);
+  put(buf);
+  return ATTN_ERR_TIMEOUT;
+}
+
+extern "C" const char* attn_version(void) { return "exact_attention_b200 0.1 sm_100a"; }

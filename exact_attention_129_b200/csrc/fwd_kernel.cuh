@@ -1,0 +1,580 @@
+// fwd_kernel.cuh -- sm_100a forward kernel: tiled exact attention with an
+// online softmax, returning O and the per-row LSE.
+//
+// The FA4 repository guide describes the forward as "load Q tile -> loop over
+// K/V blocks (pipelined) -> online softmax accumulation -> store O and LSE",
+// with row max / row sum tracking, block-range skipping for causal masks and a
+// varlen-aware scheduler; the head_dim=256 regression check times it on B200
+// with softmax_scale = hdim**-0.5.  This file is our own design of that loop
+// for one B200 SM:
+//
+//   * One CTA owns NQ query tiles of 128 rows of one (segment, head): NQ = 2
+//     for head_dim 64/128 (both tiles share every K/V tile brought on chip),
+//     NQ = 1 for head_dim 256 (its 128 x 256 fp32 accumulator fills half of
+//     tensor memory).
+//   * Warp roles: 4*NQ softmax warps (one warpgroup per query tile; thread i of
+//     a warpgroup owns row i of its tile), one TMA producer warp, one MMA warp.
+//   * Tensor memory (512 columns): two 128-column S slots and the O
+//     accumulators.  With NQ = 2 each tile has its own S slot; with NQ = 1 the
+//     two slots double-buffer S across consecutive K/V blocks.  P (bf16) is
+//     written back over the first 64 columns of its S slot and read from there
+//     by the P.V MMA (A operand in tensor memory).
+//   * Shared memory: the Q tiles, then a ring of 16 KB chunks holding K and V
+//     tiles in the order the MMA warp consumes them.  A K tile is D/64 chunks
+//     (one per 64-column panel, K-major); a V tile is D/64 chunks of
+//     8192/D key rows each (all D columns, MN-major operand).  Every chunk is
+//     written by TMA with the 128-byte swizzle.
+//   * Online softmax in the log2 domain: x = s * scale * log2(e), p = 2^(x - m).
+//     The running max m is only raised when a row's max grows by more than 8
+//     (a factor 256); until then p may exceed 1 by at most that factor, which
+//     fp32 sums and bf16 P absorb.  O is rescaled in tensor memory only when a
+//     warp has such a row.  The result is exact: O = sum p v / sum p and
+//     LSE = (m + log2 sum p) * ln 2 hold for any m.
+//   * Causal: a CTA visits only key blocks that hold an allowed key for one of
+//     its rows; element masks are applied only in blocks that cross the
+//     diagonal or the end of the segment.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace attn {
+
+// device error word codes (kernel id << 8 | wait id)
+enum : uint32_t {
+  ERR_FWD_LOAD = 0x0100,
+  ERR_FWD_MMA = 0x0200,
+  ERR_FWD_SOFTMAX = 0x0300,
+};
+
+struct FwdParams {
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  void* out;        // bf16 [Tq][Hq][D]
+  float* lse;       // fp32 [Hq][Tq] or null
+  uint32_t* err;    // device error word
+  int total_q;
+  int nheads_q;
+  int nheads_kv;
+  float scale_log2;  // scale * log2(e)
+  int return_lse;
+  uint64_t timeout_ns;
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128;               // rows per query tile
+  static constexpr int BN = 128;               // keys per block
+  static constexpr int NQ = (D == 256) ? 1 : 2;
+  static constexpr int PANELS = D / 64;        // 64-column (128-byte) panels per row
+  static constexpr int CHUNK = 16384;          // ring slot bytes
+  static constexpr int VROWS = 8192 / D;       // V key rows per chunk
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int NSLOT = (D == 64) ? 12 : 10;
+  static constexpr int SOFTMAX_WARPS = 4 * NQ;
+  static constexpr int LOAD_WARP = SOFTMAX_WARPS;
+  static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
+  static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 2);
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int O_COL0 = 256;
+  // shared memory map (offsets from a 1024-aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + NSLOT * CHUNK;
+  // barriers: q_full[NQ] kv_full[NSLOT] kv_empty[NSLOT] s_full[2] p_full[2] o_ready[NQ]
+  static constexpr int NBAR = NQ + 2 * NSLOT + 2 + 2 + NQ;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+  static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, false, false);
+  static constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct FwdSmem {
+  uint8_t* q;
+  uint8_t* ring;
+  uint64_t* q_full;
+  uint64_t* kv_full;
+  uint64_t* kv_empty;
+  uint64_t* s_full;
+  uint64_t* p_full;
+  uint64_t* o_ready;
+  uint32_t* tmem_base;
+  volatile int* abort;
+};
+
+template <int D>
+__device__ __forceinline__ FwdSmem fwd_smem(uint8_t* base) {
+  using C = FwdCfg<D>;
+  FwdSmem s;
+  s.q = base + C::OFF_Q;
+  s.ring = base + C::OFF_RING;
+  uint64_t* b = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
+  s.q_full = b;
+  s.kv_full = b + C::NQ;
+  s.kv_empty = s.kv_full + C::NSLOT;
+  s.s_full = s.kv_empty + C::NSLOT;
+  s.p_full = s.s_full + 2;
+  s.o_ready = s.p_full + 2;
+  s.tmem_base = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
+  s.abort = reinterpret_cast<volatile int*>(base + C::OFF_MISC + 4);
+  return s;
+}
+
+// Number of key blocks a CTA visits and the rows it covers.
+struct FwdTile {
+  int q0, sq, k0, sk;   // segment offsets / lengths
+  int m_base;           // first segment-local row of the CTA
+  int n_blocks;         // key blocks to visit
+  int h, hk;
+};
+
+template <int D, bool CAUSAL>
+__device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t) {
+  using C = FwdCfg<D>;
+  const int b = blockIdx.z;
+  t.h = blockIdx.y;
+  t.hk = t.h / (p.nheads_q / p.nheads_kv);
+  t.q0 = p.cu_q[b];
+  t.sq = p.cu_q[b + 1] - t.q0;
+  t.k0 = p.cu_k[b];
+  t.sk = p.cu_k[b + 1] - t.k0;
+  // causal: heaviest tiles (bottom of the segment) first
+  const int m_tile = CAUSAL ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
+  t.m_base = m_tile * C::BM * C::NQ;
+  if (t.m_base >= t.sq) return false;
+  int n_end = t.sk;
+  if (CAUSAL) {
+    const int last_row = min(t.sq, t.m_base + C::BM * C::NQ) - 1;
+    n_end = min(t.sk, last_row + (t.sk - t.sq) + 1);
+  }
+  t.n_blocks = n_end > 0 ? (n_end + C::BN - 1) / C::BN : 0;
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// producer warp: Q once, then K/V chunks in MMA consumption order
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, const FwdSmem& s,
+                                         const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                                         const CUtensorMap* tmV) {
+  using C = FwdCfg<D>;
+  if (t.n_blocks == 0) return;  // nothing to attend to: no copy may outlive the CTA
+  for (int qt = 0; qt < C::NQ; ++qt) {
+    if (t.m_base + qt * C::BM >= t.sq) break;
+    mbar_expect_tx(&s.q_full[qt], C::Q_BYTES);
+    for (int pn = 0; pn < C::PANELS; ++pn)
+      tma_load_3d(s.q + qt * C::Q_BYTES + pn * C::CHUNK, tmQ, &s.q_full[qt], pn * 64, t.h,
+                  t.q0 + t.m_base + qt * C::BM);
+  }
+  uint32_t ring = 0;
+  // one K or V tile = PANELS chunks
+  auto load_tile = [&](bool is_v, int j) -> bool {
+    for (int c = 0; c < C::PANELS; ++c, ++ring) {
+      const uint32_t slot = ring % C::NSLOT;
+      if (ring >= (uint32_t)C::NSLOT) {
+        if (!mbar_wait(&s.kv_empty[slot], ((ring / C::NSLOT) - 1) & 1, s.abort, p.err,
+                       ERR_FWD_LOAD | 1, p.timeout_ns))
+          return false;
+      }
+      uint8_t* dst = s.ring + slot * C::CHUNK;
+      mbar_expect_tx(&s.kv_full[slot], C::CHUNK);
+      const int row = t.k0 + j * C::BN;
+      if (!is_v) {
+        tma_load_3d(dst, tmK, &s.kv_full[slot], c * 64, t.hk, row);
+      } else {
+        for (int pn = 0; pn < C::PANELS; ++pn)
+          tma_load_3d(dst + pn * (C::VROWS * 128), tmV, &s.kv_full[slot], pn * 64, t.hk,
+                      row + c * C::VROWS);
+      }
+    }
+    return true;
+  };
+  const int n = t.n_blocks;
+  if (C::NQ == 2) {
+    for (int j = 0; j < n; ++j) {
+      if (!load_tile(false, j)) return;
+      if (!load_tile(true, j)) return;
+    }
+  } else {
+    if (n > 0 && !load_tile(false, 0)) return;
+    for (int j = 0; j < n; ++j) {
+      if (j + 1 < n && !load_tile(false, j + 1)) return;
+      if (!load_tile(true, j)) return;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// MMA warp (one thread issues)
+// ---------------------------------------------------------------------------
+template <int D>
+struct FwdMma {
+  using C = FwdCfg<D>;
+  const FwdParams& p;
+  const FwdSmem& s;
+  uint32_t tmem;
+  uint32_t ring = 0;
+
+  __device__ FwdMma(const FwdParams& p_, const FwdSmem& s_, uint32_t tmem_)
+      : p(p_), s(s_), tmem(tmem_) {}
+
+  __device__ uint32_t take() {
+    const uint32_t b = ring;
+    ring += C::PANELS;
+    return b;
+  }
+  __device__ bool wait_tile(uint32_t base) {
+    for (int c = 0; c < C::PANELS; ++c) {
+      const uint32_t r = base + c;
+      if (!mbar_wait(&s.kv_full[r % C::NSLOT], (r / C::NSLOT) & 1, s.abort, p.err,
+                     ERR_FWD_MMA | 1, p.timeout_ns))
+        return false;
+    }
+    tc_fence_after();
+    return true;
+  }
+  __device__ void release_tile(uint32_t base) {
+    for (int c = 0; c < C::PANELS; ++c) mma_commit(&s.kv_empty[(base + c) % C::NSLOT]);
+  }
+  // S[slot] = Q[qt] . K^T
+  __device__ void issue_s(int qt, int slot, uint32_t kbase) {
+    const uint32_t d_tmem = tmem + slot * 128;
+    const uint32_t qaddr = smem_u32(s.q + qt * C::Q_BYTES);
+#pragma unroll
+    for (int c = 0; c < C::PANELS; ++c) {
+      const uint32_t kaddr = smem_u32(s.ring + ((kbase + c) % C::NSLOT) * C::CHUNK);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = sdesc_sw128(qaddr + c * C::CHUNK + kk * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
+        mma_ss(d_tmem, ad, bd, C::IDESC_S, (c | kk) != 0);
+      }
+    }
+  }
+  // O[qt] (+)= P[slot] . V
+  __device__ void issue_pv(int qt, int slot, uint32_t vbase, bool accumulate) {
+    const uint32_t d_tmem = tmem + C::O_COL0 + qt * D;
+    const uint32_t p_tmem = tmem + slot * 128;
+#pragma unroll
+    for (int c = 0; c < C::PANELS; ++c) {
+      const uint32_t vaddr = smem_u32(s.ring + ((vbase + c) % C::NSLOT) * C::CHUNK);
+#pragma unroll
+      for (int kk = 0; kk < C::VROWS / 16; ++kk) {
+        const int kstep = c * (C::VROWS / 16) + kk;  // 16 keys per step
+        const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, C::VROWS * 128, 1024);
+        mma_ts(d_tmem, p_tmem + kstep * 8, bd, C::IDESC_O, (accumulate || kstep) ? 1u : 0u);
+      }
+    }
+  }
+};
+
+template <int D>
+__device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, const FwdSmem& s,
+                                        uint32_t tmem) {
+  using C = FwdCfg<D>;
+  FwdMma<D> m(p, s, tmem);
+  const int n = t.n_blocks;
+  if (n == 0) return;
+  int nq = 0;
+  for (int qt = 0; qt < C::NQ; ++qt)
+    if (t.m_base + qt * C::BM < t.sq) nq = qt + 1;
+  for (int qt = 0; qt < nq; ++qt)
+    if (!mbar_wait(&s.q_full[qt], 0, s.abort, p.err, ERR_FWD_MMA | 2, p.timeout_ns)) return;
+  tc_fence_after();
+
+  if (C::NQ == 2) {
+    uint32_t kb = m.take();
+    if (!m.wait_tile(kb)) return;
+    for (int qt = 0; qt < nq; ++qt) {
+      m.issue_s(qt, qt, kb);
+      mma_commit(&s.s_full[qt]);
+    }
+    m.release_tile(kb);
+    for (int j = 1; j <= n; ++j) {
+      const uint32_t vb = m.take();  // V_{j-1}
+      const bool more = j < n;
+      if (more) kb = m.take();       // K_j
+      for (int qt = 0; qt < nq; ++qt) {
+        if (!mbar_wait(&s.p_full[qt], (j - 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
+                       p.timeout_ns))
+          return;
+        tc_fence_after();
+        if (qt == 0 && !m.wait_tile(vb)) return;
+        m.issue_pv(qt, qt, vb, j > 1);
+        mma_commit(&s.o_ready[qt]);
+        if (more) {
+          if (qt == 0 && !m.wait_tile(kb)) return;
+          m.issue_s(qt, qt, kb);
+          mma_commit(&s.s_full[qt]);
+        }
+      }
+      m.release_tile(vb);
+      if (more) m.release_tile(kb);
+    }
+  } else {
+    uint32_t kb = m.take();
+    if (!m.wait_tile(kb)) return;
+    m.issue_s(0, 0, kb);
+    mma_commit(&s.s_full[0]);
+    m.release_tile(kb);
+    if (n > 1) {
+      kb = m.take();
+      if (!m.wait_tile(kb)) return;
+      m.issue_s(0, 1, kb);
+      mma_commit(&s.s_full[1]);
+      m.release_tile(kb);
+    }
+    for (int j = 0; j < n; ++j) {
+      const int slot = j & 1;
+      const uint32_t vb = m.take();
+      if (!mbar_wait(&s.p_full[slot], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
+                     p.timeout_ns))
+        return;
+      tc_fence_after();
+      if (!m.wait_tile(vb)) return;
+      m.issue_pv(0, slot, vb, j > 0);
+      mma_commit(&s.o_ready[0]);
+      m.release_tile(vb);
+      if (j + 2 < n) {
+        kb = m.take();
+        if (!m.wait_tile(kb)) return;
+        m.issue_s(0, slot, kb);
+        mma_commit(&s.s_full[slot]);
+        m.release_tile(kb);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// softmax warpgroup: one thread per query row
+// ---------------------------------------------------------------------------
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t,
+                                            const FwdSmem& s, uint32_t tmem, int qt) {
+  using C = FwdCfg<D>;
+  const int warp = (threadIdx.x >> 5) & 3;  // warp within the warpgroup = TMEM lane quadrant
+  const int lane = lane_id();
+  const int row_in_tile = warp * 32 + lane;
+  const int row = t.m_base + qt * C::BM + row_in_tile;  // segment-local query row
+  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const int n = t.n_blocks;
+  const float c = p.scale_log2;
+  // keys [0, key_lim) are allowed for this row
+  const int key_lim = CAUSAL ? min(t.sk, row + (t.sk - t.sq) + 1) : t.sk;
+  // block j needs element masks for this warpgroup when it crosses the causal
+  // diagonal of the tile's first row or the end of the keys
+  const int tile_row0 = t.m_base + qt * C::BM;
+  const int mask_from = CAUSAL ? min(t.sk, tile_row0 + (t.sk - t.sq) + 1) : t.sk;
+
+  float m_run = -INFINITY;  // running max, log2 domain
+  float l_run = 0.f;
+  bool ok = true;
+
+  for (int j = 0; j < n; ++j) {
+    const int slot = (C::NQ == 2) ? qt : (j & 1);
+    const uint32_t parity = (C::NQ == 2) ? (j & 1) : ((j >> 1) & 1);
+    if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], parity, s.abort, p.err,
+                                           ERR_FWD_SOFTMAX | 1, p.timeout_ns))) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    const uint32_t s_addr = tmem + lane_base + slot * 128;
+    float sv[128];
+    {
+      uint32_t r[32];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        tmem_ld32(s_addr + cc * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = __uint_as_float(r[i]);
+      }
+    }
+    if ((j + 1) * C::BN > mask_from) {
+      const int lim = key_lim - j * C::BN;
+#pragma unroll
+      for (int i = 0; i < 128; ++i)
+        if (i >= lim) sv[i] = -INFINITY;
+    }
+    float mx = sv[0];
+#pragma unroll
+    for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
+    const float m_new = fmaxf(m_run, mx * c);
+    bool rescale = false;
+    float alpha = 1.f;
+    if (j == 0) {
+      m_run = m_new;
+    } else if (m_new - m_run > 8.f) {
+      alpha = ex2(m_run - m_new);
+      rescale = true;
+      m_run = m_new;
+      l_run *= alpha;
+    }
+    const float m_sub = (m_run == -INFINITY) ? 0.f : m_run;
+    // P = 2^(s*c - m), rounded to bf16 and written over the first 64 columns of S
+    float lsum = 0.f;
+    {
+      uint32_t pk[32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2(fmaf(sv[half * 64 + 2 * i], c, -m_sub));
+          const float p1 = ex2(fmaf(sv[half * 64 + 2 * i + 1], c, -m_sub));
+          lsum += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        tmem_st32(s_addr + half * 32, pk);
+      }
+    }
+    l_run += lsum;
+    if (__any_sync(0xffffffffu, rescale)) {
+      // O must not be rescaled while the previous P.V MMA may still write it
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (j - 1) & 1, s.abort, p.err,
+                                             ERR_FWD_SOFTMAX | 2, p.timeout_ns))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t o_addr = tmem + lane_base + C::O_COL0 + qt * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(o_addr + cc * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+        tmem_st32(o_addr + cc * 32, r);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(&s.p_full[slot]);
+  }
+
+  // ---- epilogue: O / l -> bf16, staged through this tile's Q buffer ----
+  const bool row_valid = row < t.sq;
+  const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+  uint8_t* stage = s.q + qt * C::Q_BYTES;
+  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  if (ok && n > 0) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (n - 1) & 1, s.abort, p.err,
+                                           ERR_FWD_SOFTMAX | 3, p.timeout_ns)))
+      ok = false;
+  }
+  if (ok) {
+    tc_fence_after();
+    const uint32_t o_addr = tmem + lane_base + C::O_COL0 + qt * D;
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t r[32];
+      if (n > 0) {
+        tmem_ld32(o_addr + cc * 32, r);
+        tmem_ld_wait(r);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = 0u;
+      }
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {  // 4 chunks of 8 columns
+        uint4 v;
+        v.x = pack_bf16(__uint_as_float(r[g * 8 + 0]) * inv_l, __uint_as_float(r[g * 8 + 1]) * inv_l);
+        v.y = pack_bf16(__uint_as_float(r[g * 8 + 2]) * inv_l, __uint_as_float(r[g * 8 + 3]) * inv_l);
+        v.z = pack_bf16(__uint_as_float(r[g * 8 + 4]) * inv_l, __uint_as_float(r[g * 8 + 5]) * inv_l);
+        v.w = pack_bf16(__uint_as_float(r[g * 8 + 6]) * inv_l, __uint_as_float(r[g * 8 + 7]) * inv_l);
+        const int chunk = cc * 4 + g;
+        *reinterpret_cast<uint4*>(stage + row_in_tile * (D * 2) +
+                                  ((chunk ^ (row_in_tile & 7)) * 16)) = v;
+      }
+    }
+  }
+  named_bar_sync(1 + qt, 128);
+  if (ok) {
+    const int rows_left = t.sq - tile_row0;
+    uint8_t* out = static_cast<uint8_t*>(p.out);
+    const int tid = threadIdx.x & 127;
+#pragma unroll 4
+    for (int q = tid; q < C::BM * CPR; q += 128) {
+      const int r = q / CPR, ch = q % CPR;
+      if (r < rows_left) {
+        const uint4 v =
+            *reinterpret_cast<const uint4*>(stage + r * (D * 2) + ((ch ^ (r & 7)) * 16));
+        const size_t grow = static_cast<size_t>(t.q0 + tile_row0 + r);
+        *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + t.h) * D) * 2 + ch * 16) = v;
+      }
+    }
+    if (p.return_lse && row_valid) {
+      const float lse =
+          (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+      p.lse[static_cast<size_t>(t.h) * p.total_q + t.q0 + row] = lse;
+    }
+  }
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  FwdTile t;
+  if (!fwd_tile<D, CAUSAL>(p, t)) return;  // uniform across the CTA
+  const FwdSmem s = fwd_smem<D>(base);
+  const int warp = threadIdx.x >> 5;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NQ; ++i) mbar_init(&s.q_full[i], 1);
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(&s.kv_full[i], 1);
+      mbar_init(&s.kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.s_full[i], 1);
+      mbar_init(&s.p_full[i], 128);
+    }
+    for (int i = 0; i < C::NQ; ++i) mbar_init(&s.o_ready[i], 1);
+    *s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::LOAD_WARP && lane_id() == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(s.tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s.tmem_base;
+
+  if (warp < C::SOFTMAX_WARPS) {
+    const int qt = warp / 4;
+    if (t.m_base + qt * C::BM < t.sq) fwd_softmax<D, CAUSAL>(p, t, s, tmem, qt);
+  } else if (warp == C::LOAD_WARP) {
+    if (lane_id() == 0) fwd_load<D>(p, t, s, &tmQ, &tmK, &tmV);
+  } else if (warp == C::MMA_WARP) {
+    if (lane_id() == 0) fwd_mma<D>(p, t, s, tmem);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

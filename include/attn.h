@@ -1,0 +1,155 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact-attention library (libattn.so).
+ *
+ * The library computes exact scaled-dot-product attention in bf16 with fp32
+ * accumulation:
+ *
+ *   forward   O = softmax(scale * Q K^T + mask) V   and the per-row
+ *             log-sum-exp LSE_i = log sum_j exp(scale * q_i . k_j) over the
+ *             allowed keys j (natural log of the scaled scores),
+ *   backward  dQ, dK, dV of a loss L given dO = dL/dO, with P recomputed
+ *             from the LSE.
+ *
+ * This is the operation the attention pages benchmark: the cosmos-framework
+ * issue #118 calls it through a varlen frontend (cu_seqlens, max_seqlen,
+ * 32 query / 8 key-value heads, head_dim 128); the flash-attention issue #2729
+ * repro calls the forward with out=, lse= and return_lse= and checks it against
+ * torch's scaled_dot_product_attention; the FA4 head_dim=256 regression check
+ * times forward and backward with softmax_scale = hdim**-0.5, MHA and GQA
+ * (nheads_kv = 1), causal and not; the FA4 repository guide describes the
+ * forward as "load Q tile -> loop over K/V blocks -> online softmax -> store O
+ * and LSE" and the backward as a preprocess, a main kernel and a postprocess.
+ *
+ * Layouts (row-major, last index fastest, every pointer DEVICE memory):
+ *   q, out, dout, dq : bf16  [total_q][nheads_q][head_dim]
+ *   k, v, dk, dv     : bf16  [total_k][nheads_kv][head_dim]
+ *   lse              : fp32  [nheads_q][total_q]
+ *   cu_seqlens_q/_k  : int32 [batch + 1], cu[0] = 0, non-decreasing,
+ *                      cu_q[batch] = total_q, cu_k[batch] = total_k.
+ * Segment b holds query rows [cu_q[b], cu_q[b+1]) and key rows
+ * [cu_k[b], cu_k[b+1]); a dense (batch, seqlen) tensor is the packed case with
+ * cu = {0, S, 2S, ...} and needs no copy.  A segment may be empty.
+ *
+ * Heads: query head h reads key/value head h / (nheads_q / nheads_kv)
+ * (contiguous groups; nheads_q must be a multiple of nheads_kv).  MHA is
+ * nheads_kv = nheads_q, MQA is nheads_kv = 1.
+ *
+ * Causal masking is bottom-right aligned: query row i of a segment may see key
+ * j iff j <= i + (s_k - s_q).  A query row that sees no key gets O = 0,
+ * LSE = -inf and contributes nothing to any gradient.
+ *
+ * head_dim is 64, 128 or 256.  scale must be finite and > 0 (the pages use
+ * head_dim^-0.5).  Every base pointer must be 16-byte aligned.
+ *
+ * Ownership: the caller allocates every buffer, including the workspace the
+ * backward needs.  The library allocates no device memory, keeps no state
+ * between calls except one device error word per device, and never
+ * synchronises the stream except in attn_last_device_error.  All work is
+ * enqueued on `stream` (0 = legacy default stream).
+ *
+ * Errors: arguments are checked on the host before anything is launched;
+ * a bad argument returns ATTN_ERR_INVALID_ARG (or ATTN_ERR_UNSUPPORTED for a
+ * head_dim or device the library has no kernel for) and launches nothing.
+ * A failed launch returns ATTN_ERR_CUDA.  Every wait inside a kernel is
+ * bounded; if one runs out, the kernel records it in the device error word and
+ * exits without trapping, and attn_last_device_error reports ATTN_ERR_TIMEOUT.
+ * The contents of cu_seqlens are not checked on the device: they must satisfy
+ * the conditions above and max_seqlen_q/k must bound every segment length.
+ */
+#ifndef EXACT_ATTENTION_B200_ATTN_H
+#define EXACT_ATTENTION_B200_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* attn_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,
+  ATTN_ERR_UNSUPPORTED = 2,
+  ATTN_ERR_CUDA = 3,
+  ATTN_ERR_TIMEOUT = 4
+} attn_status_t;
+
+/*
+ * Forward pass (the FA4 guide's "load Q tile -> loop over K/V blocks
+ * (pipelined) -> online softmax accumulation -> store O and LSE"; issue #2729's
+ * _flash_attn_fwd(q, k, v, out=, lse=, return_lse=)).
+ *
+ *   q, k, v        inputs, layouts above (read only).
+ *   cu_seqlens_q/k device int32 [batch+1].
+ *   batch          number of segments, >= 1.
+ *   total_q        rows of q/out (= cu_q[batch]); sizes the LSE rows.
+ *   total_k        rows of k/v  (= cu_k[batch]).
+ *   max_seqlen_q/k upper bounds of the segment lengths (>= 0).
+ *   nheads_q, nheads_kv, head_dim, scale, causal  as described above.
+ *   return_lse     0: lse is not written (may be NULL); 1: lse must be valid.
+ *   out            bf16 [total_q][nheads_q][head_dim], written.
+ *   lse            fp32 [nheads_q][total_q], written iff return_lse.
+ *   stream         CUDA stream.
+ * Returns ATTN_OK once the kernel is enqueued.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v,
+                       const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                       int32_t batch, int32_t total_q, int32_t total_k,
+                       int32_t max_seqlen_q, int32_t max_seqlen_k,
+                       int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                       float scale, int32_t causal, int32_t return_lse,
+                       void* out, float* lse, attn_stream_t stream);
+
+/*
+ * Bytes of device workspace attn_bwd needs for these sizes (a pure function of
+ * its arguments; 0 for invalid sizes).  The workspace holds the fp32 dQ
+ * accumulator and the fp32 row-dot D_i = dO_i . O_i.
+ */
+size_t attn_bwd_workspace_size(int32_t batch, int32_t total_q, int32_t nheads_q,
+                               int32_t head_dim);
+
+/*
+ * Backward pass (the FA4 guide's backward: a preprocess kernel, the main
+ * kernel that recomputes P from the LSE, and a postprocess kernel).
+ *
+ *   q, k, v, out   as given to / produced by attn_fwd.
+ *   lse            fp32 [nheads_q][total_q] from attn_fwd(return_lse = 1).
+ *   dout           bf16 like out: the incoming gradient dL/dO.
+ *   dq             bf16 like q, written.
+ *   dk, dv         bf16 like k and v, written; for GQA each key/value head
+ *                  receives the sum over its group of query heads.
+ *   workspace      device memory of at least attn_bwd_workspace_size(...)
+ *                  bytes, 256-byte aligned; its contents on entry do not
+ *                  matter and are clobbered.
+ * Other arguments as for attn_fwd.  Calls that share a workspace must not
+ * overlap on the GPU.
+ */
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                       const float* lse, const void* dout,
+                       const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                       int32_t batch, int32_t total_q, int32_t total_k,
+                       int32_t max_seqlen_q, int32_t max_seqlen_k,
+                       int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                       float scale, int32_t causal,
+                       void* dq, void* dk, void* dv,
+                       void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word.  Returns ATTN_OK, ATTN_ERR_TIMEOUT (a bounded wait in a kernel ran out;
+ * `msg` names the kernel and the wait) or ATTN_ERR_CUDA (the stream reported
+ * an error).  `msg` (may be NULL) receives a NUL-terminated description of at
+ * most msg_len bytes.
+ */
+attn_status_t attn_last_device_error(attn_stream_t stream, char* msg, size_t msg_len);
+
+/* Library version string, e.g. "exact_attention_b200 0.1 sm_100a". */
+const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_B200_ATTN_H */

@@ -1,0 +1,93 @@
+"""CPU tests of the C ABI: the library loads, exports every declared symbol and
+rejects bad arguments on the host without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_129_b200 as ea
+from exact_attention_129_b200 import build as eab
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    eab.build()
+    return ea.library()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) >= {"attn_fwd", "attn_bwd", "attn_bwd_workspace_size",
+                          "attn_last_device_error", "attn_version"}
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version(lib):
+    assert b"sm_100a" in lib.attn_version()
+
+
+def _fwd(lib, **kw):
+    a = dict(q=16, k=16, v=16, cu_q=16, cu_k=16, batch=1, tq=128, tk=128, mq=128, mk=128,
+             hq=4, hkv=2, d=128, scale=0.088, causal=0, rl=1, out=16, lse=16)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return lib.attn_fwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["cu_q"]), vp(a["cu_k"]),
+                        a["batch"], a["tq"], a["tk"], a["mq"], a["mk"], a["hq"], a["hkv"],
+                        a["d"], a["scale"], a["causal"], a["rl"], vp(a["out"]),
+                        vp(a["lse"]), None)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(d=96), 2),            # head_dim without a kernel
+    (dict(d=32), 2),
+    (dict(hq=3, hkv=2), 1),     # heads not a multiple
+    (dict(q=8), 1),             # misaligned pointer
+    (dict(out=24), 1),
+    (dict(lse=0), 1),           # return_lse without an lse buffer
+    (dict(batch=0), 1),
+    (dict(q=0), 1),
+    (dict(scale=0.0), 1),
+    (dict(scale=-1.0), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(mq=-1), 1),
+])
+def test_fwd_rejects_bad_arguments_without_launching(lib, bad, code):
+    # every case fails in host validation, before any device call
+    assert _fwd(lib, **bad) == code
+
+
+def test_bwd_rejects_small_workspace(lib):
+    vp = ctypes.c_void_p
+    need = lib.attn_bwd_workspace_size(1, 128, 4, 128)
+    assert need > 0
+    rc = lib.attn_bwd(vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), 1, 128,
+                      128, 128, 128, 4, 2, 128, 0.088, 0, vp(16), vp(16), vp(16), vp(256),
+                      need - 1, None)
+    assert rc == 1
+    rc = lib.attn_bwd(vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), 1, 128,
+                      128, 128, 128, 4, 2, 128, 0.088, 0, vp(16), vp(16), vp(16), vp(100),
+                      need, None)
+    assert rc == 1  # workspace not 256-byte aligned
+
+
+def test_workspace_size_rejects_bad_sizes(lib):
+    assert lib.attn_bwd_workspace_size(0, 128, 4, 128) == 0
+    assert lib.attn_bwd_workspace_size(1, 128, 0, 128) == 0
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(4, 2, 64, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        ea.attn_fwd(q, q, q, cu, cu, 4, 4)
