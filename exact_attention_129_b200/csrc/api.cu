@@ -136,6 +136,84 @@ attn_status_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+template <int D, bool CAUSAL>
+attn_status_t launch_bwd_main(const BwdArgs& a, const BwdParams& bp, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  static std::once_flag attr_once[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once[dev], [&] {
+    attr_err = cudaFuncSetAttribute(attn_bwd_main_kernel<D, CAUSAL>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+  CUtensorMap mk, mv, mq, mo;
+  if (!make_map(&mk, a.k, a.total_k, a.hkv, D, 128) ||
+      !make_map(&mv, a.v, a.total_k, a.hkv, D, 128) ||
+      !make_map(&mq, a.q, a.total_q, a.hq, D, C::BM) ||
+      !make_map(&mo, a.dout, a.total_q, a.hq, D, C::BM))
+    return ATTN_ERR_CUDA;
+  const int n_blocks = (a.max_k + C::BN - 1) / C::BN;
+  if (n_blocks == 0) return ATTN_OK;
+  dim3 grid(n_blocks * C::NSPLIT, a.hkv, a.batch);
+  attn_bwd_main_kernel<D, CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mk, mv, mq, mo, bp);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D>
+attn_status_t bwd_launch_d(const BwdArgs& a, cudaStream_t stream) {
+  float* dq_acc = static_cast<float*>(a.workspace);
+  float* delta = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) +
+                                          bwd_align256(static_cast<size_t>(a.total_q) * a.hq * D * 4));
+  const long long n_rh = static_cast<long long>(a.total_q) * a.hq;
+  if (n_rh > 0) {
+    const long long threads = n_rh * (D / 8);
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+    attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
+        static_cast<const uint16_t*>(a.out), static_cast<const uint16_t*>(a.dout), delta, dq_acc,
+        a.total_q, a.hq);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  BwdParams bp;
+  bp.cu_q = a.cu_q;
+  bp.cu_k = a.cu_k;
+  bp.lse = a.lse;
+  bp.delta = delta;
+  bp.dq_acc = dq_acc;
+  bp.dk = a.dk;
+  bp.dv = a.dv;
+  bp.err = a.err;
+  bp.total_q = a.total_q;
+  bp.nheads_q = a.hq;
+  bp.nheads_kv = a.hkv;
+  bp.scale = a.scale;
+  bp.scale_log2 = a.scale * 1.4426950408889634f;
+  bp.timeout_ns = a.timeout_ns;
+  if (a.total_k > 0) {
+    attn_status_t st = a.causal ? launch_bwd_main<D, true>(a, bp, stream)
+                                : launch_bwd_main<D, false>(a, bp, stream);
+    if (st != ATTN_OK) return st;
+  }
+  if (n_rh > 0) {
+    const long long n8 = n_rh * D / 8;
+    long long blocks = (n8 + 255) / 256;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    attn_bwd_dq_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        dq_acc, static_cast<uint16_t*>(a.dq), n8, a.scale);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+attn_status_t bwd_launch(const BwdArgs& a, cudaStream_t stream) {
+  switch (a.d) {
+    case 64: return bwd_launch_d<64>(a, stream);
+    case 128: return bwd_launch_d<128>(a, stream);
+    default: return bwd_launch_d<256>(a, stream);
+  }
+}
+
 }  // namespace
 }  // namespace attn
 

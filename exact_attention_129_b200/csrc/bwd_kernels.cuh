@@ -1,12 +1,46 @@
-// bwd_kernels.cuh -- backward pass (placeholder until the kernels land).
+// bwd_kernels.cuh -- sm_100a backward pass: dQ, dK, dV of exact attention,
+// recomputing P from the forward's LSE.
+//
+// The FA4 repository guide splits its backward into a preprocess kernel, a main
+// kernel and a postprocess kernel; the plainest reading of that split (and of
+// the method: P = exp(S - LSE), dS = P * (dP - D), D_i = dO_i . O_i) is:
+//
+//   1. preprocess: D_i = sum_d dO_id O_id (fp32) and a zeroed fp32 dQ accumulator;
+//   2. main: per key block, loop over the query blocks (and, for GQA, over the
+//      query heads of the group) recomputing S^T = K Q^T and dP^T = V dO^T with
+//      tcgen05 MMAs, forming P^T and dS^T elementwise, accumulating dV += P^T dO
+//      and dK += dS^T Q in tensor memory for the whole loop (so the GQA group sum
+//      costs nothing extra) and computing dQ^T = K^T dS^T per query block, which
+//      is added into the fp32 accumulator with coalesced reductions;
+//   3. postprocess: dQ = scale * accumulator, rounded to bf16.
+//
+// Main-kernel layout for one CTA (128 keys; head_dim 256 is split into two
+// 128-wide halves handled by two CTAs, each recomputing S and dP in full):
+//   tensor memory: S^T x2 (64 cols each; P^T in bf16 is written back over the
+//                  first 32), dP^T (64), dQ^T (64), dV (DH), dK (DH)  = 512 cols
+//   shared memory: K and V tiles (resident), a ring of NST (Q, dO) stages of
+//                  64 query rows, two dS^T tiles (128 keys x 64 queries, bf16,
+//                  128-byte swizzled: the same bytes are the K-major A operand of
+//                  dK += dS^T Q and the MN-major B operand of dQ^T = K^T dS^T),
+//                  and per-block LSE/D vectors.
+//   warps: 4 elementwise warps (thread = key row = TMEM lane), 1 TMA warp,
+//          1 MMA warp.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
 #include "attn.h"
+#include "ptx.cuh"
 
 namespace attn {
+
+enum : uint32_t {
+  ERR_BWD_LOAD = 0x0500,
+  ERR_BWD_MMA = 0x0600,
+  ERR_BWD_ELEM = 0x0700,
+};
 
 struct BwdArgs {
   const void *q, *k, *v, *out, *dout;
@@ -20,11 +54,575 @@ struct BwdArgs {
   uint64_t timeout_ns;
 };
 
+// workspace: fp32 dQ accumulator [Tq][Hq][D], then fp32 D_i [Hq][Tq]
+inline size_t bwd_align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 inline size_t bwd_workspace_bytes(int batch, int total_q, int hq, int d) {
-  (void)batch; (void)total_q; (void)hq; (void)d;
-  return 256;
+  (void)batch;
+  const size_t rows = static_cast<size_t>(total_q > 0 ? total_q : 1);
+  return bwd_align256(rows * hq * d * 4) + bwd_align256(rows * hq * 4);
 }
 
-inline attn_status_t bwd_launch(const BwdArgs&, cudaStream_t) { return ATTN_ERR_UNSUPPORTED; }
+struct BwdParams {
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  const float* lse;    // [Hq][Tq]
+  const float* delta;  // [Hq][Tq]
+  float* dq_acc;       // [Tq][Hq][D]
+  void* dk;            // bf16 [Tk][Hkv][D]
+  void* dv;
+  uint32_t* err;
+  int total_q;
+  int nheads_q;
+  int nheads_kv;
+  float scale;
+  float scale_log2;
+  uint64_t timeout_ns;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int BN = 128;                 // keys per CTA
+  static constexpr int BM = 64;                  // query rows per iteration
+  static constexpr int DH = (D == 256) ? 128 : D;  // accumulator width per CTA
+  static constexpr int NSPLIT = D / DH;
+  static constexpr int PANELS = D / 64;
+  static constexpr int KV_PANEL = BN * 128;      // 16 KB: 128 rows x 64 cols
+  static constexpr int QD_PANEL = BM * 128;      // 8 KB: 64 rows x 64 cols
+  static constexpr int K_BYTES = PANELS * KV_PANEL + (D == 64 ? KV_PANEL : 0);  // + zero panel
+  static constexpr int V_BYTES = PANELS * KV_PANEL;
+  static constexpr int STAGE_BYTES = 2 * PANELS * QD_PANEL;  // Q_i then dO_i
+  static constexpr int NST = (D == 256) ? 1 : (D == 128 ? 3 : 4);
+  static constexpr int DS_BYTES = BN * BM * 2;   // 16 KB
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + K_BYTES;
+  static constexpr int OFF_ST = OFF_V + V_BYTES;
+  static constexpr int OFF_DS = OFF_ST + NST * STAGE_BYTES;
+  static constexpr int OFF_LSD = OFF_DS + 2 * DS_BYTES;      // NST x 128 floats
+  static constexpr int OFF_BAR = OFF_LSD + NST * 128 * 4;
+  // kv_full, qdo_full[NST], qdo_empty[NST], s_full[2], dp_full, dp_free,
+  // ds_ready[2], ds_free[2], dq_full, dq_free, dkv_full
+  static constexpr int NBAR = 1 + 2 * NST + 2 + 2 + 2 + 2 + 3;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static constexpr int THREADS = 192;
+  static constexpr int LOAD_WARP = 4, MMA_WARP = 5;
+  // tensor memory columns
+  static constexpr int COL_S = 0, COL_DP = 128, COL_DQ = 192, COL_DV = 256, COL_DK = 256 + DH;
+  static constexpr uint32_t IDESC_SDP = idesc_bf16(128, BM, false, false);
+  static constexpr uint32_t IDESC_KV = idesc_bf16(128, DH, false, true);
+  static constexpr uint32_t IDESC_DQ = idesc_bf16(128, BM, true, true);
+};
+
+struct BwdSmem {
+  uint8_t *k, *v, *st, *ds;
+  float* lsd;
+  uint64_t *kv_full, *qdo_full, *qdo_empty, *s_full, *dp_full, *dp_free, *ds_ready, *ds_free,
+      *dq_full, *dq_free, *dkv_full;
+  uint32_t* tmem_base;
+  volatile int* abort;
+};
+
+template <int D>
+__device__ __forceinline__ BwdSmem bwd_smem(uint8_t* base) {
+  using C = BwdCfg<D>;
+  BwdSmem s;
+  s.k = base + C::OFF_K;
+  s.v = base + C::OFF_V;
+  s.st = base + C::OFF_ST;
+  s.ds = base + C::OFF_DS;
+  s.lsd = reinterpret_cast<float*>(base + C::OFF_LSD);
+  uint64_t* b = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
+  s.kv_full = b;
+  s.qdo_full = b + 1;
+  s.qdo_empty = s.qdo_full + C::NST;
+  s.s_full = s.qdo_empty + C::NST;
+  s.dp_full = s.s_full + 2;
+  s.dp_free = s.dp_full + 1;
+  s.ds_ready = s.dp_free + 1;
+  s.ds_free = s.ds_ready + 2;
+  s.dq_full = s.ds_free + 2;
+  s.dq_free = s.dq_full + 1;
+  s.dkv_full = s.dq_free + 1;
+  s.tmem_base = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
+  s.abort = reinterpret_cast<volatile int*>(base + C::OFF_MISC + 4);
+  return s;
+}
+
+// The CTA's key block and the query blocks that can see it.
+struct BwdTile {
+  int q0, sq, k0, sk;
+  int n_base;   // first segment-local key row
+  int dh;       // accumulator half (head_dim 256) or 0
+  int hk;
+  int h0;       // first query head of the group
+  int G;        // query heads per key/value head
+  int m_lo, m_hi;  // query blocks [m_lo, m_hi) of BM rows
+  int n_iter;   // G * (m_hi - m_lo)
+};
+
+template <int D, bool CAUSAL>
+__device__ __forceinline__ bool bwd_tile(const BwdParams& p, BwdTile& t) {
+  using C = BwdCfg<D>;
+  const int b = blockIdx.z;
+  t.hk = blockIdx.y;
+  t.G = p.nheads_q / p.nheads_kv;
+  t.h0 = t.hk * t.G;
+  const int nb = blockIdx.x / C::NSPLIT;
+  t.dh = blockIdx.x % C::NSPLIT;
+  t.q0 = p.cu_q[b];
+  t.sq = p.cu_q[b + 1] - t.q0;
+  t.k0 = p.cu_k[b];
+  t.sk = p.cu_k[b + 1] - t.k0;
+  t.n_base = nb * C::BN;
+  if (t.n_base >= t.sk) return false;
+  t.m_hi = (t.sq + C::BM - 1) / C::BM;
+  t.m_lo = 0;
+  if (CAUSAL) {
+    // query row i sees key j iff j <= i + (sk - sq): the first row that sees
+    // this block's first key is n_base - (sk - sq)
+    const int first = t.n_base - (t.sk - t.sq);
+    t.m_lo = first > 0 ? first / C::BM : 0;
+  }
+  if (t.m_lo > t.m_hi) t.m_lo = t.m_hi;
+  t.n_iter = t.G * (t.m_hi - t.m_lo);
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// TMA warp
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void bwd_load(const BwdParams& p, const BwdTile& t, const BwdSmem& s,
+                                         const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                         const CUtensorMap* tmQ, const CUtensorMap* tmO) {
+  // all 32 lanes: lane 0 issues the copies, every lane fills part of the
+  // per-block LSE (log2 domain) and D_i vectors and arrives on qdo_full
+  using C = BwdCfg<D>;
+  if (t.n_iter == 0) return;
+  const int lane = lane_id();
+  if (lane == 0) {
+    mbar_expect_tx(s.kv_full, 2 * C::PANELS * C::KV_PANEL);
+    for (int pn = 0; pn < C::PANELS; ++pn) {
+      tma_load_3d(s.k + pn * C::KV_PANEL, tmK, s.kv_full, pn * 64, t.hk, t.k0 + t.n_base);
+      tma_load_3d(s.v + pn * C::KV_PANEL, tmV, s.kv_full, pn * 64, t.hk, t.k0 + t.n_base);
+    }
+  }
+  const int mcount = t.m_hi - t.m_lo;
+  int issued = 0;
+  for (int i = 0; i < t.n_iter; ++i) {
+    const int st = i % C::NST;
+    if (i >= C::NST) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.qdo_empty[st], ((i / C::NST) - 1) & 1, s.abort,
+                                             p.err, ERR_BWD_LOAD | 1, p.timeout_ns)))
+        break;
+    }
+    const int h = t.h0 + i / mcount;
+    const int m0 = (t.m_lo + i % mcount) * C::BM;
+    float* lsd = s.lsd + st * 128;
+#pragma unroll
+    for (int r = lane; r < C::BM; r += 32) {
+      const int qrow = m0 + r;
+      float l2 = INFINITY;  // rows outside the segment, or rows that saw no key: P = 0
+      float dl = 0.f;
+      if (qrow < t.sq) {
+        const size_t idx = static_cast<size_t>(h) * p.total_q + t.q0 + qrow;
+        const float l = p.lse[idx];
+        if (l != -INFINITY) l2 = l * 1.4426950408889634f;
+        dl = p.delta[idx];
+      }
+      lsd[r] = l2;
+      lsd[64 + r] = dl;
+    }
+    if (lane == 0) {
+      uint8_t* dst = s.st + st * C::STAGE_BYTES;
+      const int row = t.q0 + m0;
+      mbar_expect_tx(&s.qdo_full[st], C::STAGE_BYTES);
+      for (int pn = 0; pn < C::PANELS; ++pn) {
+        tma_load_3d(dst + pn * C::QD_PANEL, tmQ, &s.qdo_full[st], pn * 64, h, row);
+        tma_load_3d(dst + (C::PANELS + pn) * C::QD_PANEL, tmO, &s.qdo_full[st], pn * 64, h,
+                    row);
+      }
+    } else {
+      mbar_arrive(&s.qdo_full[st]);
+    }
+    ++issued;
+  }
+  if (*s.abort && lane == 0) {
+    // let this CTA's own copies land before its shared memory is released
+    mbar_wait_drain(s.kv_full, 0, 100000000ull);
+    for (int i = issued > C::NST ? issued - C::NST : 0; i < issued; ++i)
+      mbar_wait_drain(&s.qdo_full[i % C::NST], (i / C::NST) & 1, 100000000ull);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// MMA warp (one thread issues)
+// ---------------------------------------------------------------------------
+template <int D>
+struct BwdMma {
+  using C = BwdCfg<D>;
+  const BwdParams& p;
+  const BwdSmem& s;
+  const BwdTile& t;
+  uint32_t tmem;
+  __device__ BwdMma(const BwdParams& p_, const BwdSmem& s_, const BwdTile& t_, uint32_t tm)
+      : p(p_), s(s_), t(t_), tmem(tm) {}
+
+  __device__ bool wait(uint64_t* bar, uint32_t parity, uint32_t code) {
+    if (!mbar_wait(bar, parity, s.abort, p.err, ERR_BWD_MMA | code, p.timeout_ns)) return false;
+    tc_fence_after();
+    return true;
+  }
+  // X^T = A B^T with A = K or V (128 keys x D, K-major) and B = Q_i or dO_i (64 x D)
+  __device__ void issue_kt(uint32_t d_col, const uint8_t* a, const uint8_t* b) {
+    const uint32_t aa = smem_u32(a), ba = smem_u32(b);
+#pragma unroll
+    for (int pn = 0; pn < C::PANELS; ++pn)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tmem + d_col, sdesc_sw128(aa + pn * C::KV_PANEL + kk * 32, 16, 1024),
+               sdesc_sw128(ba + pn * C::QD_PANEL + kk * 32, 16, 1024), C::IDESC_SDP,
+               (pn | kk) != 0);
+  }
+  __device__ void grads(int j, bool first) {
+    const int bj = j & 1;
+    const uint8_t* stg = s.st + (j % C::NST) * C::STAGE_BYTES;
+    const uint32_t q_half = smem_u32(stg) + t.dh * 2 * C::QD_PANEL;
+    const uint32_t do_half = smem_u32(stg) + (C::PANELS + t.dh * 2) * C::QD_PANEL;
+    const uint32_t ds = smem_u32(s.ds + bj * C::DS_BYTES);
+    // dV += P^T dO  (A = P^T in tensor memory, B = dO rows, MN-major)
+#pragma unroll
+    for (int ks = 0; ks < C::BM / 16; ++ks)
+      mma_ts(tmem + C::COL_DV, tmem + C::COL_S + bj * 64 + ks * 8,
+             sdesc_sw128(do_half + ks * 2048, C::QD_PANEL, 1024), C::IDESC_KV,
+             (!first || ks) ? 1u : 0u);
+    // dK += dS^T Q  (A = dS^T K-major in shared memory)
+#pragma unroll
+    for (int ks = 0; ks < C::BM / 16; ++ks)
+      mma_ss(tmem + C::COL_DK, sdesc_sw128(ds + ks * 32, 16, 1024),
+             sdesc_sw128(q_half + ks * 2048, C::QD_PANEL, 1024), C::IDESC_KV,
+             (!first || ks) ? 1u : 0u);
+  }
+  __device__ void dq(int j) {
+    const int bj = j & 1;
+    const uint32_t ka = smem_u32(s.k) + t.dh * 2 * C::KV_PANEL;
+    const uint32_t ds = smem_u32(s.ds + bj * C::DS_BYTES);
+    // dQ^T = K^T dS^T  (A = K tile read MN-major, B = dS^T MN-major)
+#pragma unroll
+    for (int ks = 0; ks < C::BN / 16; ++ks)
+      mma_ss(tmem + C::COL_DQ, sdesc_sw128(ka + ks * 2048, C::KV_PANEL, 1024),
+             sdesc_sw128(ds + ks * 2048, C::QD_PANEL, 1024), C::IDESC_DQ, ks ? 1u : 0u);
+  }
+};
+
+template <int D>
+__device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, const BwdSmem& s,
+                                        uint32_t tmem) {
+  using C = BwdCfg<D>;
+  if (t.n_iter == 0) return;
+  BwdMma<D> m(p, s, t, tmem);
+  if (!m.wait(s.kv_full, 0, 1)) return;
+  auto do_grads = [&](int j) -> bool {
+    if (!m.wait(&s.ds_ready[j & 1], (j >> 1) & 1, 2)) return false;
+    m.grads(j, j == 0);
+    if (j >= 1 && !m.wait(s.dq_free, (j - 1) & 1, 3)) return false;
+    m.dq(j);
+    mma_commit(s.dq_full);
+    mma_commit(&s.qdo_empty[j % C::NST]);
+    mma_commit(&s.ds_free[j & 1]);
+    return true;
+  };
+  for (int i = 0; i < t.n_iter; ++i) {
+    const int st = i % C::NST;
+    // with a single (Q, dO) stage, block i can only be loaded once block i-1's
+    // gradient MMAs have released it
+    if (C::NST == 1 && i >= 1 && !do_grads(i - 1)) return;
+    if (!m.wait(&s.qdo_full[st], (i / C::NST) & 1, 4)) return;
+    const uint8_t* stg = s.st + st * C::STAGE_BYTES;
+    m.issue_kt(C::COL_S + (i & 1) * 64, s.k, stg);
+    mma_commit(&s.s_full[i & 1]);
+    if (i >= 1 && !m.wait(s.dp_free, (i - 1) & 1, 5)) return;
+    m.issue_kt(C::COL_DP, s.v, stg + C::PANELS * C::QD_PANEL);
+    mma_commit(s.dp_full);
+    if (C::NST > 1 && i >= 1 && !do_grads(i - 1)) return;
+  }
+  if (!do_grads(t.n_iter - 1)) return;
+  mma_commit(s.dkv_full);
+}
+
+// ---------------------------------------------------------------------------
+// elementwise warps: thread = key row
+// ---------------------------------------------------------------------------
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, const BwdSmem& s,
+                                         uint32_t tmem) {
+  using C = BwdCfg<D>;
+  const int tid = threadIdx.x;  // 0..127
+  const int warp = tid >> 5;
+  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const int kr = t.n_base + tid;  // segment-local key row
+  const bool key_ok = kr < t.sk;
+  const int mcount = t.m_hi - t.m_lo;
+  const float c = p.scale_log2;
+  const int causal_off = t.sk - t.sq;
+  bool ok = true;
+  auto uniform_wait = [&](uint64_t* bar, uint32_t parity, uint32_t code) -> bool {
+    const bool r = __all_sync(0xffffffffu, mbar_wait(bar, parity, s.abort, p.err,
+                                                       ERR_BWD_ELEM | code, p.timeout_ns));
+    if (r) tc_fence_after();
+    return r;
+  };
+  // dQ^T of iteration j: thread = feature d (of this CTA's half), 64 query columns
+  auto dq_out = [&](int j) -> bool {
+    if (!uniform_wait(s.dq_full, j & 1, 1)) return false;
+    const int h = t.h0 + j / mcount;
+    const int m0 = (t.m_lo + j % mcount) * C::BM;
+    const int rows = min(C::BM, t.sq - m0);
+    const bool d_ok = tid < C::DH;
+    float* acc = p.dq_acc + (static_cast<size_t>(t.q0 + m0) * p.nheads_q + h) * D +
+                 t.dh * C::DH + tid;
+    const size_t row_stride = static_cast<size_t>(p.nheads_q) * D;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_base + C::COL_DQ + half * 32, r);
+      tmem_ld_wait(r);
+      if (d_ok) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (half * 32 + i < rows)
+            atomicAdd(acc + (half * 32 + i) * row_stride, __uint_as_float(r[i]));
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(s.dq_free);
+    return true;
+  };
+
+  for (int i = 0; i < t.n_iter && ok; ++i) {
+    const int b = i & 1;
+    const int m0 = (t.m_lo + i % mcount) * C::BM;
+    if (!uniform_wait(&s.qdo_full[i % C::NST], (i / C::NST) & 1, 6) ||
+        !uniform_wait(&s.s_full[b], (i >> 1) & 1, 2) || !uniform_wait(s.dp_full, i & 1, 3)) {
+      ok = false;
+      break;
+    }
+    const float* lse2 = s.lsd + (i % C::NST) * 128;  // LSE in the log2 domain
+    const float* dlt = lse2 + 64;                     // D_i
+    float sv[64], dp[64];
+    {
+      uint32_t r[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32(tmem + lane_base + C::COL_S + b * 64 + hh * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) sv[hh * 32 + x] = __uint_as_float(r[x]);
+        tmem_ld32(tmem + lane_base + C::COL_DP + hh * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) dp[hh * 32 + x] = __uint_as_float(r[x]);
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(s.dp_free);
+    // causal: query column j of this block sees this key iff m0 + j >= kr - causal_off
+    const int jmin = CAUSAL ? (kr - causal_off - m0) : 0;
+    uint32_t pk[32];
+    uint4 dsk[8];
+#pragma unroll
+    for (int x = 0; x < 64; x += 2) {
+      float p0 = ex2(fmaf(sv[x], c, -lse2[x]));
+      float p1 = ex2(fmaf(sv[x + 1], c, -lse2[x + 1]));
+      if (!key_ok || (CAUSAL && x < jmin)) p0 = 0.f;
+      if (!key_ok || (CAUSAL && x + 1 < jmin)) p1 = 0.f;
+      const float d0 = p0 * (dp[x] - dlt[x]);
+      const float d1 = p1 * (dp[x + 1] - dlt[x + 1]);
+      pk[x >> 1] = pack_bf16(p0, p1);
+      const uint32_t dpk = pack_bf16(d0, d1);
+      const int w = (x >> 1) & 3;
+      if (w == 0) dsk[x >> 3].x = dpk;
+      else if (w == 1) dsk[x >> 3].y = dpk;
+      else if (w == 2) dsk[x >> 3].z = dpk;
+      else dsk[x >> 3].w = dpk;
+    }
+    tmem_st32(tmem + lane_base + C::COL_S + b * 64, pk);
+    if (i >= 2 && !uniform_wait(&s.ds_free[b], ((i - 2) >> 1) & 1, 4)) {
+      ok = false;
+      break;
+    }
+    uint8_t* dsrow = s.ds + b * C::DS_BYTES + tid * 128;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch)
+      *reinterpret_cast<uint4*>(dsrow + ((ch ^ (tid & 7)) * 16)) = dsk[ch];
+    tmem_st_wait();
+    fence_async_smem();
+    tc_fence_before();
+    mbar_arrive(&s.ds_ready[b]);
+    if (i >= 1 && !dq_out(i - 1)) {
+      ok = false;
+      break;
+    }
+  }
+  if (ok && t.n_iter > 0) ok = dq_out(t.n_iter - 1);
+  if (ok && t.n_iter > 0) ok = uniform_wait(s.dkv_full, 0, 5);
+  if (!ok) return;
+  // dK (x scale) and dV rows of this CTA's half -> bf16.  The TMEM loads are
+  // warp-collective, so every lane runs them; only valid key rows store.
+  const size_t grow = static_cast<size_t>(t.k0 + (key_ok ? kr : 0));
+  const size_t off = ((grow * p.nheads_kv + t.hk) * D + t.dh * C::DH) * 2;
+#pragma unroll 1
+  for (int which = 0; which < 2; ++which) {
+    uint8_t* dst = static_cast<uint8_t*>(which ? p.dk : p.dv) + off;
+    const float f = which ? p.scale : 1.f;
+    const int col0 = which ? C::COL_DK : C::COL_DV;
+#pragma unroll 1
+    for (int cc = 0; cc < C::DH / 32; ++cc) {
+      uint32_t r[32];
+      if (t.n_iter > 0) {
+        tmem_ld32(tmem + lane_base + col0 + cc * 32, r);
+        tmem_ld_wait(r);
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) r[x] = 0u;
+      }
+      if (key_ok) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint4 v;
+          v.x = pack_bf16(__uint_as_float(r[g * 8 + 0]) * f, __uint_as_float(r[g * 8 + 1]) * f);
+          v.y = pack_bf16(__uint_as_float(r[g * 8 + 2]) * f, __uint_as_float(r[g * 8 + 3]) * f);
+          v.z = pack_bf16(__uint_as_float(r[g * 8 + 4]) * f, __uint_as_float(r[g * 8 + 5]) * f);
+          v.w = pack_bf16(__uint_as_float(r[g * 8 + 6]) * f, __uint_as_float(r[g * 8 + 7]) * f);
+          *reinterpret_cast<uint4*>(dst + (cc * 32 + g * 8) * 2) = v;
+        }
+      }
+    }
+  }
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+    attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ CUtensorMap tmQ,
+                         const __grid_constant__ CUtensorMap tmO, const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  BwdTile t;
+  if (!bwd_tile<D, CAUSAL>(p, t)) return;
+  const BwdSmem s = bwd_smem<D>(base);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(s.kv_full, 1);
+    for (int i = 0; i < C::NST; ++i) {
+      mbar_init(&s.qdo_full[i], 32);
+      mbar_init(&s.qdo_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.s_full[i], 1);
+      mbar_init(&s.ds_ready[i], 128);
+      mbar_init(&s.ds_free[i], 1);
+    }
+    mbar_init(s.dp_full, 1);
+    mbar_init(s.dp_free, 128);
+    mbar_init(s.dq_full, 1);
+    mbar_init(s.dq_free, 128);
+    mbar_init(s.dkv_full, 1);
+    *s.abort = 0;
+    fence_mbar_init();
+  }
+  if (D == 64 && warp < 4) {
+    // zero panel after the K tile: the dQ^T MMA reads head_dim 64 as M = 128
+    uint4* z = reinterpret_cast<uint4*>(s.k + C::PANELS * C::KV_PANEL);
+    for (int i = threadIdx.x; i < C::KV_PANEL / 16; i += 128) z[i] = make_uint4(0, 0, 0, 0);
+    fence_async_smem();
+  }
+  if (warp == C::LOAD_WARP && lane_id() == 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(s.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s.tmem_base;
+  if (warp < 4) {
+    bwd_elem<D, CAUSAL>(p, t, s, tmem);
+  } else if (warp == C::LOAD_WARP) {
+    bwd_load<D>(p, t, s, &tmK, &tmV, &tmQ, &tmO);
+  } else {
+    if (lane_id() == 0) bwd_mma<D>(p, t, s, tmem);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// preprocess: D_i = dO_i . O_i, zero the dQ accumulator
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const uint16_t* __restrict__ out,
+                                                           const uint16_t* __restrict__ dout,
+                                                           float* __restrict__ delta,
+                                                           float* __restrict__ dq_acc,
+                                                           int total_q, int hq) {
+  constexpr int TPR = D / 8;  // threads per (row, head), 8 elements each
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long rh = gid / TPR;  // (row, head) index in [Tq][Hq] order
+  const int part = static_cast<int>(gid % TPR);
+  const long long n_rh = static_cast<long long>(total_q) * hq;
+  float acc = 0.f;
+  if (rh < n_rh) {
+    const uint4 a = *reinterpret_cast<const uint4*>(out + rh * D + part * 8);
+    const uint4 b = *reinterpret_cast<const uint4*>(dout + rh * D + part * 8);
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
+      acc = fmaf(__uint_as_float(av[i] & 0xffff0000u), __uint_as_float(bv[i] & 0xffff0000u), acc);
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + rh * D + part * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, TPR);
+  if (rh < n_rh && part == 0) {
+    const long long row = rh / hq;
+    const int h = static_cast<int>(rh % hq);
+    delta[static_cast<long long>(h) * total_q + row] = acc;
+  }
+}
+
+// postprocess: dQ = scale * accumulator -> bf16
+__global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restrict__ acc,
+                                                          uint16_t* __restrict__ dq,
+                                                          long long n8, float scale) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    uint4 o;
+    o.x = pack_bf16(a.x * scale, a.y * scale);
+    o.y = pack_bf16(a.z * scale, a.w * scale);
+    o.z = pack_bf16(b.x * scale, b.y * scale);
+    o.w = pack_bf16(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[i] = o;
+  }
+}
 
 }  // namespace attn

@@ -172,14 +172,25 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, c
                   t.q0 + t.m_base + qt * C::BM);
   }
   uint32_t ring = 0;
+  // on the way out after a timed-out wait elsewhere: let every copy this CTA
+  // issued land before its shared memory is released
+  auto drain = [&]() {
+    for (int qt = 0; qt < C::NQ; ++qt)
+      if (t.m_base + qt * C::BM < t.sq) mbar_wait_drain(&s.q_full[qt], 0, 100000000ull);
+    const uint32_t first = ring > (uint32_t)C::NSLOT ? ring - C::NSLOT : 0u;
+    for (uint32_t r = first; r < ring; ++r)
+      mbar_wait_drain(&s.kv_full[r % C::NSLOT], (r / C::NSLOT) & 1, 100000000ull);
+  };
   // one K or V tile = PANELS chunks
   auto load_tile = [&](bool is_v, int j) -> bool {
     for (int c = 0; c < C::PANELS; ++c, ++ring) {
       const uint32_t slot = ring % C::NSLOT;
       if (ring >= (uint32_t)C::NSLOT) {
         if (!mbar_wait(&s.kv_empty[slot], ((ring / C::NSLOT) - 1) & 1, s.abort, p.err,
-                       ERR_FWD_LOAD | 1, p.timeout_ns))
+                       ERR_FWD_LOAD | 1, p.timeout_ns)) {
+          drain();
           return false;
+        }
       }
       uint8_t* dst = s.ring + slot * C::CHUNK;
       mbar_expect_tx(&s.kv_full[slot], C::CHUNK);

@@ -72,6 +72,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Bounded wait that ignores the abort flag: used on the way out of a CTA that
+// gave up, to let its own TMA copies land before the shared memory is released.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), shared::cta destination, no multicast
 // ---------------------------------------------------------------------------
