@@ -22,13 +22,15 @@ import os
 import torch
 
 __all__ = ["attn_fwd", "attn_bwd", "attention", "bwd_workspace_size", "last_device_error",
+           "set_timing_events", "KERNEL_FWD", "KERNEL_BWD_MAIN",
            "library", "LIB_PATH", "AttnError", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED",
           3: "ATTN_ERR_CUDA", 4: "ATTN_ERR_TIMEOUT"}
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_last_device_error",
-            "attn_version")
+            "attn_set_timing_events", "attn_version")
+KERNEL_FWD, KERNEL_BWD_MAIN = 0, 1
 
 
 class AttnError(RuntimeError):
@@ -60,6 +62,8 @@ def library() -> ctypes.CDLL:
         lib.attn_last_device_error.argtypes = [vp, ctypes.c_char_p, ctypes.c_size_t]
         lib.attn_last_device_error.restype = ctypes.c_int
         lib.attn_version.restype = ctypes.c_char_p
+        lib.attn_set_timing_events.argtypes = [i32, vp, vp]
+        lib.attn_set_timing_events.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -141,6 +145,17 @@ def attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, 
     if rc != 0:
         raise AttnError("attn_bwd", rc)
     return dq, dk, dv
+
+
+def set_timing_events(kernel: int, start=None, stop=None):
+    """Record torch.cuda.Event pair around one kernel of later calls (None: off)."""
+    if start is not None and (start.cuda_event == 0 or stop.cuda_event == 0):
+        raise ValueError("record the events once before passing them (torch creates them lazily)")
+    sp = ctypes.c_void_p(start.cuda_event) if start is not None else None
+    ep = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
+    rc = library().attn_set_timing_events(int(kernel), sp, ep)
+    if rc != 0:
+        raise AttnError("attn_set_timing_events", rc)
 
 
 def last_device_error(stream=None):

@@ -23,6 +23,19 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// caller-owned events recorded around one kernel (attn_set_timing_events)
+struct TimingEvents {
+  cudaEvent_t start = nullptr, stop = nullptr;
+};
+thread_local TimingEvents t_events[2];
+
+void record_start(int kernel, cudaStream_t s) {
+  if (t_events[kernel].start) cudaEventRecord(t_events[kernel].start, s);
+}
+void record_stop(int kernel, cudaStream_t s) {
+  if (t_events[kernel].stop) cudaEventRecord(t_events[kernel].stop, s);
+}
+
 struct DeviceState {
   std::once_flag once;
   cudaError_t init_status = cudaSuccess;
@@ -132,8 +145,11 @@ attn_status_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   const int m_tiles = (max_q + C::BM * C::NQ - 1) / (C::BM * C::NQ);
   if (m_tiles == 0) return ATTN_OK;
   dim3 grid(m_tiles, hq, batch);
+  record_start(ATTN_KERNEL_FWD, stream);
   attn_fwd_kernel<D, CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  record_stop(ATTN_KERNEL_FWD, stream);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D, bool CAUSAL>
@@ -157,8 +173,11 @@ attn_status_t launch_bwd_main(const BwdArgs& a, const BwdParams& bp, cudaStream_
   const int n_blocks = (a.max_k + C::BN - 1) / C::BN;
   if (n_blocks == 0) return ATTN_OK;
   dim3 grid(n_blocks * C::NSPLIT, a.hkv, a.batch);
+  record_start(ATTN_KERNEL_BWD_MAIN, stream);
   attn_bwd_main_kernel<D, CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mk, mv, mq, mo, bp);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  record_stop(ATTN_KERNEL_BWD_MAIN, stream);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D>
@@ -352,6 +371,14 @@ extern "C" attn_status_t attn_last_device_error(attn_stream_t stream, char* msg,
                 kid < sizeof(kernels) / sizeof(kernels[0]) ? kernels[kid] : "?", word & 0xffu);
   put(buf);
   return ATTN_ERR_TIMEOUT;
+}
+
+extern "C" attn_status_t attn_set_timing_events(int32_t kernel, void* start, void* stop) {
+  if (kernel != ATTN_KERNEL_FWD && kernel != ATTN_KERNEL_BWD_MAIN) return ATTN_ERR_INVALID_ARG;
+  if ((start == nullptr) != (stop == nullptr)) return ATTN_ERR_INVALID_ARG;
+  t_events[kernel].start = static_cast<cudaEvent_t>(start);
+  t_events[kernel].stop = static_cast<cudaEvent_t>(stop);
+  return ATTN_OK;
 }
 
 extern "C" const char* attn_version(void) { return "exact_attention_b200 0.1 sm_100a"; }

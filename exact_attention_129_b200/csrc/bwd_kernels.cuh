@@ -1,9 +1,10 @@
 // bwd_kernels.cuh -- sm_100a backward pass: dQ, dK, dV of exact attention,
 // recomputing P from the forward's LSE.
 //
-// The FA4 repository guide splits its backward into a preprocess kernel, a main
-// kernel and a postprocess kernel; the plainest reading of that split (and of
-// the method: P = exp(S - LSE), dS = P * (dP - D), D_i = dO_i . O_i) is:
+// The FA4 repository guide (Backward Kernels) splits its backward into a
+// preprocess kernel, a main kernel and a postprocess kernel; the plainest
+// reading of that split, with the method's P = exp(S - LSE), dS = P * (dP - D)
+// and D_i = dO_i . O_i, is:
 //
 //   1. preprocess: D_i = sum_d dO_id O_id (fp32) and a zeroed fp32 dQ accumulator;
 //   2. main: per key block, loop over the query blocks (and, for GQA, over the

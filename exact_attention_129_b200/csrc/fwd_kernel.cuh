@@ -1,12 +1,13 @@
 // fwd_kernel.cuh -- sm_100a forward kernel: tiled exact attention with an
 // online softmax, returning O and the per-row LSE.
 //
-// The FA4 repository guide describes the forward as "load Q tile -> loop over
-// K/V blocks (pipelined) -> online softmax accumulation -> store O and LSE",
-// with row max / row sum tracking, block-range skipping for causal masks and a
-// varlen-aware scheduler; the head_dim=256 regression check times it on B200
-// with softmax_scale = hdim**-0.5.  This file is our own design of that loop
-// for one B200 SM:
+// The FA4 repository guide (Key Patterns, Core Abstractions) describes the
+// forward as a Q tile kept on chip while K/V blocks stream past it through a
+// pipeline, an online softmax that tracks each row's max and sum, block ranges
+// that skip fully masked blocks under causal masks, and a scheduler that knows
+// about varlen batches; the "FA4 head_dim=256 B200 Regression Check" times it on
+// B200 at head_dim^-0.5 scale.  This file is our own design of that loop for one
+// B200 SM:
 //
 //   * One CTA owns NQ query tiles of 128 rows of one (segment, head): NQ = 2
 //     for head_dim 64/128 (both tiles share every K/V tile brought on chip),

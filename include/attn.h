@@ -11,14 +11,17 @@
  *             from the LSE.
  *
  * This is the operation the attention pages benchmark: the cosmos-framework
- * issue #118 calls it through a varlen frontend (cu_seqlens, max_seqlen,
- * 32 query / 8 key-value heads, head_dim 128); the flash-attention issue #2729
- * repro calls the forward with out=, lse= and return_lse= and checks it against
- * torch's scaled_dot_product_attention; the FA4 head_dim=256 regression check
- * times forward and backward with softmax_scale = hdim**-0.5, MHA and GQA
- * (nheads_kv = 1), causal and not; the FA4 repository guide describes the
- * forward as "load Q tile -> loop over K/V blocks -> online softmax -> store O
- * and LSE" and the backward as a preprocess, a main kernel and a postprocess.
+ * issue #118 ("FA2 vs NATTEN on A100", benchmark script) calls it through a
+ * varlen frontend with cu_seqlens and max_seqlen, 32 query / 8 key-value heads
+ * and head_dim 128; the flash-attention issue #2729 ("FA4/B200 return_lse=True
+ * makes D64 forward about 19% faster", repro script) calls the forward with
+ * caller-provided out and lse buffers and a return_lse switch and checks it
+ * against torch's scaled_dot_product_attention; the "FA4 head_dim=256 B200
+ * Regression Check" (Environment, Results) times forward and backward at
+ * head_dim^-0.5 scale, MHA and GQA with one key-value head, causal and not; the
+ * FA4 repository guide (Key Patterns, Backward Kernels) describes a forward that
+ * streams K/V blocks past a resident Q tile with an online softmax and writes O
+ * and the LSE, and a backward split into preprocess, main and postprocess kernels.
  *
  * Layouts (row-major, last index fastest, every pointer DEVICE memory):
  *   q, out, dout, dq : bf16  [total_q][nheads_q][head_dim]
@@ -77,9 +80,9 @@ typedef enum {
 } attn_status_t;
 
 /*
- * Forward pass (the FA4 guide's "load Q tile -> loop over K/V blocks
- * (pipelined) -> online softmax accumulation -> store O and LSE"; issue #2729's
- * _flash_attn_fwd(q, k, v, out=, lse=, return_lse=)).
+ * Forward pass (FA4 repository guide, Key Patterns: a resident Q tile, a
+ * pipelined loop over K/V blocks with an online softmax, then O and the LSE are
+ * stored; issue #2729's repro calls the forward with out, lse and return_lse).
  *
  *   q, k, v        inputs, layouts above (read only).
  *   cu_seqlens_q/k device int32 [batch+1].
@@ -111,8 +114,8 @@ size_t attn_bwd_workspace_size(int32_t batch, int32_t total_q, int32_t nheads_q,
                                int32_t head_dim);
 
 /*
- * Backward pass (the FA4 guide's backward: a preprocess kernel, the main
- * kernel that recomputes P from the LSE, and a postprocess kernel).
+ * Backward pass (FA4 repository guide, Backward Kernels: a preprocess kernel,
+ * the main kernel that recomputes P from the LSE, and a postprocess kernel).
  *
  *   q, k, v, out   as given to / produced by attn_fwd.
  *   lse            fp32 [nheads_q][total_q] from attn_fwd(return_lse = 1).
@@ -144,6 +147,19 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  * most msg_len bytes.
  */
 attn_status_t attn_last_device_error(attn_stream_t stream, char* msg, size_t msg_len);
+
+/*
+ * Profiling aid (not part of the computation).  After this call, in the calling
+ * host thread, every attn_fwd (kernel = ATTN_KERNEL_FWD) or attn_bwd
+ * (kernel = ATTN_KERNEL_BWD_MAIN: its main kernel, between the preprocess and
+ * the dQ conversion) records `start` just before and `stop` just after that
+ * kernel on the call's stream, so cudaEventElapsedTime gives the kernel's own
+ * duration.  start/stop are cudaEvent_t handles owned by the caller; passing
+ * NULL for both turns recording off.  Returns ATTN_ERR_INVALID_ARG for an
+ * unknown kernel id or for exactly one NULL event.
+ */
+enum { ATTN_KERNEL_FWD = 0, ATTN_KERNEL_BWD_MAIN = 1 };
+attn_status_t attn_set_timing_events(int32_t kernel, void* start, void* stop);
 
 /* Library version string, e.g. "exact_attention_b200 0.1 sm_100a". */
 const char* attn_version(void);

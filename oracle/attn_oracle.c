@@ -22,14 +22,15 @@
  *     dK_j  = scale * sum_{h in group(hk)} sum_i dS_ij q_i
  *     dV_j  =         sum_{h in group(hk)} sum_i P_ij dO_i
  *
- * Sources: the attention pages of this project -- the flash-attention issue
- * "[FA4/B200] return_lse=True makes D64 forward about 19% faster" (its repro
- * checks the kernel against torch's scaled_dot_product_attention and allocates
- * the LSE as (batch, heads, seqlen)), the FA4 head_dim=256 regression check
- * ("softmax_scale = hdim**-0.5"), and the FA4 repository guide (online softmax
- * with row max / row sum, "Packs multiple Q heads per KV head" for GQA, varlen
- * through cu_seqlens).  The pages print no formulas; the ones above are the
- * textbook definition of softmax attention and of its gradient.
+ * Sources: the flash-attention issue "[FA4/B200] return_lse=True makes D64
+ * forward about 19% faster" (its repro checks the kernel against torch's
+ * scaled_dot_product_attention and allocates the LSE as batch x heads x seqlen),
+ * the "FA4 head_dim=256 B200 Regression Check" (Environment: the softmax scale is
+ * head_dim^-0.5) and the FA4 repository guide (Core Abstractions: an online
+ * softmax that tracks each row's max and sum; Other Components: several query
+ * heads share one key/value head for GQA; Public API: varlen through
+ * cu_seqlens).  The pages print no formulas; the ones above are the textbook
+ * definition of softmax attention and of its gradient.
  *
  * Readings where the pages are silent:
  *   - GQA map: contiguous groups, hk = h / G.
