@@ -27,9 +27,9 @@ __all__ = ["attn_fwd", "attn_bwd", "attention", "bwd_workspace_size", "last_devi
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED",
-          3: "ATTN_ERR_CUDA", 4: "ATTN_ERR_TIMEOUT"}
+          3: "ATTN_ERR_CUDA", 4: "ATTN_ERR_TIMEOUT", 5: "ATTN_ERR_SCRATCH_TOO_SMALL"}
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_last_device_error",
-            "attn_set_timing_events", "attn_version")
+            "attn_set_timing_events", "attn_bwd_static_scratch", "attn_version")
 KERNEL_FWD, KERNEL_BWD_MAIN = 0, 1
 
 
@@ -64,6 +64,10 @@ def library() -> ctypes.CDLL:
         lib.attn_version.restype = ctypes.c_char_p
         lib.attn_set_timing_events.argtypes = [i32, vp, vp]
         lib.attn_set_timing_events.restype = ctypes.c_int
+        lib.attn_bwd_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                                i32, i32, i32, i32, i32, f32, i32, vp, vp, vp,
+                                                vp]
+        lib.attn_bwd_static_scratch.restype = ctypes.c_int
         _lib = lib
     return _lib
 

@@ -333,6 +333,50 @@ extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, c
   return bwd_launch(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------------------
+// attn_bwd_static_scratch: the backward for callers that cannot allocate.
+// Its scratch is this file-scope device array; in host code the name is only a
+// host-side stand-in, so the device address is looked up once per device with
+// cudaGetSymbolAddress and handed to the kernels as the workspace pointer.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_static_scratch[ATTN_STATIC_SCRATCH_BYTES];
+
+namespace {
+struct StaticScratch {
+  std::once_flag once;
+  cudaError_t status = cudaSuccess;
+  void* ptr = nullptr;
+};
+StaticScratch g_scratch[kMaxDevices];
+}  // namespace
+
+extern "C" attn_status_t attn_bwd_static_scratch(
+    const void* q, const void* k, const void* v, const void* out, const float* lse,
+    const void* dout, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch,
+    int32_t total_q, int32_t total_k, int32_t max_seqlen_q, int32_t max_seqlen_k,
+    int32_t nheads_q, int32_t nheads_kv, int32_t head_dim, float scale, int32_t causal,
+    void* dq, void* dk, void* dv, attn_stream_t stream) {
+  attn_status_t st = check_common(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                  max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim,
+                                  scale);
+  if (st != ATTN_OK) return st;
+  const size_t need = bwd_workspace_bytes(batch, total_q, nheads_q, head_dim);
+  if (need > ATTN_STATIC_SCRATCH_BYTES) return ATTN_ERR_SCRATCH_TOO_SMALL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  StaticScratch& sc = g_scratch[dev];
+  std::call_once(sc.once, [&sc] {
+    // runs with `dev` current: the address is that device's copy of the array
+    sc.status = cudaGetSymbolAddress(&sc.ptr, g_static_scratch);
+  });
+  if (sc.status != cudaSuccess || sc.ptr == nullptr) return ATTN_ERR_CUDA;
+  // attn_bwd's own checks and launches, with the array as its workspace; its
+  // preprocess kernel zeroes the dQ accumulator and rewrites D_i on every call
+  return attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                  max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim, scale, causal, dq,
+                  dk, dv, sc.ptr, ATTN_STATIC_SCRATCH_BYTES, stream);
+}
+
 extern "C" attn_status_t attn_last_device_error(attn_stream_t stream, char* msg,
                                                 size_t msg_len) {
   auto put = [&](const char* m) {

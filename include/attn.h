@@ -76,7 +76,8 @@ typedef enum {
   ATTN_ERR_INVALID_ARG = 1,
   ATTN_ERR_UNSUPPORTED = 2,
   ATTN_ERR_CUDA = 3,
-  ATTN_ERR_TIMEOUT = 4
+  ATTN_ERR_TIMEOUT = 4,
+  ATTN_ERR_SCRATCH_TOO_SMALL = 5 /* attn_bwd_static_scratch: problem too large */
 } attn_status_t;
 
 /*
@@ -138,6 +139,45 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        float scale, int32_t causal,
                        void* dq, void* dk, void* dv,
                        void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * Backward pass that allocates nothing and takes no workspace.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers that
+ * cannot call cudaMalloc and have no spare device buffer to lend as workspace:
+ * plug-ins whose host process owns all device memory and exposes no allocator,
+ * services that have reserved the whole device for their own pool (where a
+ * foreign allocation fails or fragments it), and latency-critical loops that ban
+ * allocator calls because cudaMalloc/cudaFree can synchronise the device.
+ *
+ * It computes exactly what attn_bwd computes, with the same arguments minus the
+ * workspace: the scratch attn_bwd would take from `workspace` (the fp32 dQ
+ * accumulator and the fp32 row-dot D_i) lives instead in one file-scope device
+ * array of ATTN_STATIC_SCRATCH_BYTES inside the library, which every GPU that
+ * loads the library holds until the process exits.
+ *
+ * Limits and rules:
+ *   - the problem must fit: attn_bwd_workspace_size(batch, total_q, nheads_q,
+ *     head_dim) <= ATTN_STATIC_SCRATCH_BYTES, else ATTN_ERR_SCRATCH_TOO_SMALL is
+ *     returned and nothing is launched;
+ *   - the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture;
+ *   - every call on a device shares the one array and finds the previous call's
+ *     contents in it; the call clears what must start at zero itself, but calls
+ *     that overlap on the GPU (other streams, other host threads) race on it and
+ *     must be serialised by the caller;
+ *   - no cudaMalloc, cudaFree or other allocating routine is called.
+ */
+#define ATTN_STATIC_SCRATCH_BYTES (64u << 20)
+attn_status_t attn_bwd_static_scratch(const void* q, const void* k, const void* v,
+                                      const void* out, const float* lse, const void* dout,
+                                      const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                      int32_t batch, int32_t total_q, int32_t total_k,
+                                      int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                      int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                                      float scale, int32_t causal,
+                                      void* dq, void* dk, void* dv, attn_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's error
