@@ -96,6 +96,25 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // bf16 [rows][heads][D] viewed as a 3-D tensor (D, heads, rows); box of
 // 64 columns x 1 head x box_rows rows, 128-byte swizzle.
+// fp32 [rows][heads][d] viewed as (d, heads, rows); box of box_cols x 1 x box_rows,
+// no swizzle (the dQ accumulator, written by TMA reduce-adds)
+bool make_map_f32(CUtensorMap* map, const void* ptr, int rows, int heads, int d, int box_cols,
+                  int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(heads) * d * 4};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), 1u,
+                             static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map(CUtensorMap* map, const void* ptr, int rows, int heads, int d, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
@@ -164,17 +183,19 @@ attn_status_t launch_bwd_main(const BwdArgs& a, const BwdParams& bp, cudaStream_
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
-  CUtensorMap mk, mv, mq, mo;
+  CUtensorMap mk, mv, mq, mo, mdq;
   if (!make_map(&mk, a.k, a.total_k, a.hkv, D, 128) ||
       !make_map(&mv, a.v, a.total_k, a.hkv, D, 128) ||
       !make_map(&mq, a.q, a.total_q, a.hq, D, C::BM) ||
-      !make_map(&mo, a.dout, a.total_q, a.hq, D, C::BM))
+      !make_map(&mo, a.dout, a.total_q, a.hq, D, C::BM) ||
+      !make_map_f32(&mdq, bp.dq_acc, a.total_q, a.hq, D, 32, C::BM / 2))
     return ATTN_ERR_CUDA;
   const int n_blocks = (a.max_k + C::BN - 1) / C::BN;
   if (n_blocks == 0) return ATTN_OK;
   dim3 grid(n_blocks * C::NSPLIT, a.hkv, a.batch);
   record_start(ATTN_KERNEL_BWD_MAIN, stream);
-  attn_bwd_main_kernel<D, CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mk, mv, mq, mo, bp);
+  attn_bwd_main_kernel<D, CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mk, mv, mq, mo, mdq,
+                                                                                bp);
   const cudaError_t e = cudaGetLastError();
   record_stop(ATTN_KERNEL_BWD_MAIN, stream);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -424,5 +445,12 @@ extern "C" attn_status_t attn_set_timing_events(int32_t kernel, void* start, voi
   t_events[kernel].stop = static_cast<cudaEvent_t>(stop);
   return ATTN_OK;
 }
+
+#ifdef ATTN_TRACE
+extern "C" int attn_debug_set_trace(void* buf) {
+  unsigned long long* p = static_cast<unsigned long long*>(buf);
+  return cudaMemcpyToSymbol(g_attn_trace, &p, sizeof(p)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 extern "C" const char* attn_version(void) { return "exact_attention_b200 0.1 sm_100a"; }

@@ -17,8 +17,9 @@
 //
 // Main-kernel layout for one CTA (128 keys; head_dim 256 is split into two
 // 128-wide halves handled by two CTAs, each recomputing S and dP in full):
-//   tensor memory: S^T x2 (64 cols each; P^T in bf16 is written back over the
-//                  first 32), dP^T (64), dQ^T (64), dV (DH), dK (DH)  = 512 cols
+//   tensor memory: S^T x2 (64 cols each; P^T in bf16 is written back over
+//                  columns 0-15 and 32-47), dP^T (64), dQ^T (64), dV (DH),
+//                  dK (DH)  = 512 cols
 //   shared memory: K and V tiles (resident), a ring of NST (Q, dO) stages of
 //                  64 query rows, two dS^T tiles (128 keys x 64 queries, bf16,
 //                  128-byte swizzled: the same bytes are the K-major A operand of
@@ -99,15 +100,23 @@ struct BwdCfg {
   static constexpr int OFF_ST = OFF_V + V_BYTES;
   static constexpr int OFF_DS = OFF_ST + NST * STAGE_BYTES;
   static constexpr int OFF_LSD = OFF_DS + 2 * DS_BYTES;      // NST x 128 floats
-  static constexpr int OFF_BAR = OFF_LSD + NST * 128 * 4;
+  // dQ^T staging for the TMA reduce-add: per elementwise warp 64 queries x 32
+  // features fp32 (head_dim 256 has no room left and adds with atomics instead)
+  static constexpr bool DQ_TMA = (D != 256);
+  static constexpr int DQ_WARP_BYTES = (BM / 2) * 32 * 4;  // 4 KB: 32 queries x 32 features
+  static constexpr int OFF_DQS = OFF_LSD + NST * 128 * 4;
+  static constexpr int OFF_BAR = OFF_DQS + (DQ_TMA ? 2 * (DH / 32) * DQ_WARP_BYTES : 0);
   // kv_full, qdo_full[NST], qdo_empty[NST], s_full[2], dp_full, dp_free,
   // ds_ready[2], ds_free[2], dq_full, dq_free, dkv_full
   static constexpr int NBAR = 1 + 2 * NST + 2 + 2 + 2 + 2 + 3;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static constexpr int THREADS = 192;
-  static constexpr int LOAD_WARP = 4, MMA_WARP = 5;
+  // warps 0-7: two elementwise warpgroups (each takes 32 of the 64 query
+  // columns of a block, thread = key row); warp 8: TMA; warp 9: MMA
+  static constexpr int ELEM_THREADS = 256;
+  static constexpr int THREADS = 320;
+  static constexpr int LOAD_WARP = 8, MMA_WARP = 9;
   // tensor memory columns
   static constexpr int COL_S = 0, COL_DP = 128, COL_DQ = 192, COL_DV = 256, COL_DK = 256 + DH;
   static constexpr uint32_t IDESC_SDP = idesc_bf16(128, BM, false, false);
@@ -116,7 +125,7 @@ struct BwdCfg {
 };
 
 struct BwdSmem {
-  uint8_t *k, *v, *st, *ds;
+  uint8_t *k, *v, *st, *ds, *dqs;
   float* lsd;
   uint64_t *kv_full, *qdo_full, *qdo_empty, *s_full, *dp_full, *dp_free, *ds_ready, *ds_free,
       *dq_full, *dq_free, *dkv_full;
@@ -133,6 +142,7 @@ __device__ __forceinline__ BwdSmem bwd_smem(uint8_t* base) {
   s.st = base + C::OFF_ST;
   s.ds = base + C::OFF_DS;
   s.lsd = reinterpret_cast<float*>(base + C::OFF_LSD);
+  s.dqs = base + C::OFF_DQS;
   uint64_t* b = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
   s.kv_full = b;
   s.qdo_full = b + 1;
@@ -292,10 +302,12 @@ struct BwdMma {
     const uint32_t q_half = smem_u32(stg) + t.dh * 2 * C::QD_PANEL;
     const uint32_t do_half = smem_u32(stg) + (C::PANELS + t.dh * 2) * C::QD_PANEL;
     const uint32_t ds = smem_u32(s.ds + bj * C::DS_BYTES);
-    // dV += P^T dO  (A = P^T in tensor memory, B = dO rows, MN-major)
+    // dV += P^T dO  (A = P^T in tensor memory, B = dO rows, MN-major).  The
+    // P of query columns [32 w, 32 w + 32) sits at columns 32 w .. 32 w + 15 of
+    // the S buffer, 8 columns per 16-query k-step.
 #pragma unroll
     for (int ks = 0; ks < C::BM / 16; ++ks)
-      mma_ts(tmem + C::COL_DV, tmem + C::COL_S + bj * 64 + ks * 8,
+      mma_ts(tmem + C::COL_DV, tmem + C::COL_S + bj * 64 + (ks >> 1) * 32 + (ks & 1) * 8,
              sdesc_sw128(do_half + ks * 2048, C::QD_PANEL, 1024), C::IDESC_KV,
              (!first || ks) ? 1u : 0u);
     // dK += dS^T Q  (A = dS^T K-major in shared memory)
@@ -323,12 +335,17 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, co
   using C = BwdCfg<D>;
   if (t.n_iter == 0) return;
   BwdMma<D> m(p, s, t, tmem);
+  TRACE_INIT();
   if (!m.wait(s.kv_full, 0, 1)) return;
   auto do_grads = [&](int j) -> bool {
     if (!m.wait(&s.ds_ready[j & 1], (j >> 1) & 1, 2)) return false;
+    if (j < 200) TRACE(2048 + j * 8 + 4);
     m.grads(j, j == 0);
+    if (j < 200) TRACE(2048 + j * 8 + 5);
     if (j >= 1 && !m.wait(s.dq_free, (j - 1) & 1, 3)) return false;
+    if (j < 200) TRACE(2048 + j * 8 + 6);
     m.dq(j);
+    if (j < 200) TRACE(2048 + j * 8 + 7);
     mma_commit(s.dq_full);
     mma_commit(&s.qdo_empty[j % C::NST]);
     mma_commit(&s.ds_free[j & 1]);
@@ -340,11 +357,15 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, co
     // gradient MMAs have released it
     if (C::NST == 1 && i >= 1 && !do_grads(i - 1)) return;
     if (!m.wait(&s.qdo_full[st], (i / C::NST) & 1, 4)) return;
+    if (i < 200) TRACE(2048 + i * 8 + 0);
     const uint8_t* stg = s.st + st * C::STAGE_BYTES;
     m.issue_kt(C::COL_S + (i & 1) * 64, s.k, stg);
     mma_commit(&s.s_full[i & 1]);
+    if (i < 200) TRACE(2048 + i * 8 + 1);
     if (i >= 1 && !m.wait(s.dp_free, (i - 1) & 1, 5)) return;
+    if (i < 200) TRACE(2048 + i * 8 + 2);
     m.issue_kt(C::COL_DP, s.v, stg + C::PANELS * C::QD_PANEL);
+    if (i < 200) TRACE(2048 + i * 8 + 3);
     mma_commit(s.dp_full);
     if (C::NST > 1 && i >= 1 && !do_grads(i - 1)) return;
   }
@@ -357,47 +378,72 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, co
 // ---------------------------------------------------------------------------
 template <int D, bool CAUSAL>
 __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, const BwdSmem& s,
-                                         uint32_t tmem) {
+                                         uint32_t tmem, const CUtensorMap* tmDQ) {
+  // two warpgroups: warpgroup wg handles query columns [32 wg, 32 wg + 32) of
+  // every block; within a warpgroup, thread = key row = TMEM lane
   using C = BwdCfg<D>;
-  const int tid = threadIdx.x;  // 0..127
-  const int warp = tid >> 5;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  const int kr = t.n_base + tid;  // segment-local key row
+  const int tid = threadIdx.x;       // 0..255
+  const int wg = tid >> 7;
+  const int row = tid & 127;         // key row within the block / TMEM lane
+  const int wq = row >> 5;           // lane quadrant of this warp
+  const int lane = tid & 31;
+  const int qc0 = wg * 32;           // first query column of this warpgroup
+  const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+  const int kr = t.n_base + row;     // segment-local key row
   const bool key_ok = kr < t.sk;
   const int mcount = t.m_hi - t.m_lo;
   const float c = p.scale_log2;
   const int causal_off = t.sk - t.sq;
   bool ok = true;
+  TRACE_INIT();
   auto uniform_wait = [&](uint64_t* bar, uint32_t parity, uint32_t code) -> bool {
     const bool r = __all_sync(0xffffffffu, mbar_wait(bar, parity, s.abort, p.err,
                                                        ERR_BWD_ELEM | code, p.timeout_ns));
     if (r) tc_fence_after();
     return r;
   };
-  // dQ^T of iteration j: thread = feature d (of this CTA's half), 64 query columns
+  // dQ^T of iteration j, this warpgroup's 32 query columns: thread = feature d.
+  // With DQ_TMA each warp stages 32 queries x 32 features in shared memory and
+  // one lane adds the tile into the fp32 accumulator with a TMA reduce; query
+  // rows beyond the segment hold exact zeros (their P is 0), so adding them is
+  // harmless.
   auto dq_out = [&](int j) -> bool {
     if (!uniform_wait(s.dq_full, j & 1, 1)) return false;
     const int h = t.h0 + j / mcount;
     const int m0 = (t.m_lo + j % mcount) * C::BM;
-    const int rows = min(C::BM, t.sq - m0);
-    const bool d_ok = tid < C::DH;
-    float* acc = p.dq_acc + (static_cast<size_t>(t.q0 + m0) * p.nheads_q + h) * D +
-                 t.dh * C::DH + tid;
-    const size_t row_stride = static_cast<size_t>(p.nheads_q) * D;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_base + C::COL_DQ + half * 32, r);
-      tmem_ld_wait(r);
-      if (d_ok) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (half * 32 + i < rows)
-            atomicAdd(acc + (half * 32 + i) * row_stride, __uint_as_float(r[i]));
-      }
-    }
+    const bool d_ok = row < C::DH;
+    uint32_t r0[32];
+    tmem_ld32(tmem + lane_base + C::COL_DQ + qc0, r0);
+    tmem_ld_wait(r0);
     tc_fence_before();
     mbar_arrive(s.dq_free);
+    if constexpr (C::DQ_TMA) {
+      if (d_ok) {
+        // slots: (DH / 32) per warpgroup; only warps with d < DH stage
+        float* stg =
+            reinterpret_cast<float*>(s.dqs + (wg * (C::DH / 32) + wq) * C::DQ_WARP_BYTES);
+        if (lane == 0) bulk_wait_read0();  // the previous reduce has read the buffer
+        __syncwarp();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) stg[x * 32 + lane] = __uint_as_float(r0[x]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(tmDQ, stg, t.dh * C::DH + wq * 32, h, t.q0 + m0 + qc0);
+          bulk_commit();
+        }
+      }
+    } else {
+      const int rows = min(C::BM, t.sq - m0) - qc0;
+      float* acc = p.dq_acc + (static_cast<size_t>(t.q0 + m0 + qc0) * p.nheads_q + h) * D +
+                   t.dh * C::DH + row;
+      const size_t row_stride = static_cast<size_t>(p.nheads_q) * D;
+      if (d_ok) {
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          if (x < rows) atomicAdd(acc + x * row_stride, __uint_as_float(r0[x]));
+      }
+    }
     return true;
   };
 
@@ -409,95 +455,107 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
       ok = false;
       break;
     }
-    const float* lse2 = s.lsd + (i % C::NST) * 128;  // LSE in the log2 domain
-    const float* dlt = lse2 + 64;                     // D_i
-    float sv[64], dp[64];
-    {
-      uint32_t r[32];
+    if (tid == 0 && i < 200) TRACE(i * 8 + 0);
+    const float* lse2 = s.lsd + (i % C::NST) * 128 + qc0;  // LSE in the log2 domain
+    const float* dlt = s.lsd + (i % C::NST) * 128 + 64 + qc0;  // D_i
+    uint32_t sr[32], dr[32];
+    tmem_ld32(tmem + lane_base + C::COL_S + b * 64 + qc0, sr);
+    tmem_ld32(tmem + lane_base + C::COL_DP + qc0, dr);
+    tmem_ld_wait(sr);
+    tmem_ld_wait(dr);
+    tc_fence_before();
+    if (tid == 0 && i < 200) TRACE(i * 8 + 1);
+    mbar_arrive(s.dp_free);
+    // causal: query column x of this block sees this key iff m0 + x >= kr - causal_off
+    const int jmin = CAUSAL ? (kr - causal_off - m0 - qc0) : 0;
+    uint32_t pk[16];
+    uint4 dsk[4];
+    const uint64_t c2 = f2_pack(c, c);
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        tmem_ld32(tmem + lane_base + C::COL_S + b * 64 + hh * 32, r);
-        tmem_ld_wait(r);
+    for (int x4 = 0; x4 < 8; ++x4) {
+      const float4 l4 = reinterpret_cast<const float4*>(lse2)[x4];
+      const float4 d4 = reinterpret_cast<const float4*>(dlt)[x4];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) sv[hh * 32 + x] = __uint_as_float(r[x]);
-        tmem_ld32(tmem + lane_base + C::COL_DP + hh * 32, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) dp[hh * 32 + x] = __uint_as_float(r[x]);
+      for (int hp = 0; hp < 2; ++hp) {
+        const int x = x4 * 4 + hp * 2;
+        float e0, e1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[x]), __uint_as_float(sr[x + 1])), c2,
+                         hp ? f2_pack(-l4.z, -l4.w) : f2_pack(-l4.x, -l4.y)),
+                  e0, e1);
+        float p0 = ex2(e0), p1 = ex2(e1);
+        if (!key_ok || (CAUSAL && x < jmin)) p0 = 0.f;
+        if (!key_ok || (CAUSAL && x + 1 < jmin)) p1 = 0.f;
+        float d0, d1;
+        f2_unpack(f2_mul(f2_pack(p0, p1),
+                         f2_add(f2_pack(__uint_as_float(dr[x]), __uint_as_float(dr[x + 1])),
+                                hp ? f2_pack(-d4.z, -d4.w) : f2_pack(-d4.x, -d4.y))),
+                  d0, d1);
+        pk[x >> 1] = pack_bf16(p0, p1);
+        const uint32_t dpk = pack_bf16(d0, d1);
+        const int w = (x >> 1) & 3;
+        if (w == 0) dsk[x >> 3].x = dpk;
+        else if (w == 1) dsk[x >> 3].y = dpk;
+        else if (w == 2) dsk[x >> 3].z = dpk;
+        else dsk[x >> 3].w = dpk;
       }
     }
-    tc_fence_before();
-    mbar_arrive(s.dp_free);
-    // causal: query column j of this block sees this key iff m0 + j >= kr - causal_off
-    const int jmin = CAUSAL ? (kr - causal_off - m0) : 0;
-    uint32_t pk[32];
-    uint4 dsk[8];
-#pragma unroll
-    for (int x = 0; x < 64; x += 2) {
-      float p0 = ex2(fmaf(sv[x], c, -lse2[x]));
-      float p1 = ex2(fmaf(sv[x + 1], c, -lse2[x + 1]));
-      if (!key_ok || (CAUSAL && x < jmin)) p0 = 0.f;
-      if (!key_ok || (CAUSAL && x + 1 < jmin)) p1 = 0.f;
-      const float d0 = p0 * (dp[x] - dlt[x]);
-      const float d1 = p1 * (dp[x + 1] - dlt[x + 1]);
-      pk[x >> 1] = pack_bf16(p0, p1);
-      const uint32_t dpk = pack_bf16(d0, d1);
-      const int w = (x >> 1) & 3;
-      if (w == 0) dsk[x >> 3].x = dpk;
-      else if (w == 1) dsk[x >> 3].y = dpk;
-      else if (w == 2) dsk[x >> 3].z = dpk;
-      else dsk[x >> 3].w = dpk;
-    }
-    tmem_st32(tmem + lane_base + C::COL_S + b * 64, pk);
+    // P (bf16 pairs) goes over the first 16 of this warpgroup's own 32 score
+    // columns, which this warpgroup has already read: the other warpgroup may
+    // still be reading its own columns
+    tmem_st16(tmem + lane_base + C::COL_S + b * 64 + wg * 32, pk);
+    if (tid == 0 && i < 200) TRACE(i * 8 + 2);
     if (i >= 2 && !uniform_wait(&s.ds_free[b], ((i - 2) >> 1) & 1, 4)) {
       ok = false;
       break;
     }
-    uint8_t* dsrow = s.ds + b * C::DS_BYTES + tid * 128;
+    uint8_t* dsrow = s.ds + b * C::DS_BYTES + row * 128;
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-      *reinterpret_cast<uint4*>(dsrow + ((ch ^ (tid & 7)) * 16)) = dsk[ch];
+    for (int ch = 0; ch < 4; ++ch)
+      *reinterpret_cast<uint4*>(dsrow + (((wg * 4 + ch) ^ (row & 7)) * 16)) = dsk[ch];
     tmem_st_wait();
     fence_async_smem();
     tc_fence_before();
+    if (tid == 0 && i < 200) TRACE(i * 8 + 3);
     mbar_arrive(&s.ds_ready[b]);
     if (i >= 1 && !dq_out(i - 1)) {
       ok = false;
       break;
     }
+    if (tid == 0 && i < 200) TRACE(i * 8 + 4);
   }
   if (ok && t.n_iter > 0) ok = dq_out(t.n_iter - 1);
+  if constexpr (C::DQ_TMA) {
+    if (lane == 0) bulk_wait0();  // this warp's reduces are complete
+  }
   if (ok && t.n_iter > 0) ok = uniform_wait(s.dkv_full, 0, 5);
   if (!ok) return;
-  // dK (x scale) and dV rows of this CTA's half -> bf16.  The TMEM loads are
-  // warp-collective, so every lane runs them; only valid key rows store.
+  // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale), bf16.
+  // The TMEM loads are warp-collective, so every lane runs them; only valid
+  // key rows store.
   const size_t grow = static_cast<size_t>(t.k0 + (key_ok ? kr : 0));
   const size_t off = ((grow * p.nheads_kv + t.hk) * D + t.dh * C::DH) * 2;
+  uint8_t* dst = static_cast<uint8_t*>(wg ? p.dk : p.dv) + off;
+  const float f = wg ? p.scale : 1.f;
+  const int col0 = wg ? C::COL_DK : C::COL_DV;
 #pragma unroll 1
-  for (int which = 0; which < 2; ++which) {
-    uint8_t* dst = static_cast<uint8_t*>(which ? p.dk : p.dv) + off;
-    const float f = which ? p.scale : 1.f;
-    const int col0 = which ? C::COL_DK : C::COL_DV;
-#pragma unroll 1
-    for (int cc = 0; cc < C::DH / 32; ++cc) {
-      uint32_t r[32];
-      if (t.n_iter > 0) {
-        tmem_ld32(tmem + lane_base + col0 + cc * 32, r);
-        tmem_ld_wait(r);
-      } else {
+  for (int cc = 0; cc < C::DH / 32; ++cc) {
+    uint32_t r[32];
+    if (t.n_iter > 0) {
+      tmem_ld32(tmem + lane_base + col0 + cc * 32, r);
+      tmem_ld_wait(r);
+    } else {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) r[x] = 0u;
-      }
-      if (key_ok) {
+      for (int x = 0; x < 32; ++x) r[x] = 0u;
+    }
+    if (key_ok) {
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint4 v;
-          v.x = pack_bf16(__uint_as_float(r[g * 8 + 0]) * f, __uint_as_float(r[g * 8 + 1]) * f);
-          v.y = pack_bf16(__uint_as_float(r[g * 8 + 2]) * f, __uint_as_float(r[g * 8 + 3]) * f);
-          v.z = pack_bf16(__uint_as_float(r[g * 8 + 4]) * f, __uint_as_float(r[g * 8 + 5]) * f);
-          v.w = pack_bf16(__uint_as_float(r[g * 8 + 6]) * f, __uint_as_float(r[g * 8 + 7]) * f);
-          *reinterpret_cast<uint4*>(dst + (cc * 32 + g * 8) * 2) = v;
-        }
+      for (int g = 0; g < 4; ++g) {
+        uint4 v;
+        v.x = pack_bf16(__uint_as_float(r[g * 8 + 0]) * f, __uint_as_float(r[g * 8 + 1]) * f);
+        v.y = pack_bf16(__uint_as_float(r[g * 8 + 2]) * f, __uint_as_float(r[g * 8 + 3]) * f);
+        v.z = pack_bf16(__uint_as_float(r[g * 8 + 4]) * f, __uint_as_float(r[g * 8 + 5]) * f);
+        v.w = pack_bf16(__uint_as_float(r[g * 8 + 6]) * f, __uint_as_float(r[g * 8 + 7]) * f);
+        *reinterpret_cast<uint4*>(dst + (cc * 32 + g * 8) * 2) = v;
       }
     }
   }
@@ -508,7 +566,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmQ,
-                         const __grid_constant__ CUtensorMap tmO, const BwdParams p) {
+                         const __grid_constant__ CUtensorMap tmO,
+                         const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
@@ -525,21 +584,22 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.ds_ready[i], 128);
+      mbar_init(&s.ds_ready[i], C::ELEM_THREADS);
       mbar_init(&s.ds_free[i], 1);
     }
     mbar_init(s.dp_full, 1);
-    mbar_init(s.dp_free, 128);
+    mbar_init(s.dp_free, C::ELEM_THREADS);
     mbar_init(s.dq_full, 1);
-    mbar_init(s.dq_free, 128);
+    mbar_init(s.dq_free, C::ELEM_THREADS);
     mbar_init(s.dkv_full, 1);
     *s.abort = 0;
     fence_mbar_init();
   }
-  if (D == 64 && warp < 4) {
+  if (D == 64 && warp < 8) {
     // zero panel after the K tile: the dQ^T MMA reads head_dim 64 as M = 128
     uint4* z = reinterpret_cast<uint4*>(s.k + C::PANELS * C::KV_PANEL);
-    for (int i = threadIdx.x; i < C::KV_PANEL / 16; i += 128) z[i] = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < C::KV_PANEL / 16; i += C::ELEM_THREADS)
+      z[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
   }
   if (warp == C::LOAD_WARP && lane_id() == 0) {
@@ -556,8 +616,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s.tmem_base;
-  if (warp < 4) {
-    bwd_elem<D, CAUSAL>(p, t, s, tmem);
+  if (warp < 8) {
+    bwd_elem<D, CAUSAL>(p, t, s, tmem, &tmDQ);
   } else if (warp == C::LOAD_WARP) {
     bwd_load<D>(p, t, s, &tmK, &tmV, &tmQ, &tmO);
   } else {

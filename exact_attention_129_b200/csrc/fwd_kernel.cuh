@@ -289,6 +289,7 @@ template <int D>
 __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, const FwdSmem& s,
                                         uint32_t tmem) {
   using C = FwdCfg<D>;
+  TRACE_INIT();
   FwdMma<D> m(p, s, tmem);
   const int n = t.n_blocks;
   if (n == 0) return;
@@ -316,13 +317,17 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
                        p.timeout_ns))
           return;
         tc_fence_after();
+        if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 0);
         if (qt == 0 && !m.wait_tile(vb)) return;
+        if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 1);
         m.issue_pv(qt, qt, vb, j > 1);
         mma_commit(&s.o_ready[qt]);
         if (more) {
           if (qt == 0 && !m.wait_tile(kb)) return;
+          if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 2);
           m.issue_s(qt, qt, kb);
           mma_commit(&s.s_full[qt]);
+          if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 3);
         }
       }
       m.release_tile(vb);
@@ -384,6 +389,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   const int tile_row0 = t.m_base + qt * C::BM;
   const int mask_from = CAUSAL ? min(t.sk, tile_row0 + (t.sk - t.sq) + 1) : t.sk;
 
+  TRACE_INIT();
   float m_run = -INFINITY;  // running max, log2 domain
   float l_run = 0.f;
   bool ok = true;
@@ -397,28 +403,37 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       break;
     }
     tc_fence_after();
+    if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 0);
     const uint32_t s_addr = tmem + lane_base + slot * 128;
-    float sv[128];
-    {
-      uint32_t r[32];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        tmem_ld32(s_addr + cc * 32, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = __uint_as_float(r[i]);
-      }
-    }
+    uint32_t sr[128];  // the row's 128 scores (fp32 bits)
+    tmem_ld128(s_addr, sr);
+    tmem_ld_wait(sr);
+    if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 1);
     if ((j + 1) * C::BN > mask_from) {
       const int lim = key_lim - j * C::BN;
 #pragma unroll
       for (int i = 0; i < 128; ++i)
-        if (i >= lim) sv[i] = -INFINITY;
+        if (i >= lim) sr[i] = 0xff800000u;  // -inf
     }
-    float mx = sv[0];
+    // row max: 8 independent chains of three-input max, then a short tree
+    float mx;
+    {
+      float ch[8];
 #pragma unroll
-    for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
+      for (int k = 0; k < 8; ++k)
+        ch[k] = fmax3(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]),
+                      __uint_as_float(sr[k + 16]));
+#pragma unroll
+      for (int i = 24; i < 120; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          ch[k] = fmax3(ch[k], __uint_as_float(sr[i + k]), __uint_as_float(sr[i + 8 + k]));
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ch[k] = fmaxf(ch[k], __uint_as_float(sr[120 + k]));
+      mx = fmaxf(fmax3(ch[0], ch[1], ch[2]), fmax3(ch[3], ch[4], fmax3(ch[5], ch[6], ch[7])));
+    }
     const float m_new = fmaxf(m_run, mx * c);
+    if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 2);
     bool rescale = false;
     float alpha = 1.f;
     if (j == 0) {
@@ -430,23 +445,38 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       l_run *= alpha;
     }
     const float m_sub = (m_run == -INFINITY) ? 0.f : m_run;
-    // P = 2^(s*c - m), rounded to bf16 and written over the first 64 columns of S
-    float lsum = 0.f;
+    // P = 2^(s*c - m) on pairs (packed fp32x2 FMA), rounded to bf16 and written
+    // over the first 64 columns of S; the row sum uses 4 independent accumulators
+    float lsum;
     {
+      const uint64_t cc2 = f2_pack(c, c), mm2 = f2_pack(-m_sub, -m_sub);
+      uint64_t acc[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) acc[a] = 0ull;
       uint32_t pk[32];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(fmaf(sv[half * 64 + 2 * i], c, -m_sub));
-          const float p1 = ex2(fmaf(sv[half * 64 + 2 * i + 1], c, -m_sub));
-          lsum += p0 + p1;
+          const int col = half * 64 + 2 * i;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2,
+                           mm2),
+                    x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
           pk[i] = pack_bf16(p0, p1);
         }
         tmem_st32(s_addr + half * 32, pk);
       }
+      float a0, a1, a2, a3, a4, a5, a6, a7;
+      f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+      f2_unpack(f2_add(acc[2], acc[3]), a2, a3);
+      (void)a4; (void)a5; (void)a6; (void)a7;
+      lsum = (a0 + a1) + (a2 + a3);
     }
     l_run += lsum;
+    if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 3);
     if (__any_sync(0xffffffffu, rescale)) {
       // O must not be rescaled while the previous P.V MMA may still write it
       if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (j - 1) & 1, s.abort, p.err,
@@ -468,6 +498,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     }
     tmem_st_wait();
     tc_fence_before();
+    if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 4);
     mbar_arrive(&s.p_full[slot]);
   }
 
