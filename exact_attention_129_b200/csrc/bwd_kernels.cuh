@@ -93,7 +93,7 @@ struct BwdCfg {
   static constexpr int K_BYTES = PANELS * KV_PANEL + (D == 64 ? KV_PANEL : 0);  // + zero panel
   static constexpr int V_BYTES = PANELS * KV_PANEL;
   static constexpr int STAGE_BYTES = 2 * PANELS * QD_PANEL;  // Q_i then dO_i
-  static constexpr int NST = (D == 256) ? 1 : (D == 128 ? 3 : 4);
+  static constexpr int NST = (D == 256) ? 1 : (D == 128 ? 3 : 4);  // (Q, dO) stages
   static constexpr int DS_BYTES = BN * BM * 2;   // 16 KB
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + K_BYTES;
@@ -221,6 +221,26 @@ __device__ __forceinline__ void bwd_load(const BwdParams& p, const BwdTile& t, c
   }
   const int mcount = t.m_hi - t.m_lo;
   int issued = 0;
+  // LSE (log2 domain) and D_i for rows lane and lane + 32 of block i, loaded
+  // one block ahead so their global-memory latency overlaps the waits
+  auto fetch = [&](int i, float (&l2)[2], float (&dl)[2]) {
+    const int h = t.h0 + i / mcount;
+    const int m0 = (t.m_lo + i % mcount) * C::BM;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int qrow = m0 + lane + 32 * u;
+      l2[u] = INFINITY;  // rows outside the segment, or rows that saw no key: P = 0
+      dl[u] = 0.f;
+      if (qrow < t.sq) {
+        const size_t idx = static_cast<size_t>(h) * p.total_q + t.q0 + qrow;
+        const float l = p.lse[idx];
+        if (l != -INFINITY) l2[u] = l * 1.4426950408889634f;
+        dl[u] = p.delta[idx];
+      }
+    }
+  };
+  float nl2[2], ndl[2];
+  fetch(0, nl2, ndl);
   for (int i = 0; i < t.n_iter; ++i) {
     const int st = i % C::NST;
     if (i >= C::NST) {
@@ -231,20 +251,11 @@ __device__ __forceinline__ void bwd_load(const BwdParams& p, const BwdTile& t, c
     const int h = t.h0 + i / mcount;
     const int m0 = (t.m_lo + i % mcount) * C::BM;
     float* lsd = s.lsd + st * 128;
-#pragma unroll
-    for (int r = lane; r < C::BM; r += 32) {
-      const int qrow = m0 + r;
-      float l2 = INFINITY;  // rows outside the segment, or rows that saw no key: P = 0
-      float dl = 0.f;
-      if (qrow < t.sq) {
-        const size_t idx = static_cast<size_t>(h) * p.total_q + t.q0 + qrow;
-        const float l = p.lse[idx];
-        if (l != -INFINITY) l2 = l * 1.4426950408889634f;
-        dl = p.delta[idx];
-      }
-      lsd[r] = l2;
-      lsd[64 + r] = dl;
-    }
+    lsd[lane] = nl2[0];
+    lsd[lane + 32] = nl2[1];
+    lsd[64 + lane] = ndl[0];
+    lsd[64 + lane + 32] = ndl[1];
+    if (i + 1 < t.n_iter) fetch(i + 1, nl2, ndl);
     if (lane == 0) {
       uint8_t* dst = s.st + st * C::STAGE_BYTES;
       const int row = t.q0 + m0;
@@ -340,15 +351,17 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, co
   auto do_grads = [&](int j) -> bool {
     if (!m.wait(&s.ds_ready[j & 1], (j >> 1) & 1, 2)) return false;
     if (j < 200) TRACE(2048 + j * 8 + 4);
+    // dV and dK first: they are the last readers of the (Q, dO) stage, which is
+    // released right after them so the next load has the most slack
     m.grads(j, j == 0);
+    mma_commit(&s.qdo_empty[j % C::NST]);
     if (j < 200) TRACE(2048 + j * 8 + 5);
     if (j >= 1 && !m.wait(s.dq_free, (j - 1) & 1, 3)) return false;
     if (j < 200) TRACE(2048 + j * 8 + 6);
     m.dq(j);
-    if (j < 200) TRACE(2048 + j * 8 + 7);
     mma_commit(s.dq_full);
-    mma_commit(&s.qdo_empty[j % C::NST]);
-    mma_commit(&s.ds_free[j & 1]);
+    mma_commit(&s.ds_free[j & 1]);  // dK and dQ have read the dS buffer
+    if (j < 200) TRACE(2048 + j * 8 + 7);
     return true;
   };
   for (int i = 0; i < t.n_iter; ++i) {
@@ -416,7 +429,8 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     tmem_ld32(tmem + lane_base + C::COL_DQ + qc0, r0);
     tmem_ld_wait(r0);
     tc_fence_before();
-    mbar_arrive(s.dq_free);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.dq_free);
     if constexpr (C::DQ_TMA) {
       if (d_ok) {
         // slots: (DH / 32) per warpgroup; only warps with d < DH stage
@@ -465,7 +479,8 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     tmem_ld_wait(dr);
     tc_fence_before();
     if (tid == 0 && i < 200) TRACE(i * 8 + 1);
-    mbar_arrive(s.dp_free);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.dp_free);
     // causal: query column x of this block sees this key iff m0 + x >= kr - causal_off
     const int jmin = CAUSAL ? (kr - causal_off - m0 - qc0) : 0;
     uint32_t pk[16];
@@ -504,6 +519,7 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     // still be reading its own columns
     tmem_st16(tmem + lane_base + C::COL_S + b * 64 + wg * 32, pk);
     if (tid == 0 && i < 200) TRACE(i * 8 + 2);
+    // the dS buffer b is free once the dK and dQ MMAs of block i-2 are done
     if (i >= 2 && !uniform_wait(&s.ds_free[b], ((i - 2) >> 1) & 1, 4)) {
       ok = false;
       break;
@@ -516,7 +532,8 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     fence_async_smem();
     tc_fence_before();
     if (tid == 0 && i < 200) TRACE(i * 8 + 3);
-    mbar_arrive(&s.ds_ready[b]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.ds_ready[b]);
     if (i >= 1 && !dq_out(i - 1)) {
       ok = false;
       break;
@@ -584,13 +601,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.ds_ready[i], C::ELEM_THREADS);
+      mbar_init(&s.ds_ready[i], C::ELEM_THREADS / 32);
       mbar_init(&s.ds_free[i], 1);
     }
     mbar_init(s.dp_full, 1);
-    mbar_init(s.dp_free, C::ELEM_THREADS);
+    mbar_init(s.dp_free, C::ELEM_THREADS / 32);
     mbar_init(s.dq_full, 1);
-    mbar_init(s.dq_free, C::ELEM_THREADS);
+    mbar_init(s.dq_free, C::ELEM_THREADS / 32);
     mbar_init(s.dkv_full, 1);
     *s.abort = 0;
     fence_mbar_init();

@@ -312,18 +312,20 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
       const uint32_t vb = m.take();  // V_{j-1}
       const bool more = j < n;
       if (more) kb = m.take();       // K_j
+      // the tiles arrive long before the softmax is done: wait for them first so
+      // only the P barrier sits between the softmax and the next MMAs
+      if (!m.wait_tile(vb)) return;
+      if (more && !m.wait_tile(kb)) return;
       for (int qt = 0; qt < nq; ++qt) {
         if (!mbar_wait(&s.p_full[qt], (j - 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
                        p.timeout_ns))
           return;
         tc_fence_after();
         if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 0);
-        if (qt == 0 && !m.wait_tile(vb)) return;
         if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 1);
         m.issue_pv(qt, qt, vb, j > 1);
         mma_commit(&s.o_ready[qt]);
         if (more) {
-          if (qt == 0 && !m.wait_tile(kb)) return;
           if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 2);
           m.issue_s(qt, qt, kb);
           mma_commit(&s.s_full[qt]);
@@ -499,7 +501,8 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     tmem_st_wait();
     tc_fence_before();
     if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 4);
-    mbar_arrive(&s.p_full[slot]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.p_full[slot]);
   }
 
   // ---- epilogue: O / l -> bf16, staged through this tile's Q buffer ----
@@ -583,7 +586,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.p_full[i], 128);
+      mbar_init(&s.p_full[i], 4);  // one arrival per softmax warp
     }
     for (int i = 0; i < C::NQ; ++i) mbar_init(&s.o_ready[i], 1);
     *s.abort = 0;
