@@ -107,8 +107,11 @@ struct BwdCfg {
   static constexpr int OFF_DQS = OFF_LSD + NST * 128 * 4;
   static constexpr int OFF_BAR = OFF_DQS + (DQ_TMA ? 2 * (DH / 32) * DQ_WARP_BYTES : 0);
   // kv_full, qdo_full[NST], qdo_empty[NST], s_full[2], dp_full, dp_free,
-  // ds_ready[2], ds_free[2], dq_full, dq_free, dkv_full
-  static constexpr int NBAR = 1 + 2 * NST + 2 + 2 + 2 + 2 + 3;
+  // ds_ready[2], ds_free[2], dq_full, dq_free, dkv_full, oth_full, oth_empty
+  // (head_dim 256 splits its single stage: qdo_full/qdo_empty[0] track this
+  // CTA's own head_dim half of Q and dO plus the LSE/D vectors, oth_full /
+  // oth_empty the other half, which only S and dP read)
+  static constexpr int NBAR = 1 + 2 * NST + 2 + 2 + 2 + 2 + 3 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -128,7 +131,7 @@ struct BwdSmem {
   uint8_t *k, *v, *st, *ds, *dqs;
   float* lsd;
   uint64_t *kv_full, *qdo_full, *qdo_empty, *s_full, *dp_full, *dp_free, *ds_ready, *ds_free,
-      *dq_full, *dq_free, *dkv_full;
+      *dq_full, *dq_free, *dkv_full, *oth_full, *oth_empty;
   uint32_t* tmem_base;
   volatile int* abort;
 };
@@ -155,6 +158,8 @@ __device__ __forceinline__ BwdSmem bwd_smem(uint8_t* base) {
   s.dq_full = s.ds_free + 2;
   s.dq_free = s.dq_full + 1;
   s.dkv_full = s.dq_free + 1;
+  s.oth_full = s.dkv_full + 1;
+  s.oth_empty = s.oth_full + 1;
   s.tmem_base = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
   s.abort = reinterpret_cast<volatile int*>(base + C::OFF_MISC + 4);
   return s;
@@ -243,6 +248,25 @@ __device__ __forceinline__ void bwd_load(const BwdParams& p, const BwdTile& t, c
   fetch(0, nl2, ndl);
   for (int i = 0; i < t.n_iter; ++i) {
     const int st = i % C::NST;
+    if constexpr (C::NSPLIT == 2) {
+      // the other head_dim half of Q_i and dO_i: free once S and dP of block
+      // i-1 are done, long before the own half
+      if (i >= 1 && !__all_sync(0xffffffffu,
+                                mbar_wait(s.oth_empty, (i - 1) & 1, s.abort, p.err,
+                                          ERR_BWD_LOAD | 2, p.timeout_ns)))
+        break;
+      if (lane == 0) {
+        const int h = t.h0 + i / mcount;
+        const int row = t.q0 + (t.m_lo + i % mcount) * C::BM;
+        mbar_expect_tx(s.oth_full, 4 * C::QD_PANEL);
+        for (int pp = 0; pp < 2; ++pp) {
+          const int pn = 2 * (1 - t.dh) + pp;
+          tma_load_3d(s.st + pn * C::QD_PANEL, tmQ, s.oth_full, pn * 64, h, row);
+          tma_load_3d(s.st + (C::PANELS + pn) * C::QD_PANEL, tmO, s.oth_full, pn * 64, h, row);
+        }
+      }
+      __syncwarp();
+    }
     if (i >= C::NST) {
       if (!__all_sync(0xffffffffu, mbar_wait(&s.qdo_empty[st], ((i / C::NST) - 1) & 1, s.abort,
                                              p.err, ERR_BWD_LOAD | 1, p.timeout_ns)))
@@ -256,23 +280,42 @@ __device__ __forceinline__ void bwd_load(const BwdParams& p, const BwdTile& t, c
     lsd[64 + lane] = ndl[0];
     lsd[64 + lane + 32] = ndl[1];
     if (i + 1 < t.n_iter) fetch(i + 1, nl2, ndl);
-    if (lane == 0) {
-      uint8_t* dst = s.st + st * C::STAGE_BYTES;
-      const int row = t.q0 + m0;
-      mbar_expect_tx(&s.qdo_full[st], C::STAGE_BYTES);
-      for (int pn = 0; pn < C::PANELS; ++pn) {
-        tma_load_3d(dst + pn * C::QD_PANEL, tmQ, &s.qdo_full[st], pn * 64, h, row);
-        tma_load_3d(dst + (C::PANELS + pn) * C::QD_PANEL, tmO, &s.qdo_full[st], pn * 64, h,
-                    row);
+    if constexpr (C::NSPLIT == 2) {
+      // own head_dim half of Q_i and dO_i (with the LSE/D vectors above); the
+      // other half was issued earlier, as soon as S and dP of block i-1 ended
+      if (lane == 0) {
+        uint8_t* dst = s.st;
+        const int row = t.q0 + m0;
+        mbar_expect_tx(&s.qdo_full[0], 4 * C::QD_PANEL);
+        for (int pp = 0; pp < 2; ++pp) {
+          const int pn = 2 * t.dh + pp;
+          tma_load_3d(dst + pn * C::QD_PANEL, tmQ, &s.qdo_full[0], pn * 64, h, row);
+          tma_load_3d(dst + (C::PANELS + pn) * C::QD_PANEL, tmO, &s.qdo_full[0], pn * 64, h,
+                      row);
+        }
+      } else {
+        mbar_arrive(&s.qdo_full[0]);
       }
     } else {
-      mbar_arrive(&s.qdo_full[st]);
+      if (lane == 0) {
+        uint8_t* dst = s.st + st * C::STAGE_BYTES;
+        const int row = t.q0 + m0;
+        mbar_expect_tx(&s.qdo_full[st], C::STAGE_BYTES);
+        for (int pn = 0; pn < C::PANELS; ++pn) {
+          tma_load_3d(dst + pn * C::QD_PANEL, tmQ, &s.qdo_full[st], pn * 64, h, row);
+          tma_load_3d(dst + (C::PANELS + pn) * C::QD_PANEL, tmO, &s.qdo_full[st], pn * 64, h,
+                      row);
+        }
+      } else {
+        mbar_arrive(&s.qdo_full[st]);
+      }
     }
     ++issued;
   }
   if (*s.abort && lane == 0) {
     // let this CTA's own copies land before its shared memory is released
     mbar_wait_drain(s.kv_full, 0, 100000000ull);
+    if (C::NSPLIT == 2 && issued > 0) mbar_wait_drain(s.oth_full, (issued - 1) & 1, 100000000ull);
     for (int i = issued > C::NST ? issued - C::NST : 0; i < issued; ++i)
       mbar_wait_drain(&s.qdo_full[i % C::NST], (i / C::NST) & 1, 100000000ull);
   }
@@ -306,6 +349,18 @@ struct BwdMma {
         mma_ss(tmem + d_col, sdesc_sw128(aa + pn * C::KV_PANEL + kk * 32, 16, 1024),
                sdesc_sw128(ba + pn * C::QD_PANEL + kk * 32, 16, 1024), C::IDESC_SDP,
                (pn | kk) != 0);
+  }
+  // the K-steps of X^T = A B^T over panels [p0, p0 + 2) only (head_dim 256)
+  __device__ void issue_kt_pair(uint32_t d_col, const uint8_t* a, const uint8_t* b, int p0,
+                                bool first) {
+    const uint32_t aa = smem_u32(a), ba = smem_u32(b);
+#pragma unroll
+    for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tmem + d_col, sdesc_sw128(aa + (p0 + pp) * C::KV_PANEL + kk * 32, 16, 1024),
+               sdesc_sw128(ba + (p0 + pp) * C::QD_PANEL + kk * 32, 16, 1024), C::IDESC_SDP,
+               (!first || pp || kk) ? 1u : 0u);
   }
   __device__ void grads(int j, bool first) {
     const int bj = j & 1;
@@ -364,6 +419,41 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, co
     if (j < 200) TRACE(2048 + j * 8 + 7);
     return true;
   };
+  if constexpr (C::NSPLIT == 2) {
+    // head_dim 256: the stage's other head_dim half arrives early, so S_i and
+    // dP_i start on it while the own half (freed by the dV/dK MMAs of block
+    // i-1) is still loading; dQ of block i-1 fills the rest of that gap
+    auto grads_part = [&](int j) -> bool {
+      if (!m.wait(&s.ds_ready[j & 1], (j >> 1) & 1, 2)) return false;
+      m.grads(j, j == 0);
+      mma_commit(&s.qdo_empty[0]);
+      return true;
+    };
+    auto dq_part = [&](int j) -> bool {
+      if (j >= 1 && !m.wait(s.dq_free, (j - 1) & 1, 3)) return false;
+      m.dq(j);
+      mma_commit(s.dq_full);
+      mma_commit(&s.ds_free[j & 1]);
+      return true;
+    };
+    const int own = 2 * t.dh, oth = 2 * (1 - t.dh);
+    for (int i = 0; i < t.n_iter; ++i) {
+      if (i >= 1 && !grads_part(i - 1)) return;
+      if (!m.wait(s.oth_full, i & 1, 7)) return;
+      m.issue_kt_pair(C::COL_S + (i & 1) * 64, s.k, s.st, oth, true);
+      if (i >= 1 && !m.wait(s.dp_free, (i - 1) & 1, 5)) return;
+      m.issue_kt_pair(C::COL_DP, s.v, s.st + C::PANELS * C::QD_PANEL, oth, true);
+      if (i >= 1 && !dq_part(i - 1)) return;
+      if (!m.wait(&s.qdo_full[0], i & 1, 4)) return;
+      m.issue_kt_pair(C::COL_S + (i & 1) * 64, s.k, s.st, own, false);
+      mma_commit(&s.s_full[i & 1]);
+      m.issue_kt_pair(C::COL_DP, s.v, s.st + C::PANELS * C::QD_PANEL, own, false);
+      mma_commit(s.dp_full);
+      mma_commit(s.oth_empty);
+    }
+    if (!grads_part(t.n_iter - 1) || !dq_part(t.n_iter - 1)) return;
+    mma_commit(s.dkv_full);
+  } else {
   for (int i = 0; i < t.n_iter; ++i) {
     const int st = i % C::NST;
     // with a single (Q, dO) stage, block i can only be loaded once block i-1's
@@ -384,6 +474,7 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, co
   }
   if (!do_grads(t.n_iter - 1)) return;
   mma_commit(s.dkv_full);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -609,6 +700,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     mbar_init(s.dq_full, 1);
     mbar_init(s.dq_free, C::ELEM_THREADS / 32);
     mbar_init(s.dkv_full, 1);
+    mbar_init(s.oth_full, 1);
+    mbar_init(s.oth_empty, 1);
     *s.abort = 0;
     fence_mbar_init();
   }

@@ -303,6 +303,39 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
 }
 
 // ---------------------------------------------------------------------------
+// 2^x for a pair of fp32 values on the FMA pipe (no special-function unit):
+// x = n + f with n = round(x), |f| <= 1/2 (n is read off the low mantissa bits
+// of x + 1.5 * 2^23), 2^f ~ a degree-3 polynomial, and 2^n is applied by adding
+// n to the exponent field.  The polynomial minimises the maximum relative error
+// on [-1/2, 1/2] (a discrete minimax fit, exp2_poly_fit.py): 7.5e-5, far below
+// bf16 resolution.  x is clamped to >= -125 so 2^n stays a normal number;
+// results below 2^-125 come out as about 2^-125 instead of 0, so callers must
+// not use it where an exact 0 matters (masked, -inf scores).
+// ---------------------------------------------------------------------------
+namespace exp2poly {
+constexpr float kC0 = 0.99992806f, kC1 = 0.69326085f, kC2 = 0.24261115f, kC3 = 0.05517222f;
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+}  // namespace exp2poly
+
+__device__ __forceinline__ void exp2_fma_pair(uint64_t x2, float& r0, float& r1) {
+  using namespace exp2poly;
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t2 = f2_add(x2, f2_pack(kRound, kRound));
+  const uint64_t n2 = f2_add(t2, f2_pack(-kRound, -kRound));
+  const uint64_t f2 = f2_fma(n2, f2_pack(-1.f, -1.f), x2);
+  uint64_t p2 = f2_fma(f2_pack(kC3, kC3), f2, f2_pack(kC2, kC2));
+  p2 = f2_fma(p2, f2, f2_pack(kC1, kC1));
+  p2 = f2_fma(p2, f2, f2_pack(kC0, kC0));
+  float p0, p1, t0, t1;
+  f2_unpack(p2, p0, p1);
+  f2_unpack(t2, t0, t1);
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// ---------------------------------------------------------------------------
 // misc
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float ex2(float x) {
