@@ -159,7 +159,9 @@ def max_over_ranks(x: float, world: int, dev) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    # NCCL reduces device tensors; the gloo backend (CPU tests) host tensors
+    where = dev if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=where)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 

@@ -29,7 +29,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so"
 STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED",
           3: "ATTN_ERR_CUDA", 4: "ATTN_ERR_TIMEOUT", 5: "ATTN_ERR_SCRATCH_TOO_SMALL"}
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_last_device_error",
-            "attn_set_timing_events", "attn_bwd_static_scratch", "attn_version")
+            "attn_set_timing_events", "attn_bwd_static_scratch", "attn_watchdog_selftest",
+            "attn_version")
 KERNEL_FWD, KERNEL_BWD_MAIN = 0, 1
 
 
@@ -68,6 +69,8 @@ def library() -> ctypes.CDLL:
                                                 i32, i32, i32, i32, i32, f32, i32, vp, vp, vp,
                                                 vp]
         lib.attn_bwd_static_scratch.restype = ctypes.c_int
+        lib.attn_watchdog_selftest.argtypes = [i32, vp]
+        lib.attn_watchdog_selftest.restype = ctypes.c_int
         _lib = lib
     return _lib
 

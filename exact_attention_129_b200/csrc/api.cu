@@ -429,7 +429,8 @@ extern "C" attn_status_t attn_last_device_error(attn_stream_t stream, char* msg,
     return ATTN_OK;
   }
   static const char* kernels[] = {"?", "fwd load", "fwd mma", "fwd softmax", "bwd preprocess",
-                                  "bwd load", "bwd mma", "bwd softmax", "bwd dq convert"};
+                                  "bwd load", "bwd mma", "bwd softmax", "bwd dq convert",
+                                  "watchdog self-test"};
   const uint32_t kid = (word >> 8) & 0xff;
   char buf[128];
   std::snprintf(buf, sizeof(buf), "timed-out wait in %s (wait %u)",
@@ -452,5 +453,30 @@ extern "C" int attn_debug_set_trace(void* buf) {
   return cudaMemcpyToSymbol(g_attn_trace, &p, sizeof(p)) == cudaSuccess ? 0 : -1;
 }
 #endif
+
+namespace attn {
+// One thread waits on a barrier that is never arrived on; the bounded wait
+// runs out, records ERR_SELFTEST in the error word and returns.
+__global__ void attn_watchdog_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    mbar_wait(&bar, 0, &abort_flag, err, ERR_SELFTEST, timeout_ns);
+  }
+}
+}  // namespace attn
+
+extern "C" attn_status_t attn_watchdog_selftest(int32_t timeout_us, attn_stream_t stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  DeviceState* ds = device_state(&dev);
+  if (!ds) return ATTN_ERR_CUDA;
+  attn_watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      ds->err, static_cast<uint64_t>(timeout_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
 
 extern "C" const char* attn_version(void) { return "exact_attention_b200 0.1 sm_100a"; }

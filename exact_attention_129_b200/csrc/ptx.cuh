@@ -10,6 +10,9 @@
 
 namespace attn {
 
+// device error word code of the watchdog self-test (kernel id 9 << 8 | wait 1)
+constexpr uint32_t ERR_SELFTEST = 0x0901;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

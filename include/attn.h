@@ -201,6 +201,17 @@ attn_status_t attn_last_device_error(attn_stream_t stream, char* msg, size_t msg
 enum { ATTN_KERNEL_FWD = 0, ATTN_KERNEL_BWD_MAIN = 1 };
 attn_status_t attn_set_timing_events(int32_t kernel, void* start, void* stop);
 
+/*
+ * Watchdog self-test (diagnostic, not part of the computation): launches one
+ * CTA whose thread waits, through the same bounded wait every kernel uses, on a
+ * shared-memory barrier that nothing ever arrives on.  The wait gives up after
+ * timeout_us microseconds (1..1000000), records the give-up in the device error
+ * word and the kernel exits normally: nothing traps or hangs.  A following
+ * attn_last_device_error(stream, ...) then reports ATTN_ERR_TIMEOUT naming the
+ * self-test.  Returns ATTN_ERR_INVALID_ARG for an out-of-range timeout.
+ */
+attn_status_t attn_watchdog_selftest(int32_t timeout_us, attn_stream_t stream);
+
 /* Library version string, e.g. "exact_attention_b200 0.1 sm_100a". */
 const char* attn_version(void);
 

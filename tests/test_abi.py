@@ -91,3 +91,9 @@ def test_python_binding_refuses_cpu_tensors():
     cu = torch.tensor([0, 4], dtype=torch.int32)
     with pytest.raises(ValueError):
         ea.attn_fwd(q, q, q, cu, cu, 4, 4)
+
+
+def test_watchdog_selftest_rejects_bad_timeouts(lib):
+    # validated on the host, before any device call
+    assert lib.attn_watchdog_selftest(0, None) == 1
+    assert lib.attn_watchdog_selftest(2_000_000, None) == 1
