@@ -148,10 +148,16 @@ attn_status_t check_common(const void* q, const void* k, const void* v,
 }
 
 template <int D, bool CAUSAL>
-attn_status_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                         const FwdParams& p, int batch, int hq, int max_q,
+attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_q, int total_k,
+                         int hkv, const FwdParams& p, int batch, int hq, int max_q,
                          cudaStream_t stream) {
   using C = FwdCfg<D>;
+  // Q: one 128-row box per 64-column panel; K: one BN-row box per panel;
+  // V: VROWS rows per box, all panels of a chunk together
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, total_q, hq, D, C::BM) || !make_map(&mk, k, total_k, hkv, D, C::BN) ||
+      !make_map(&mv, v, total_k, hkv, D, C::VROWS))
+    return ATTN_ERR_CUDA;
   static std::once_flag attr_once[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -291,24 +297,18 @@ extern "C" attn_status_t attn_fwd(const void* q, const void* k, const void* v,
   p.return_lse = return_lse ? 1 : 0;
   p.timeout_ns = wait_timeout_ns();
 
-  CUtensorMap mq, mk, mv;
-  const int vrows = 8192 / head_dim;
-  if (!make_map(&mq, q, total_q, nheads_q, head_dim, 128) ||
-      !make_map(&mk, k, total_k, nheads_kv, head_dim, 128) ||
-      !make_map(&mv, v, total_k, nheads_kv, head_dim, vrows))
-    return ATTN_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool c = causal != 0;
+  auto run = [&](auto launch) {
+    return launch(q, k, v, total_q, total_k, nheads_kv, p, batch, nheads_q, max_seqlen_q, s);
+  };
   switch (head_dim) {
     case 64:
-      return c ? launch_fwd<64, true>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s)
-               : launch_fwd<64, false>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s);
+      return c ? run(launch_fwd<64, true>) : run(launch_fwd<64, false>);
     case 128:
-      return c ? launch_fwd<128, true>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s)
-               : launch_fwd<128, false>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s);
+      return c ? run(launch_fwd<128, true>) : run(launch_fwd<128, false>);
     default:
-      return c ? launch_fwd<256, true>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s)
-               : launch_fwd<256, false>(mq, mk, mv, p, batch, nheads_q, max_seqlen_q, s);
+      return c ? run(launch_fwd<256, true>) : run(launch_fwd<256, false>);
   }
 }
 

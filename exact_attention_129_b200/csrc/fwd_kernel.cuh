@@ -67,31 +67,45 @@ struct FwdParams {
 
 template <int D>
 struct FwdCfg {
+  // head_dim 64/128 (DBUF): two query tiles share every K/V block, blocks are 64
+  // keys and each tile double-buffers S, so S(j+1) is computed while the softmax
+  // works on S(j).  head_dim 256: one query tile, 128-key blocks, the two S slots
+  // double-buffer S (the 128 x 256 fp32 O fills half of tensor memory).
+  static constexpr bool DBUF = (D != 256);
   static constexpr int BM = 128;               // rows per query tile
-  static constexpr int BN = 128;               // keys per block
-  static constexpr int NQ = (D == 256) ? 1 : 2;
+  static constexpr int BN = DBUF ? 64 : 128;   // keys per block
+  static constexpr int NQ = DBUF ? 2 : 1;      // query tiles per CTA
+  static constexpr int NSS = DBUF ? 4 : 2;     // S slots (tile, buffer)
   static constexpr int PANELS = D / 64;        // 64-column (128-byte) panels per row
-  static constexpr int CHUNK = 16384;          // ring slot bytes
-  static constexpr int VROWS = 8192 / D;       // V key rows per chunk
+  static constexpr int QPANEL = BM * 128;      // 16 KB: 128 rows x 64 columns
+  static constexpr int CHUNK = BN * 128;       // ring slot: one K panel of BN rows
+  static constexpr int VROWS = CHUNK / (2 * D);  // V key rows per chunk (all D columns)
   static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int NSLOT = (D == 64) ? 12 : 10;
+  static constexpr int NSLOT = (D == 64) ? 24 : (D == 128 ? 20 : 10);
+  // ring barriers guard G chunks each: a whole K or V tile when the tile is
+  // small (fewer waits and commits per key), single chunks for head_dim 256
+  static constexpr int G = DBUF ? PANELS : 1;
+  static constexpr int NSTAGE = NSLOT / G;
   static constexpr int SOFTMAX_WARPS = 4 * NQ;
   static constexpr int LOAD_WARP = SOFTMAX_WARPS;
-  static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
-  static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 2);
+  static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;  // one MMA warp per query tile
+  static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 1 + NQ);
   static constexpr int TMEM_COLS = 512;
-  static constexpr int O_COL0 = 256;
+  static constexpr int O_COL0 = 256;           // S slots use columns [0, 256)
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
   static constexpr int OFF_BAR = OFF_RING + NSLOT * CHUNK;
-  // barriers: q_full[NQ] kv_full[NSLOT] kv_empty[NSLOT] s_full[2] p_full[2] o_ready[NQ]
-  static constexpr int NBAR = NQ + 2 * NSLOT + 2 + 2 + NQ;
+  // barriers: q_full[NQ] kv_full[NSTAGE] kv_empty[NSTAGE] s_full[NSS] p_full[NSS] o_ready[NQ]
+  static constexpr int NBAR = NQ + 2 * NSTAGE + 2 * NSS + NQ;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(NSS * BN <= O_COL0 && O_COL0 + NQ * D <= TMEM_COLS, "tensor memory budget");
+  static_assert(VROWS % 16 == 0 && BN % VROWS == 0 && BN / VROWS == PANELS, "V chunking");
+  static_assert(NSLOT % G == 0 && NSTAGE >= 2, "ring stages");
 };
 
 struct FwdSmem {
@@ -116,10 +130,10 @@ __device__ __forceinline__ FwdSmem fwd_smem(uint8_t* base) {
   uint64_t* b = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
   s.q_full = b;
   s.kv_full = b + C::NQ;
-  s.kv_empty = s.kv_full + C::NSLOT;
-  s.s_full = s.kv_empty + C::NSLOT;
-  s.p_full = s.s_full + 2;
-  s.o_ready = s.p_full + 2;
+  s.kv_empty = s.kv_full + C::NSTAGE;
+  s.s_full = s.kv_empty + C::NSTAGE;
+  s.p_full = s.s_full + C::NSS;
+  s.o_ready = s.p_full + C::NSS;
   s.tmem_base = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
   s.abort = reinterpret_cast<volatile int*>(base + C::OFF_MISC + 4);
   return s;
@@ -169,7 +183,7 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, c
     if (t.m_base + qt * C::BM >= t.sq) break;
     mbar_expect_tx(&s.q_full[qt], C::Q_BYTES);
     for (int pn = 0; pn < C::PANELS; ++pn)
-      tma_load_3d(s.q + qt * C::Q_BYTES + pn * C::CHUNK, tmQ, &s.q_full[qt], pn * 64, t.h,
+      tma_load_3d(s.q + qt * C::Q_BYTES + pn * C::QPANEL, tmQ, &s.q_full[qt], pn * 64, t.h,
                   t.q0 + t.m_base + qt * C::BM);
   }
   uint32_t ring = 0;
@@ -179,45 +193,41 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, c
     for (int qt = 0; qt < C::NQ; ++qt)
       if (t.m_base + qt * C::BM < t.sq) mbar_wait_drain(&s.q_full[qt], 0, 100000000ull);
     const uint32_t first = ring > (uint32_t)C::NSLOT ? ring - C::NSLOT : 0u;
-    for (uint32_t r = first; r < ring; ++r)
-      mbar_wait_drain(&s.kv_full[r % C::NSLOT], (r / C::NSLOT) & 1, 100000000ull);
+    for (uint32_t r = first; r < ring; r += C::G)
+      mbar_wait_drain(&s.kv_full[(r % C::NSLOT) / C::G], (r / C::NSLOT) & 1, 100000000ull);
   };
-  // one K or V tile = PANELS chunks
+  // one K or V tile = PANELS chunks; one ring barrier per G chunks
   auto load_tile = [&](bool is_v, int j) -> bool {
     for (int c = 0; c < C::PANELS; ++c, ++ring) {
       const uint32_t slot = ring % C::NSLOT;
-      if (ring >= (uint32_t)C::NSLOT) {
-        if (!mbar_wait(&s.kv_empty[slot], ((ring / C::NSLOT) - 1) & 1, s.abort, p.err,
-                       ERR_FWD_LOAD | 1, p.timeout_ns)) {
-          drain();
-          return false;
+      uint64_t* full = &s.kv_full[slot / C::G];
+      if (c % C::G == 0) {
+        if (ring >= (uint32_t)C::NSLOT) {
+          if (!mbar_wait(&s.kv_empty[slot / C::G], ((ring / C::NSLOT) - 1) & 1, s.abort, p.err,
+                         ERR_FWD_LOAD | 1, p.timeout_ns)) {
+            drain();
+            return false;
+          }
         }
+        mbar_expect_tx(full, C::G * C::CHUNK);
       }
       uint8_t* dst = s.ring + slot * C::CHUNK;
-      mbar_expect_tx(&s.kv_full[slot], C::CHUNK);
       const int row = t.k0 + j * C::BN;
       if (!is_v) {
-        tma_load_3d(dst, tmK, &s.kv_full[slot], c * 64, t.hk, row);
+        tma_load_3d(dst, tmK, full, c * 64, t.hk, row);
       } else {
         for (int pn = 0; pn < C::PANELS; ++pn)
-          tma_load_3d(dst + pn * (C::VROWS * 128), tmV, &s.kv_full[slot], pn * 64, t.hk,
-                      row + c * C::VROWS);
+          tma_load_3d(dst + pn * (C::VROWS * 128), tmV, full, pn * 64, t.hk, row + c * C::VROWS);
       }
     }
     return true;
   };
+  // consumption order of the MMA warp: K_0, then K_{j+1} before V_j
   const int n = t.n_blocks;
-  if (C::NQ == 2) {
-    for (int j = 0; j < n; ++j) {
-      if (!load_tile(false, j)) return;
-      if (!load_tile(true, j)) return;
-    }
-  } else {
-    if (n > 0 && !load_tile(false, 0)) return;
-    for (int j = 0; j < n; ++j) {
-      if (j + 1 < n && !load_tile(false, j + 1)) return;
-      if (!load_tile(true, j)) return;
-    }
+  if (n > 0 && !load_tile(false, 0)) return;
+  for (int j = 0; j < n; ++j) {
+    if (j + 1 < n && !load_tile(false, j + 1)) return;
+    if (!load_tile(true, j)) return;
   }
 }
 
@@ -241,9 +251,9 @@ struct FwdMma {
     return b;
   }
   __device__ bool wait_tile(uint32_t base) {
-    for (int c = 0; c < C::PANELS; ++c) {
+    for (int c = 0; c < C::PANELS; c += C::G) {
       const uint32_t r = base + c;
-      if (!mbar_wait(&s.kv_full[r % C::NSLOT], (r / C::NSLOT) & 1, s.abort, p.err,
+      if (!mbar_wait(&s.kv_full[(r % C::NSLOT) / C::G], (r / C::NSLOT) & 1, s.abort, p.err,
                      ERR_FWD_MMA | 1, p.timeout_ns))
         return false;
     }
@@ -251,18 +261,19 @@ struct FwdMma {
     return true;
   }
   __device__ void release_tile(uint32_t base) {
-    for (int c = 0; c < C::PANELS; ++c) mma_commit(&s.kv_empty[(base + c) % C::NSLOT]);
+    for (int c = 0; c < C::PANELS; c += C::G)
+      mma_commit(&s.kv_empty[((base + c) % C::NSLOT) / C::G]);
   }
   // S[slot] = Q[qt] . K^T
   __device__ void issue_s(int qt, int slot, uint32_t kbase) {
-    const uint32_t d_tmem = tmem + slot * 128;
+    const uint32_t d_tmem = tmem + slot * C::BN;
     const uint32_t qaddr = smem_u32(s.q + qt * C::Q_BYTES);
 #pragma unroll
     for (int c = 0; c < C::PANELS; ++c) {
       const uint32_t kaddr = smem_u32(s.ring + ((kbase + c) % C::NSLOT) * C::CHUNK);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = sdesc_sw128(qaddr + c * C::CHUNK + kk * 32, 16, 1024);
+        const uint64_t ad = sdesc_sw128(qaddr + c * C::QPANEL + kk * 32, 16, 1024);
         const uint64_t bd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
         mma_ss(d_tmem, ad, bd, C::IDESC_S, (c | kk) != 0);
       }
@@ -271,7 +282,7 @@ struct FwdMma {
   // O[qt] (+)= P[slot] . V
   __device__ void issue_pv(int qt, int slot, uint32_t vbase, bool accumulate) {
     const uint32_t d_tmem = tmem + C::O_COL0 + qt * D;
-    const uint32_t p_tmem = tmem + slot * 128;
+    const uint32_t p_tmem = tmem + slot * C::BN;
 #pragma unroll
     for (int c = 0; c < C::PANELS; ++c) {
       const uint32_t vaddr = smem_u32(s.ring + ((vbase + c) % C::NSLOT) * C::CHUNK);
@@ -287,53 +298,53 @@ struct FwdMma {
 
 template <int D>
 __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, const FwdSmem& s,
-                                        uint32_t tmem) {
+                                        uint32_t tmem, int qt) {
   using C = FwdCfg<D>;
   TRACE_INIT();
   FwdMma<D> m(p, s, tmem);
   const int n = t.n_blocks;
   if (n == 0) return;
-  int nq = 0;
-  for (int qt = 0; qt < C::NQ; ++qt)
-    if (t.m_base + qt * C::BM < t.sq) nq = qt + 1;
-  for (int qt = 0; qt < nq; ++qt)
-    if (!mbar_wait(&s.q_full[qt], 0, s.abort, p.err, ERR_FWD_MMA | 2, p.timeout_ns)) return;
+  if (!mbar_wait(&s.q_full[qt], 0, s.abort, p.err, ERR_FWD_MMA | 2, p.timeout_ns)) return;
   tc_fence_after();
 
-  if (C::NQ == 2) {
+  if constexpr (C::DBUF) {
+    // This warp serves query tile qt; the other tile has its own MMA warp, so
+    // one can issue while the other waits on a barrier.  Both read every K/V
+    // tile and both release it (the ring's empty barriers count one arrival per
+    // tile).  S of block j lives in slot 2qt + (j & 1); S(j+1) is issued before
+    // P(j).V so the tensor pipe has work while the softmax runs on S(j); the
+    // slot it overwrites held P(j-1), read by the P.V this thread issued one
+    // iteration earlier on the same in-order pipe.
     uint32_t kb = m.take();
     if (!m.wait_tile(kb)) return;
-    for (int qt = 0; qt < nq; ++qt) {
-      m.issue_s(qt, qt, kb);
-      mma_commit(&s.s_full[qt]);
-    }
+    m.issue_s(qt, 2 * qt, kb);
+    mma_commit(&s.s_full[2 * qt]);
     m.release_tile(kb);
-    for (int j = 1; j <= n; ++j) {
-      const uint32_t vb = m.take();  // V_{j-1}
-      const bool more = j < n;
-      if (more) kb = m.take();       // K_j
-      // the tiles arrive long before the softmax is done: wait for them first so
-      // only the P barrier sits between the softmax and the next MMAs
-      if (!m.wait_tile(vb)) return;
-      if (more && !m.wait_tile(kb)) return;
-      for (int qt = 0; qt < nq; ++qt) {
-        if (!mbar_wait(&s.p_full[qt], (j - 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
-                       p.timeout_ns))
-          return;
-        tc_fence_after();
-        if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 0);
-        if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 1);
-        m.issue_pv(qt, qt, vb, j > 1);
-        mma_commit(&s.o_ready[qt]);
-        if (more) {
-          if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 2);
-          m.issue_s(qt, qt, kb);
-          mma_commit(&s.s_full[qt]);
-          if (j < 64) TRACE(2048 + 16 * j + 4 * qt + 3);
-        }
+    for (int j = 0; j < n; ++j) {
+      const int b = j & 1;
+      [[maybe_unused]] const int tr = (j < 64) ? 2048 + 16 * j + 8 * qt : -1;
+      TRACE(tr);
+      if (j + 1 < n) {
+        kb = m.take();
+        if (!m.wait_tile(kb)) return;
+        TRACE(tr + 1);
+        m.issue_s(qt, 2 * qt + (b ^ 1), kb);
+        mma_commit(&s.s_full[2 * qt + (b ^ 1)]);
+        m.release_tile(kb);
+        TRACE(tr + 2);
       }
+      const uint32_t vb = m.take();
+      if (!m.wait_tile(vb)) return;
+      TRACE(tr + 3);
+      if (!mbar_wait(&s.p_full[2 * qt + b], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
+                     p.timeout_ns))
+        return;
+      tc_fence_after();
+      TRACE(tr + 4);
+      m.issue_pv(qt, 2 * qt + b, vb, j > 0);
+      mma_commit(&s.o_ready[qt]);
       m.release_tile(vb);
-      if (more) m.release_tile(kb);
+      TRACE(tr + 5);
     }
   } else {
     uint32_t kb = m.take();
@@ -396,9 +407,10 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   float l_run = 0.f;
   bool ok = true;
 
+  constexpr int NCOL = C::BN;  // scores per row and block
   for (int j = 0; j < n; ++j) {
-    const int slot = (C::NQ == 2) ? qt : (j & 1);
-    const uint32_t parity = (C::NQ == 2) ? (j & 1) : ((j >> 1) & 1);
+    const int slot = C::DBUF ? 2 * qt + (j & 1) : (j & 1);
+    const uint32_t parity = (j >> 1) & 1;
     if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], parity, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 1, p.timeout_ns))) {
       ok = false;
@@ -406,15 +418,16 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     }
     tc_fence_after();
     if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 0);
-    const uint32_t s_addr = tmem + lane_base + slot * 128;
-    uint32_t sr[128];  // the row's 128 scores (fp32 bits)
-    tmem_ld128(s_addr, sr);
+    const uint32_t s_addr = tmem + lane_base + slot * NCOL;
+    uint32_t sr[NCOL];  // the row's scores for this block (fp32 bits)
+    if constexpr (NCOL == 128) tmem_ld128(s_addr, sr);
+    else tmem_ld64(s_addr, sr);
     tmem_ld_wait(sr);
     if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 1);
     if ((j + 1) * C::BN > mask_from) {
       const int lim = key_lim - j * C::BN;
 #pragma unroll
-      for (int i = 0; i < 128; ++i)
+      for (int i = 0; i < NCOL; ++i)
         if (i >= lim) sr[i] = 0xff800000u;  // -inf
     }
     // row max: 8 independent chains of three-input max, then a short tree
@@ -425,13 +438,16 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       for (int k = 0; k < 8; ++k)
         ch[k] = fmax3(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]),
                       __uint_as_float(sr[k + 16]));
+      int i = 24;
 #pragma unroll
-      for (int i = 24; i < 120; i += 16)
+      for (; i + 16 <= NCOL - 8; i += 16)
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           ch[k] = fmax3(ch[k], __uint_as_float(sr[i + k]), __uint_as_float(sr[i + 8 + k]));
 #pragma unroll
-      for (int k = 0; k < 8; ++k) ch[k] = fmaxf(ch[k], __uint_as_float(sr[120 + k]));
+      for (; i < NCOL; i += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ch[k] = fmaxf(ch[k], __uint_as_float(sr[i + k]));
       mx = fmaxf(fmax3(ch[0], ch[1], ch[2]), fmax3(ch[3], ch[4], fmax3(ch[5], ch[6], ch[7])));
     }
     const float m_new = fmaxf(m_run, mx * c);
@@ -448,7 +464,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     }
     const float m_sub = (m_run == -INFINITY) ? 0.f : m_run;
     // P = 2^(s*c - m) on pairs (packed fp32x2 FMA), rounded to bf16 and written
-    // over the first 64 columns of S; the row sum uses 4 independent accumulators
+    // over the first NCOL/2 columns of S; the row sum uses 4 independent accumulators
     float lsum;
     {
       const uint64_t cc2 = f2_pack(c, c), mm2 = f2_pack(-m_sub, -m_sub);
@@ -457,7 +473,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       for (int a = 0; a < 4; ++a) acc[a] = 0ull;
       uint32_t pk[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < NCOL / 64; ++half) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int col = half * 64 + 2 * i;
@@ -471,10 +487,9 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
         }
         tmem_st32(s_addr + half * 32, pk);
       }
-      float a0, a1, a2, a3, a4, a5, a6, a7;
+      float a0, a1, a2, a3;
       f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
       f2_unpack(f2_add(acc[2], acc[3]), a2, a3);
-      (void)a4; (void)a5; (void)a6; (void)a7;
       lsum = (a0 + a1) + (a2 + a3);
     }
     l_run += lsum;
@@ -510,6 +525,14 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
   uint8_t* stage = s.q + qt * C::Q_BYTES;
   constexpr int CPR = D / 8;  // 16-byte chunks per row
+  // The last S this warpgroup read was issued before the second-to-last P.V, so
+  // that P.V may still be running: wait for its phase first, then the last one
+  // (a single parity wait could match a phase two behind).
+  if (ok && n > 1) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (n - 2) & 1, s.abort, p.err,
+                                           ERR_FWD_SOFTMAX | 3, p.timeout_ns)))
+      ok = false;
+  }
   if (ok && n > 0) {
     if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (n - 1) & 1, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 3, p.timeout_ns)))
@@ -580,11 +603,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NQ; ++i) mbar_init(&s.q_full[i], 1);
-    for (int i = 0; i < C::NSLOT; ++i) {
+    // every MMA warp with a query tile releases each ring stage once
+    const int n_mma = (t.m_base + C::BM < t.sq && C::NQ == 2) ? 2 : 1;
+    for (int i = 0; i < C::NSTAGE; ++i) {
       mbar_init(&s.kv_full[i], 1);
-      mbar_init(&s.kv_empty[i], 1);
+      mbar_init(&s.kv_empty[i], n_mma);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NSS; ++i) {
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.p_full[i], 4);  // one arrival per softmax warp
     }
@@ -611,8 +636,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     if (t.m_base + qt * C::BM < t.sq) fwd_softmax<D, CAUSAL>(p, t, s, tmem, qt);
   } else if (warp == C::LOAD_WARP) {
     if (lane_id() == 0) fwd_load<D>(p, t, s, &tmQ, &tmK, &tmV);
-  } else if (warp == C::MMA_WARP) {
-    if (lane_id() == 0) fwd_mma<D>(p, t, s, tmem);
+  } else {
+    const int qt = warp - C::MMA_WARP;
+    if (lane_id() == 0 && t.m_base + qt * C::BM < t.sq) fwd_mma<D>(p, t, s, tmem, qt);
     __syncwarp();
   }
   tc_fence_before();
