@@ -39,8 +39,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx.cuh"
+
+// pairs out of every 8 whose 2^x runs on the FMA pipe in unmasked blocks
+#ifndef ATTN_FWD_POLY_PAIRS
+#define ATTN_FWD_POLY_PAIRS 0
+#endif
 
 namespace attn {
 
@@ -82,9 +88,10 @@ struct FwdCfg {
   static constexpr int VROWS = CHUNK / (2 * D);  // V key rows per chunk (all D columns)
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int NSLOT = (D == 64) ? 24 : (D == 128 ? 20 : 10);
-  // ring barriers guard G chunks each: a whole K or V tile when the tile is
-  // small (fewer waits and commits per key), single chunks for head_dim 256
-  static constexpr int G = DBUF ? PANELS : 1;
+  // ring barriers guard stages of G chunks.  DBUF: stage j holds K_j and
+  // V_{j-1} (exactly what one MMA iteration consumes), so each iteration waits
+  // on and releases one barrier.  head_dim 256: one chunk per stage.
+  static constexpr int G = DBUF ? 2 * PANELS : 1;
   static constexpr int NSTAGE = NSLOT / G;
   static constexpr int SOFTMAX_WARPS = 4 * NQ;
   static constexpr int LOAD_WARP = SOFTMAX_WARPS;
@@ -186,48 +193,71 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, c
       tma_load_3d(s.q + qt * C::Q_BYTES + pn * C::QPANEL, tmQ, &s.q_full[qt], pn * 64, t.h,
                   t.q0 + t.m_base + qt * C::BM);
   }
-  uint32_t ring = 0;
+  uint32_t ring = 0;  // stages issued so far
   // on the way out after a timed-out wait elsewhere: let every copy this CTA
   // issued land before its shared memory is released
   auto drain = [&]() {
     for (int qt = 0; qt < C::NQ; ++qt)
       if (t.m_base + qt * C::BM < t.sq) mbar_wait_drain(&s.q_full[qt], 0, 100000000ull);
-    const uint32_t first = ring > (uint32_t)C::NSLOT ? ring - C::NSLOT : 0u;
-    for (uint32_t r = first; r < ring; r += C::G)
-      mbar_wait_drain(&s.kv_full[(r % C::NSLOT) / C::G], (r / C::NSLOT) & 1, 100000000ull);
+    const uint32_t first = ring > (uint32_t)C::NSTAGE ? ring - C::NSTAGE : 0u;
+    for (uint32_t r = first; r < ring; ++r)
+      mbar_wait_drain(&s.kv_full[r % C::NSTAGE], (r / C::NSTAGE) & 1, 100000000ull);
   };
-  // one K or V tile = PANELS chunks; one ring barrier per G chunks
-  auto load_tile = [&](bool is_v, int j) -> bool {
-    for (int c = 0; c < C::PANELS; ++c, ++ring) {
-      const uint32_t slot = ring % C::NSLOT;
-      uint64_t* full = &s.kv_full[slot / C::G];
-      if (c % C::G == 0) {
-        if (ring >= (uint32_t)C::NSLOT) {
-          if (!mbar_wait(&s.kv_empty[slot / C::G], ((ring / C::NSLOT) - 1) & 1, s.abort, p.err,
-                         ERR_FWD_LOAD | 1, p.timeout_ns)) {
-            drain();
-            return false;
-          }
-        }
-        mbar_expect_tx(full, C::G * C::CHUNK);
-      }
-      uint8_t* dst = s.ring + slot * C::CHUNK;
-      const int row = t.k0 + j * C::BN;
-      if (!is_v) {
-        tma_load_3d(dst, tmK, full, c * 64, t.hk, row);
-      } else {
-        for (int pn = 0; pn < C::PANELS; ++pn)
-          tma_load_3d(dst + pn * (C::VROWS * 128), tmV, full, pn * 64, t.hk, row + c * C::VROWS);
-      }
+  // claim the next stage (waiting for the MMA warps to release its last use)
+  // and announce the bytes that will land in it
+  auto claim = [&](uint32_t bytes, uint8_t*& base, uint64_t*& full) -> bool {
+    const uint32_t st = ring % C::NSTAGE;
+    if (ring >= (uint32_t)C::NSTAGE &&
+        !mbar_wait(&s.kv_empty[st], ((ring / C::NSTAGE) - 1) & 1, s.abort, p.err,
+                   ERR_FWD_LOAD | 1, p.timeout_ns)) {
+      drain();
+      return false;
     }
+    full = &s.kv_full[st];
+    base = s.ring + st * (C::G * C::CHUNK);
+    mbar_expect_tx(full, bytes);
+    ++ring;
     return true;
   };
-  // consumption order of the MMA warp: K_0, then K_{j+1} before V_j
+  // K block j: one chunk per 64-column panel (BN rows, K-major)
+  auto load_k = [&](uint8_t* dst, uint64_t* full, int j, int c) {
+    tma_load_3d(dst, tmK, full, c * 64, t.hk, t.k0 + j * C::BN);
+  };
+  // rows [c*VROWS, (c+1)*VROWS) of V block j: all D columns, panel by panel
+  auto load_v = [&](uint8_t* dst, uint64_t* full, int j, int c) {
+    for (int pn = 0; pn < C::PANELS; ++pn)
+      tma_load_3d(dst + pn * (C::VROWS * 128), tmV, full, pn * 64, t.hk,
+                  t.k0 + j * C::BN + c * C::VROWS);
+  };
   const int n = t.n_blocks;
-  if (n > 0 && !load_tile(false, 0)) return;
-  for (int j = 0; j < n; ++j) {
-    if (j + 1 < n && !load_tile(false, j + 1)) return;
-    if (!load_tile(true, j)) return;
+  uint8_t* base;
+  uint64_t* full;
+  if constexpr (C::DBUF) {
+    // stage j = (K_j, V_{j-1}); the first holds only K_0, the last only V_{n-1}
+    for (int j = 0; j <= n; ++j) {
+      const uint32_t bytes = ((j < n) ? C::PANELS * C::CHUNK : 0) + ((j > 0) ? C::PANELS * C::CHUNK : 0);
+      if (!claim(bytes, base, full)) return;
+      for (int c = 0; c < C::PANELS; ++c) {
+        if (j < n) load_k(base + c * C::CHUNK, full, j, c);
+        if (j > 0) load_v(base + (C::PANELS + c) * C::CHUNK, full, j - 1, c);
+      }
+    }
+  } else {
+    // one chunk per stage, in the MMA warp's order: K_0, K_1, then V_j before K_{j+2}
+    auto load_tile = [&](bool is_v, int j) -> bool {
+      for (int c = 0; c < C::PANELS; ++c) {
+        if (!claim(C::CHUNK, base, full)) return false;
+        if (is_v) load_v(base, full, j, c);
+        else load_k(base, full, j, c);
+      }
+      return true;
+    };
+    if (n > 0 && !load_tile(false, 0)) return;
+    if (n > 1 && !load_tile(false, 1)) return;
+    for (int j = 0; j < n; ++j) {
+      if (!load_tile(true, j)) return;
+      if (j + 2 < n && !load_tile(false, j + 2)) return;
+    }
   }
 }
 
@@ -240,57 +270,75 @@ struct FwdMma {
   const FwdParams& p;
   const FwdSmem& s;
   uint32_t tmem;
-  uint32_t ring = 0;
+  uint32_t stage = 0, phase = 0;  // next ring stage to consume and its parity
+  // descriptors of chunk 0 of the ring (K-major K, MN-major V) and of Q tile 0;
+  // the start-address field is the low 14 bits, so an offset of b bytes inside
+  // shared memory is added as b / 16 without carrying into other fields
+  uint64_t kdesc0, vdesc0, qdesc0;
 
   __device__ FwdMma(const FwdParams& p_, const FwdSmem& s_, uint32_t tmem_)
-      : p(p_), s(s_), tmem(tmem_) {}
-
-  __device__ uint32_t take() {
-    const uint32_t b = ring;
-    ring += C::PANELS;
-    return b;
+      : p(p_), s(s_), tmem(tmem_) {
+    kdesc0 = sdesc_sw128(smem_u32(s.ring), 16, 1024);
+    vdesc0 = sdesc_sw128(smem_u32(s.ring), C::VROWS * 128, 1024);
+    qdesc0 = sdesc_sw128(smem_u32(s.q), 16, 1024);
   }
-  __device__ bool wait_tile(uint32_t base) {
-    for (int c = 0; c < C::PANELS; c += C::G) {
-      const uint32_t r = base + c;
-      if (!mbar_wait(&s.kv_full[(r % C::NSLOT) / C::G], (r / C::NSLOT) & 1, s.abort, p.err,
-                     ERR_FWD_MMA | 1, p.timeout_ns))
+
+  // wait for the next `count` stages; returns the first one's chunk index
+  __device__ bool wait_stages(int count, uint32_t& first_chunk) {
+    first_chunk = stage * C::G;
+    uint32_t st = stage, ph = phase;
+    for (int i = 0; i < count; ++i) {
+      if (!mbar_wait(&s.kv_full[st], ph, s.abort, p.err, ERR_FWD_MMA | 1, p.timeout_ns))
         return false;
+      if (++st == (uint32_t)C::NSTAGE) {
+        st = 0;
+        ph ^= 1u;
+      }
     }
     tc_fence_after();
     return true;
   }
-  __device__ void release_tile(uint32_t base) {
-    for (int c = 0; c < C::PANELS; c += C::G)
-      mma_commit(&s.kv_empty[((base + c) % C::NSLOT) / C::G]);
-  }
-  // S[slot] = Q[qt] . K^T
-  __device__ void issue_s(int qt, int slot, uint32_t kbase) {
-    const uint32_t d_tmem = tmem + slot * C::BN;
-    const uint32_t qaddr = smem_u32(s.q + qt * C::Q_BYTES);
-#pragma unroll
-    for (int c = 0; c < C::PANELS; ++c) {
-      const uint32_t kaddr = smem_u32(s.ring + ((kbase + c) % C::NSLOT) * C::CHUNK);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = sdesc_sw128(qaddr + c * C::QPANEL + kk * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
-        mma_ss(d_tmem, ad, bd, C::IDESC_S, (c | kk) != 0);
+  // release the next `count` stages once the MMAs issued so far have read them
+  __device__ void release_stages(int count) {
+    for (int i = 0; i < count; ++i) {
+      mma_commit(&s.kv_empty[stage]);
+      if (++stage == (uint32_t)C::NSTAGE) {
+        stage = 0;
+        phase ^= 1u;
       }
     }
   }
-  // O[qt] (+)= P[slot] . V
-  __device__ void issue_pv(int qt, int slot, uint32_t vbase, bool accumulate) {
+  __device__ static uint32_t wrap(uint32_t chunk) {
+    if constexpr (C::G == 1) {
+      if (chunk >= (uint32_t)C::NSLOT) chunk -= C::NSLOT;
+    }
+    return chunk;
+  }
+  // S[slot] = Q[qt] . K^T, K panel c in ring chunk ch0 + c
+  __device__ void issue_s(int qt, int slot, uint32_t ch0) {
+    const uint32_t d_tmem = tmem + slot * C::BN;
+    const uint64_t qd = qdesc0 + (uint64_t)(qt * (C::Q_BYTES >> 4));
+#pragma unroll
+    for (int c = 0; c < C::PANELS; ++c) {
+      const uint64_t kd = kdesc0 + (uint64_t)(wrap(ch0 + c) * (C::CHUNK >> 4));
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)  // 16 columns (32 bytes) of the panel per step
+        mma_ss(d_tmem, qd + (c * (C::QPANEL >> 4) + kk * 2), kd + kk * 2, C::IDESC_S,
+               (c | kk) != 0);
+    }
+  }
+  // O[qt] (+)= P[slot] . V, V rows [c*VROWS, (c+1)*VROWS) in ring chunk ch0 + c
+  __device__ void issue_pv(int qt, int slot, uint32_t ch0, bool accumulate) {
     const uint32_t d_tmem = tmem + C::O_COL0 + qt * D;
     const uint32_t p_tmem = tmem + slot * C::BN;
 #pragma unroll
     for (int c = 0; c < C::PANELS; ++c) {
-      const uint32_t vaddr = smem_u32(s.ring + ((vbase + c) % C::NSLOT) * C::CHUNK);
+      const uint64_t vd = vdesc0 + (uint64_t)(wrap(ch0 + c) * (C::CHUNK >> 4));
 #pragma unroll
       for (int kk = 0; kk < C::VROWS / 16; ++kk) {
-        const int kstep = c * (C::VROWS / 16) + kk;  // 16 keys per step
-        const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, C::VROWS * 128, 1024);
-        mma_ts(d_tmem, p_tmem + kstep * 8, bd, C::IDESC_O, (accumulate || kstep) ? 1u : 0u);
+        const int kstep = c * (C::VROWS / 16) + kk;  // 16 keys (2048 bytes of V) per step
+        mma_ts(d_tmem, p_tmem + kstep * 8, vd + kk * 128, C::IDESC_O,
+               (accumulate || kstep) ? 1u : 0u);
       }
     }
   }
@@ -309,73 +357,68 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
 
   if constexpr (C::DBUF) {
     // This warp serves query tile qt; the other tile has its own MMA warp, so
-    // one can issue while the other waits on a barrier.  Both read every K/V
-    // tile and both release it (the ring's empty barriers count one arrival per
+    // one can issue while the other waits on a barrier.  Both read every ring
+    // stage and both release it (the empty barriers count one arrival per
     // tile).  S of block j lives in slot 2qt + (j & 1); S(j+1) is issued before
     // P(j).V so the tensor pipe has work while the softmax runs on S(j); the
     // slot it overwrites held P(j-1), read by the P.V this thread issued one
-    // iteration earlier on the same in-order pipe.
-    uint32_t kb = m.take();
-    if (!m.wait_tile(kb)) return;
-    m.issue_s(qt, 2 * qt, kb);
+    // iteration earlier on the same in-order pipe.  Stage j holds K_j in its
+    // first PANELS chunks and V_{j-1} in the next PANELS.
+    uint32_t ch;
+    if (!m.wait_stages(1, ch)) return;
+    m.issue_s(qt, 2 * qt, ch);
     mma_commit(&s.s_full[2 * qt]);
-    m.release_tile(kb);
+    m.release_stages(1);
     for (int j = 0; j < n; ++j) {
       const int b = j & 1;
       [[maybe_unused]] const int tr = (j < 64) ? 2048 + 16 * j + 8 * qt : -1;
       TRACE(tr);
+      if (!m.wait_stages(1, ch)) return;
+      TRACE(tr + 1);
       if (j + 1 < n) {
-        kb = m.take();
-        if (!m.wait_tile(kb)) return;
-        TRACE(tr + 1);
-        m.issue_s(qt, 2 * qt + (b ^ 1), kb);
+        m.issue_s(qt, 2 * qt + (b ^ 1), ch);
         mma_commit(&s.s_full[2 * qt + (b ^ 1)]);
-        m.release_tile(kb);
-        TRACE(tr + 2);
       }
-      const uint32_t vb = m.take();
-      if (!m.wait_tile(vb)) return;
-      TRACE(tr + 3);
+      TRACE(tr + 2);
       if (!mbar_wait(&s.p_full[2 * qt + b], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
                      p.timeout_ns))
         return;
       tc_fence_after();
-      TRACE(tr + 4);
-      m.issue_pv(qt, 2 * qt + b, vb, j > 0);
+      TRACE(tr + 3);
+      m.issue_pv(qt, 2 * qt + b, ch + C::PANELS, j > 0);
       mma_commit(&s.o_ready[qt]);
-      m.release_tile(vb);
-      TRACE(tr + 5);
+      m.release_stages(1);
+      TRACE(tr + 4);
     }
   } else {
-    uint32_t kb = m.take();
-    if (!m.wait_tile(kb)) return;
-    m.issue_s(0, 0, kb);
+    // one query tile, two S slots alternating over key blocks; one chunk per stage
+    constexpr int P = C::PANELS;
+    uint32_t ch;
+    if (!m.wait_stages(P, ch)) return;
+    m.issue_s(0, 0, ch);
     mma_commit(&s.s_full[0]);
-    m.release_tile(kb);
+    m.release_stages(P);
     if (n > 1) {
-      kb = m.take();
-      if (!m.wait_tile(kb)) return;
-      m.issue_s(0, 1, kb);
+      if (!m.wait_stages(P, ch)) return;
+      m.issue_s(0, 1, ch);
       mma_commit(&s.s_full[1]);
-      m.release_tile(kb);
+      m.release_stages(P);
     }
     for (int j = 0; j < n; ++j) {
       const int slot = j & 1;
-      const uint32_t vb = m.take();
       if (!mbar_wait(&s.p_full[slot], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
                      p.timeout_ns))
         return;
       tc_fence_after();
-      if (!m.wait_tile(vb)) return;
-      m.issue_pv(0, slot, vb, j > 0);
+      if (!m.wait_stages(P, ch)) return;
+      m.issue_pv(0, slot, ch, j > 0);
       mma_commit(&s.o_ready[0]);
-      m.release_tile(vb);
+      m.release_stages(P);
       if (j + 2 < n) {
-        kb = m.take();
-        if (!m.wait_tile(kb)) return;
-        m.issue_s(0, slot, kb);
+        if (!m.wait_stages(P, ch)) return;
+        m.issue_s(0, slot, ch);
         mma_commit(&s.s_full[slot]);
-        m.release_tile(kb);
+        m.release_stages(P);
       }
     }
   }
@@ -402,6 +445,26 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   const int tile_row0 = t.m_base + qt * C::BM;
   const int mask_from = CAUSAL ? min(t.sk, tile_row0 + (t.sk - t.sq) + 1) : t.sk;
 
+  // With two query tiles, warp w of each tile shares an SM sub-partition and
+  // its special-function unit: their exp phases take turns (tile 0 first in
+  // each block) through a pair of named barriers, so one warp's loads, max and
+  // stores overlap the other's exps.  A warp that gives up on a timed-out wait
+  // still plays its remaining turns, so its partner never waits forever.
+  const bool pingpong = C::DBUF && (t.m_base + C::BM < t.sq);
+  const int bar_t0 = 3 + 2 * warp, bar_t1 = 4 + 2 * warp;  // "tile 0 / tile 1 may start"
+  auto turn_begin = [&](int k) {
+    if (qt == 0) {
+      if (k > 0) named_bar_sync(bar_t0, 64);
+    } else {
+      named_bar_sync(bar_t1, 64);
+    }
+  };
+  auto turn_end = [&](int k) {
+    if (qt == 0) named_bar_arrive(bar_t1, 64);
+    else if (k + 1 < n) named_bar_arrive(bar_t0, 64);
+  };
+  int turns_done = 0;
+
   TRACE_INIT();
   float m_run = -INFINITY;  // running max, log2 domain
   float l_run = 0.f;
@@ -414,6 +477,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], parity, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 1, p.timeout_ns))) {
       ok = false;
+      turns_done = j;
       break;
     }
     tc_fence_after();
@@ -424,7 +488,8 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     else tmem_ld64(s_addr, sr);
     tmem_ld_wait(sr);
     if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 1);
-    if ((j + 1) * C::BN > mask_from) {
+    const bool masked = (j + 1) * C::BN > mask_from;
+    if (masked) {
       const int lim = key_lim - j * C::BN;
 #pragma unroll
       for (int i = 0; i < NCOL; ++i)
@@ -464,29 +529,48 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     }
     const float m_sub = (m_run == -INFINITY) ? 0.f : m_run;
     // P = 2^(s*c - m) on pairs (packed fp32x2 FMA), rounded to bf16 and written
-    // over the first NCOL/2 columns of S; the row sum uses 4 independent accumulators
+    // over the first NCOL/2 columns of S; the row sum uses 4 independent
+    // accumulators.  With two query tiles, two softmax warps share each SM
+    // sub-partition and the special-function unit (ex2) becomes the limit, so in
+    // blocks without masked scores ATTN_FWD_POLY_PAIRS of every 8 pairs take 2^x on the FMA pipe
+    // (exp2_fma_pair); masked blocks keep ex2 everywhere so -inf gives exactly 0.
     float lsum;
     {
       const uint64_t cc2 = f2_pack(c, c), mm2 = f2_pack(-m_sub, -m_sub);
       uint64_t acc[4];
 #pragma unroll
       for (int a = 0; a < 4; ++a) acc[a] = 0ull;
-      uint32_t pk[32];
+      auto exp_rows = [&](auto use_poly) {
+        constexpr bool POLY = decltype(use_poly)::value;
+        uint32_t pk[32];
 #pragma unroll
-      for (int half = 0; half < NCOL / 64; ++half) {
+        for (int half = 0; half < NCOL / 64; ++half) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = half * 64 + 2 * i;
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2,
-                           mm2),
-                    x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
-          acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-          pk[i] = pack_bf16(p0, p1);
+          for (int i = 0; i < 32; ++i) {
+            const int col = half * 64 + 2 * i;
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2, mm2);
+            float p0, p1;
+            if (POLY && (i & 7) < ATTN_FWD_POLY_PAIRS) {
+              exp2_fma_pair(x2, p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st32(s_addr + half * 32, pk);
         }
-        tmem_st32(s_addr + half * 32, pk);
-      }
+      };
+      if (pingpong) turn_begin(j);
+      if (C::DBUF && !masked)
+        exp_rows(std::integral_constant<bool, true>());
+      else
+        exp_rows(std::integral_constant<bool, false>());
+      if (pingpong) turn_end(j);
       float a0, a1, a2, a3;
       f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
       f2_unpack(f2_add(acc[2], acc[3]), a2, a3);
@@ -499,6 +583,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (j - 1) & 1, s.abort, p.err,
                                              ERR_FWD_SOFTMAX | 2, p.timeout_ns))) {
         ok = false;
+        turns_done = j + 1;
         break;
       }
       tc_fence_after();
@@ -518,7 +603,13 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 4);
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.p_full[slot]);
+    turns_done = j + 1;
   }
+  if (pingpong)
+    for (int k = turns_done; k < n; ++k) {
+      turn_begin(k);
+      turn_end(k);
+    }
 
   // ---- epilogue: O / l -> bf16, staged through this tile's Q buffer ----
   const bool row_valid = row < t.sq;
