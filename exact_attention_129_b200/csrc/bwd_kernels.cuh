@@ -111,15 +111,18 @@ struct BwdCfg {
   // (head_dim 256 splits its single stage: qdo_full/qdo_empty[0] track this
   // CTA's own head_dim half of Q and dO plus the LSE/D vectors, oth_full /
   // oth_empty the other half, which only S and dP read)
-  static constexpr int NBAR = 1 + 2 * NST + 2 + 2 + 2 + 2 + 3 + 2;
+  static constexpr int NBAR = 1 + 2 * NST + 2 + 2 + 2 + 2 + 3 + 2 + 2;  // + s_free[2]
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // warps 0-7: two elementwise warpgroups (each takes 32 of the 64 query
-  // columns of a block, thread = key row); warp 8: TMA; warp 9: MMA
+  // columns of a block, thread = key row); warp 8: TMA; warp 9: MMA (S, dP);
+  // warp 10 (head_dim 64/128): MMA (dV, dK, dQ), so each issuer can wait on
+  // its own barriers while the other keeps the tensor pipe busy
   static constexpr int ELEM_THREADS = 256;
-  static constexpr int THREADS = 320;
-  static constexpr int LOAD_WARP = 8, MMA_WARP = 9;
+  static constexpr bool TWO_ISSUERS = (NSPLIT == 1);
+  static constexpr int THREADS = TWO_ISSUERS ? 352 : 320;
+  static constexpr int LOAD_WARP = 8, MMA_WARP = 9, GRAD_WARP = 10;
   // tensor memory columns
   static constexpr int COL_S = 0, COL_DP = 128, COL_DQ = 192, COL_DV = 256, COL_DK = 256 + DH;
   static constexpr uint32_t IDESC_SDP = idesc_bf16(128, BM, false, false);
@@ -131,7 +134,7 @@ struct BwdSmem {
   uint8_t *k, *v, *st, *ds, *dqs;
   float* lsd;
   uint64_t *kv_full, *qdo_full, *qdo_empty, *s_full, *dp_full, *dp_free, *ds_ready, *ds_free,
-      *dq_full, *dq_free, *dkv_full, *oth_full, *oth_empty;
+      *dq_full, *dq_free, *dkv_full, *oth_full, *oth_empty, *s_free;
   uint32_t* tmem_base;
   volatile int* abort;
 };
@@ -160,6 +163,7 @@ __device__ __forceinline__ BwdSmem bwd_smem(uint8_t* base) {
   s.dkv_full = s.dq_free + 1;
   s.oth_full = s.dkv_full + 1;
   s.oth_empty = s.oth_full + 1;
+  s.s_free = s.oth_empty + 1;
   s.tmem_base = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
   s.abort = reinterpret_cast<volatile int*>(base + C::OFF_MISC + 4);
   return s;
@@ -397,9 +401,10 @@ struct BwdMma {
 
 template <int D>
 __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, const BwdSmem& s,
-                                        uint32_t tmem) {
+                                        uint32_t tmem, int role) {
   using C = BwdCfg<D>;
   if (t.n_iter == 0) return;
+  if (!C::TWO_ISSUERS && role != 0) return;
   BwdMma<D> m(p, s, t, tmem);
   TRACE_INIT();
   if (!m.wait(s.kv_full, 0, 1)) return;
@@ -410,6 +415,7 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, co
     // released right after them so the next load has the most slack
     m.grads(j, j == 0);
     mma_commit(&s.qdo_empty[j % C::NST]);
+    mma_commit(&s.s_free[j & 1]);  // the dV MMA has read P^T from the S buffer
     if (j < 200) TRACE(2048 + j * 8 + 5);
     if (j >= 1 && !m.wait(s.dq_free, (j - 1) & 1, 3)) return false;
     if (j < 200) TRACE(2048 + j * 8 + 6);
@@ -453,27 +459,30 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, co
     }
     if (!grads_part(t.n_iter - 1) || !dq_part(t.n_iter - 1)) return;
     mma_commit(s.dkv_full);
+  } else if (role == 0) {
+    // S and dP of every block, running ahead of the gradient MMAs
+    for (int i = 0; i < t.n_iter; ++i) {
+      const int st = i % C::NST;
+      if (!m.wait(&s.qdo_full[st], (i / C::NST) & 1, 4)) return;
+      // S buffer (i & 1) held P^T of block i-2, read by that block's dV MMA
+      if (i >= 2 && !m.wait(&s.s_free[i & 1], ((i - 2) >> 1) & 1, 8)) return;
+      if (i < 200) TRACE(2048 + i * 8 + 0);
+      const uint8_t* stg = s.st + st * C::STAGE_BYTES;
+      m.issue_kt(C::COL_S + (i & 1) * 64, s.k, stg);
+      mma_commit(&s.s_full[i & 1]);
+      if (i < 200) TRACE(2048 + i * 8 + 1);
+      if (i >= 1 && !m.wait(s.dp_free, (i - 1) & 1, 5)) return;
+      if (i < 200) TRACE(2048 + i * 8 + 2);
+      m.issue_kt(C::COL_DP, s.v, stg + C::PANELS * C::QD_PANEL);
+      mma_commit(s.dp_full);
+      if (i < 200) TRACE(2048 + i * 8 + 3);
+    }
   } else {
-  for (int i = 0; i < t.n_iter; ++i) {
-    const int st = i % C::NST;
-    // with a single (Q, dO) stage, block i can only be loaded once block i-1's
-    // gradient MMAs have released it
-    if (C::NST == 1 && i >= 1 && !do_grads(i - 1)) return;
-    if (!m.wait(&s.qdo_full[st], (i / C::NST) & 1, 4)) return;
-    if (i < 200) TRACE(2048 + i * 8 + 0);
-    const uint8_t* stg = s.st + st * C::STAGE_BYTES;
-    m.issue_kt(C::COL_S + (i & 1) * 64, s.k, stg);
-    mma_commit(&s.s_full[i & 1]);
-    if (i < 200) TRACE(2048 + i * 8 + 1);
-    if (i >= 1 && !m.wait(s.dp_free, (i - 1) & 1, 5)) return;
-    if (i < 200) TRACE(2048 + i * 8 + 2);
-    m.issue_kt(C::COL_DP, s.v, stg + C::PANELS * C::QD_PANEL);
-    if (i < 200) TRACE(2048 + i * 8 + 3);
-    mma_commit(s.dp_full);
-    if (C::NST > 1 && i >= 1 && !do_grads(i - 1)) return;
-  }
-  if (!do_grads(t.n_iter - 1)) return;
-  mma_commit(s.dkv_full);
+    // dV, dK and dQ of every block.  The (Q, dO) stage of block j is released
+    // here: S and dP of block j completed before its dS could be ready.
+    for (int j = 0; j < t.n_iter; ++j)
+      if (!do_grads(j)) return;
+    mma_commit(s.dkv_full);
   }
 }
 
@@ -694,6 +703,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.ds_ready[i], C::ELEM_THREADS / 32);
       mbar_init(&s.ds_free[i], 1);
+      mbar_init(&s.s_free[i], 1);
     }
     mbar_init(s.dp_full, 1);
     mbar_init(s.dp_free, C::ELEM_THREADS / 32);
@@ -731,7 +741,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   } else if (warp == C::LOAD_WARP) {
     bwd_load<D>(p, t, s, &tmK, &tmV, &tmQ, &tmO);
   } else {
-    if (lane_id() == 0) bwd_mma<D>(p, t, s, tmem);
+    if (lane_id() == 0) bwd_mma<D>(p, t, s, tmem, warp - C::MMA_WARP);
     __syncwarp();
   }
   tc_fence_before();
