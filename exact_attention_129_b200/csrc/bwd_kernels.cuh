@@ -527,7 +527,6 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     const bool d_ok = row < C::DH;
     uint32_t r0[32];
     tmem_ld32(tmem + lane_base + C::COL_DQ + qc0, r0);
-    tmem_ld_wait(r0);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(s.dq_free);
@@ -573,10 +572,8 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     const float* lse2 = s.lsd + (i % C::NST) * 128 + qc0;  // LSE in the log2 domain
     const float* dlt = s.lsd + (i % C::NST) * 128 + 64 + qc0;  // D_i
     uint32_t sr[32], dr[32];
-    tmem_ld32(tmem + lane_base + C::COL_S + b * 64 + qc0, sr);
-    tmem_ld32(tmem + lane_base + C::COL_DP + qc0, dr);
-    tmem_ld_wait(sr);
-    tmem_ld_wait(dr);
+    tmem_ld32x2(tmem + lane_base + C::COL_S + b * 64 + qc0, sr, tmem + lane_base + C::COL_DP + qc0,
+                dr);
     tc_fence_before();
     if (tid == 0 && i < 200) TRACE(i * 8 + 1);
     __syncwarp();
@@ -659,7 +656,6 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     uint32_t r[32];
     if (t.n_iter > 0) {
       tmem_ld32(tmem + lane_base + col0 + cc * 32, r);
-      tmem_ld_wait(r);
     } else {
 #pragma unroll
       for (int x = 0; x < 32; ++x) r[x] = 0u;

@@ -79,7 +79,9 @@ struct FwdCfg {
   // double-buffer S (the 128 x 256 fp32 O fills half of tensor memory).
   static constexpr bool DBUF = (D != 256);
   static constexpr int BM = 128;               // rows per query tile
-  static constexpr int BN = DBUF ? 64 : 128;   // keys per block
+  // keys per block: the four S slots and O fill tensor memory exactly
+  // (4 x 96 + 2 x 64, 4 x 64 + 2 x 128, 2 x 128 + 256)
+  static constexpr int BN = (D == 64) ? 96 : (D == 128 ? 64 : 128);
   static constexpr int NQ = DBUF ? 2 : 1;      // query tiles per CTA
   static constexpr int NSS = DBUF ? 4 : 2;     // S slots (tile, buffer)
   static constexpr int PANELS = D / 64;        // 64-column (128-byte) panels per row
@@ -87,18 +89,22 @@ struct FwdCfg {
   static constexpr int CHUNK = BN * 128;       // ring slot: one K panel of BN rows
   static constexpr int VROWS = CHUNK / (2 * D);  // V key rows per chunk (all D columns)
   static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int NSLOT = (D == 64) ? 24 : (D == 128 ? 20 : 10);
+  static constexpr int NSLOT = (D == 64) ? 14 : (D == 128 ? 20 : 10);
   // ring barriers guard stages of G chunks.  DBUF: stage j holds K_j and
   // V_{j-1} (exactly what one MMA iteration consumes), so each iteration waits
   // on and releases one barrier.  head_dim 256: one chunk per stage.
   static constexpr int G = DBUF ? 2 * PANELS : 1;
   static constexpr int NSTAGE = NSLOT / G;
-  static constexpr int SOFTMAX_WARPS = 4 * NQ;
+  // head_dim 64: two threads per query row, each with half of the row's key
+  // columns, so four softmax warps share each SM sub-partition and keep its
+  // exp unit busy (one warp alone cannot: its exps are latency-bound)
+  static constexpr int ROW_SPLIT = (D == 64) ? 2 : 1;
+  static constexpr int SOFTMAX_WARPS = 4 * NQ * ROW_SPLIT;
   static constexpr int LOAD_WARP = SOFTMAX_WARPS;
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;  // one MMA warp per query tile
   static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 1 + NQ);
   static constexpr int TMEM_COLS = 512;
-  static constexpr int O_COL0 = 256;           // S slots use columns [0, 256)
+  static constexpr int O_COL0 = NSS * BN;      // S slots use columns [0, NSS * BN)
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
@@ -106,7 +112,10 @@ struct FwdCfg {
   // barriers: q_full[NQ] kv_full[NSTAGE] kv_empty[NSTAGE] s_full[NSS] p_full[NSS] o_ready[NQ]
   static constexpr int NBAR = NQ + 2 * NSTAGE + 2 * NSS + NQ;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+  // row-split exchange: [tile][block parity][half][row] fp32
+  static constexpr int OFF_XCH = OFF_MISC + 64;
+  static constexpr int XCH_BYTES = (ROW_SPLIT == 2) ? NQ * 2 * 2 * BM * 4 : 0;
+  static constexpr int SMEM_BYTES = OFF_XCH + XCH_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -126,6 +135,7 @@ struct FwdSmem {
   uint64_t* o_ready;
   uint32_t* tmem_base;
   volatile int* abort;
+  float* xch;
 };
 
 template <int D>
@@ -143,6 +153,7 @@ __device__ __forceinline__ FwdSmem fwd_smem(uint8_t* base) {
   s.o_ready = s.p_full + C::NSS;
   s.tmem_base = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
   s.abort = reinterpret_cast<volatile int*>(base + C::OFF_MISC + 4);
+  s.xch = reinterpret_cast<float*>(base + C::OFF_XCH);
   return s;
 }
 
@@ -450,7 +461,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   // each block) through a pair of named barriers, so one warp's loads, max and
   // stores overlap the other's exps.  A warp that gives up on a timed-out wait
   // still plays its remaining turns, so its partner never waits forever.
-  const bool pingpong = C::DBUF && (t.m_base + C::BM < t.sq);
+  const bool pingpong = C::DBUF && C::ROW_SPLIT == 1 && (t.m_base + C::BM < t.sq);
   const int bar_t0 = 3 + 2 * warp, bar_t1 = 4 + 2 * warp;  // "tile 0 / tile 1 may start"
   auto turn_begin = [&](int k) {
     if (qt == 0) {
@@ -486,7 +497,6 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     uint32_t sr[NCOL];  // the row's scores for this block (fp32 bits)
     if constexpr (NCOL == 128) tmem_ld128(s_addr, sr);
     else tmem_ld64(s_addr, sr);
-    tmem_ld_wait(sr);
     if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 1);
     const bool masked = (j + 1) * C::BN > mask_from;
     if (masked) {
@@ -592,7 +602,6 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t r[32];
         tmem_ld32(o_addr + cc * 32, r);
-        tmem_ld_wait(r);
 #pragma unroll
         for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
         tmem_st32(o_addr + cc * 32, r);
@@ -637,7 +646,6 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       uint32_t r[32];
       if (n > 0) {
         tmem_ld32(o_addr + cc * 32, r);
-        tmem_ld_wait(r);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) r[i] = 0u;
@@ -678,6 +686,209 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   }
 }
 
+// ---------------------------------------------------------------------------
+// softmax with two threads per query row (head_dim 64, 96-key blocks): thread
+// (row, hf) owns keys [32 hf, 32 hf + 32) and [64 + 16 hf, 80 + 16 hf) of
+// every block (so every tensor-memory access is aligned to its width) and the
+// O columns [hf D/2, (hf + 1) D/2).  Both threads of a row sit in warps of the same TMEM
+// lane quadrant; per block they exchange their partial row max through shared
+// memory and a named barrier of those two warps, and at the end their partial
+// row sums.  Every thread meets every barrier, also after a timed-out wait
+// (then it only plays the barriers), so its partner never blocks for good.
+// ---------------------------------------------------------------------------
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdTile& t,
+                                                  const FwdSmem& s, uint32_t tmem, int qt,
+                                                  int hf) {
+  using C = FwdCfg<D>;
+  constexpr int NC = C::BN / 2;  // key columns per thread and block: 32 + 16
+  constexpr int OC = D / 2;      // O columns per thread
+  static_assert(C::BN == 96 && OC % 32 == 0, "row split layout");
+  const int quad = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant
+  const int lane = lane_id();
+  const int row_in_tile = quad * 32 + lane;
+  const int row = t.m_base + qt * C::BM + row_in_tile;
+  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+  const int n = t.n_blocks;
+  const float c = p.scale_log2;
+  const int key_lim = CAUSAL ? min(t.sk, row + (t.sk - t.sq) + 1) : t.sk;
+  const int tile_row0 = t.m_base + qt * C::BM;
+  const int mask_from = CAUSAL ? min(t.sk, tile_row0 + (t.sk - t.sq) + 1) : t.sk;
+  const int pair_bar = 3 + qt * 4 + quad;
+  float* xch = s.xch + qt * (2 * 2 * C::BM);  // [block parity][half][row]
+
+  TRACE_INIT();
+  [[maybe_unused]] const bool tr_on = (hf == 0) && (row_in_tile == 0);
+  float m_run = -INFINITY;
+  float l_run = 0.f;
+  bool ok = true;
+  for (int j = 0; j < n; ++j) {
+    const int slot = 2 * qt + (j & 1);
+    [[maybe_unused]] const int tr = (tr_on && j < 64) ? 1024 * qt + j * 8 : -1;
+    if (ok)
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], (j >> 1) & 1, s.abort, p.err,
+                                             ERR_FWD_SOFTMAX | 1, p.timeout_ns));
+    const uint32_t s_addr = tmem + lane_base + slot * C::BN;
+    uint32_t sa[32], sb[16];  // keys 32 hf + i, then 64 + 16 hf + i
+    float mx = -INFINITY;
+    const bool masked = (j + 1) * C::BN > mask_from;
+    TRACE(tr);
+    if (ok) {
+      tc_fence_after();
+      tmem_ld32_16(s_addr + hf * 32, sa, s_addr + 64 + hf * 16, sb);
+      if (masked) {
+        const int lim = key_lim - j * C::BN;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (hf * 32 + i >= lim) sa[i] = 0xff800000u;  // -inf
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (64 + hf * 16 + i >= lim) sb[i] = 0xff800000u;
+      }
+      float ch[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        ch[k] = fmax3(__uint_as_float(sa[k]), __uint_as_float(sa[k + 8]),
+                      __uint_as_float(sa[k + 16]));
+        ch[k] = fmax3(ch[k], __uint_as_float(sa[k + 24]), __uint_as_float(sb[k]));
+        ch[k] = fmaxf(ch[k], __uint_as_float(sb[k + 8]));
+      }
+      mx = fmaxf(fmax3(ch[0], ch[1], ch[2]), fmax3(ch[3], ch[4], fmax3(ch[5], ch[6], ch[7])));
+    }
+    // both threads of the row have read their scores once they pass the
+    // barrier, so P may then go over the slot's first 48 columns
+    float* xb = xch + (j & 1) * (2 * C::BM);
+    xb[hf * C::BM + row_in_tile] = mx;
+    TRACE(tr + 1);
+    named_bar_sync(pair_bar, 64);
+    TRACE(tr + 2);
+    if (!ok) continue;
+    mx = fmaxf(mx, xb[(1 - hf) * C::BM + row_in_tile]);
+    const float m_new = fmaxf(m_run, mx * c);
+    bool rescale = false;
+    float alpha = 1.f;
+    if (j == 0) {
+      m_run = m_new;
+    } else if (m_new - m_run > 8.f) {
+      alpha = ex2(m_run - m_new);
+      rescale = true;
+      m_run = m_new;
+      l_run *= alpha;
+    }
+    const float m_sub = (m_run == -INFINITY) ? 0.f : m_run;
+    {
+      const uint64_t cc2 = f2_pack(c, c), mm2 = f2_pack(-m_sub, -m_sub);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pa[16], pb[8];  // P of keys 32 hf + 2i.. and 64 + 16 hf + 2i.. (bf16 pairs)
+#pragma unroll
+      for (int i = 0; i < 24; ++i) {
+        const uint32_t u0 = (i < 16) ? sa[2 * i] : sb[2 * (i - 16)];
+        const uint32_t u1 = (i < 16) ? sa[2 * i + 1] : sb[2 * (i - 16) + 1];
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(u0), __uint_as_float(u1)), cc2, mm2), x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+        if (i < 16) pa[i] = pack_bf16(p0, p1);
+        else pb[i - 16] = pack_bf16(p0, p1);
+      }
+      // key k's P is at column k / 2 of the slot
+      tmem_st16(s_addr + hf * 16, pa);
+      tmem_st8(s_addr + 32 + hf * 8, pb);
+      TRACE(tr + 3);
+      float a0, a1, a2, a3;
+      f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+      f2_unpack(f2_add(acc[2], acc[3]), a2, a3);
+      l_run += (a0 + a1) + (a2 + a3);
+    }
+    if (__any_sync(0xffffffffu, rescale)) {
+      // O must not be rescaled while the previous P.V MMA may still write it
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (j - 1) & 1, s.abort, p.err,
+                                             ERR_FWD_SOFTMAX | 2, p.timeout_ns))) {
+        ok = false;
+        continue;
+      }
+      tc_fence_after();
+      const uint32_t o_addr = tmem + lane_base + C::O_COL0 + qt * D + hf * OC;
+#pragma unroll 1
+      for (int cc = 0; cc < OC / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(o_addr + cc * 32, r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+        tmem_st32(o_addr + cc * 32, r);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.p_full[slot]);
+    TRACE(tr + 4);
+  }
+
+  // ---- epilogue: the row sum is the sum of both halves' sums ----
+  float* xe = xch + (n & 1) * (2 * C::BM);  // not read since block n-2
+  xe[hf * C::BM + row_in_tile] = l_run;
+  named_bar_sync(pair_bar, 64);
+  const float l_tot = l_run + xe[(1 - hf) * C::BM + row_in_tile];
+  const bool row_valid = row < t.sq;
+  const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+  uint8_t* stage = s.q + qt * C::Q_BYTES;
+  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  // the last S read was issued before the second-to-last P.V: wait for both
+  if (ok && n > 1)
+    ok = __all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (n - 2) & 1, s.abort, p.err,
+                                           ERR_FWD_SOFTMAX | 3, p.timeout_ns));
+  if (ok && n > 0)
+    ok = __all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (n - 1) & 1, s.abort, p.err,
+                                           ERR_FWD_SOFTMAX | 3, p.timeout_ns));
+  if (ok) {
+    tc_fence_after();
+    const uint32_t o_addr = tmem + lane_base + C::O_COL0 + qt * D + hf * OC;
+#pragma unroll 1
+    for (int cc = 0; cc < OC / 32; ++cc) {
+      uint32_t r[32];
+      if (n > 0) {
+        tmem_ld32(o_addr + cc * 32, r);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = 0u;
+      }
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint4 v;
+        v.x = pack_bf16(__uint_as_float(r[g * 8 + 0]) * inv_l, __uint_as_float(r[g * 8 + 1]) * inv_l);
+        v.y = pack_bf16(__uint_as_float(r[g * 8 + 2]) * inv_l, __uint_as_float(r[g * 8 + 3]) * inv_l);
+        v.z = pack_bf16(__uint_as_float(r[g * 8 + 4]) * inv_l, __uint_as_float(r[g * 8 + 5]) * inv_l);
+        v.w = pack_bf16(__uint_as_float(r[g * 8 + 6]) * inv_l, __uint_as_float(r[g * 8 + 7]) * inv_l);
+        const int chunk = (hf * OC + cc * 32) / 8 + g;
+        *reinterpret_cast<uint4*>(stage + row_in_tile * (D * 2) +
+                                  ((chunk ^ (row_in_tile & 7)) * 16)) = v;
+      }
+    }
+  }
+  named_bar_sync(1 + qt, 256);  // both halves of the tile
+  if (ok) {
+    const int rows_left = t.sq - tile_row0;
+    uint8_t* out = static_cast<uint8_t*>(p.out);
+    const int tid = hf * 128 + row_in_tile;
+#pragma unroll 4
+    for (int q = tid; q < C::BM * CPR; q += 256) {
+      const int r = q / CPR, ch = q % CPR;
+      if (r < rows_left) {
+        const uint4 v =
+            *reinterpret_cast<const uint4*>(stage + r * (D * 2) + ((ch ^ (r & 7)) * 16));
+        const size_t grow = static_cast<size_t>(t.q0 + tile_row0 + r);
+        *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + t.h) * D) * 2 + ch * 16) = v;
+      }
+    }
+    if (p.return_lse && row_valid && hf == 0) {
+      const float lse =
+          (l_tot > 0.f) ? (m_run + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
+      p.lse[static_cast<size_t>(t.h) * p.total_q + t.q0 + row] = lse;
+    }
+  }
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -702,7 +913,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     }
     for (int i = 0; i < C::NSS; ++i) {
       mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.p_full[i], 4);  // one arrival per softmax warp
+      mbar_init(&s.p_full[i], 4 * C::ROW_SPLIT);  // one arrival per softmax warp of the tile
     }
     for (int i = 0; i < C::NQ; ++i) mbar_init(&s.o_ready[i], 1);
     *s.abort = 0;
@@ -723,8 +934,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   const uint32_t tmem = *s.tmem_base;
 
   if (warp < C::SOFTMAX_WARPS) {
-    const int qt = warp / 4;
-    if (t.m_base + qt * C::BM < t.sq) fwd_softmax<D, CAUSAL>(p, t, s, tmem, qt);
+    const int grp = warp / 4;
+    const int qt = grp / C::ROW_SPLIT;
+    if (t.m_base + qt * C::BM < t.sq) {
+      if constexpr (C::ROW_SPLIT == 2)
+        fwd_softmax_split<D, CAUSAL>(p, t, s, tmem, qt, grp % 2);
+      else
+        fwd_softmax<D, CAUSAL>(p, t, s, tmem, qt);
+    }
   } else if (warp == C::LOAD_WARP) {
     if (lane_id() == 0) fwd_load<D>(p, t, s, &tmQ, &tmK, &tmV);
   } else {
