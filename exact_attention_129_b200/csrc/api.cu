@@ -74,6 +74,18 @@ uint64_t wait_timeout_ns() {
   return v;
 }
 
+// Test hook, read on every call so a test can switch it: the forward's softmax
+// warps idle ATTN_TEST_EPILOGUE_DELAY_US microseconds (at most 1000) before
+// their final wait.  0 or unset in normal use.
+uint64_t test_epilogue_delay_ns() {
+  const char* e = std::getenv("ATTN_TEST_EPILOGUE_DELAY_US");
+  if (!e) return 0;
+  long us = std::atol(e);
+  if (us <= 0) return 0;
+  if (us > 1000) us = 1000;
+  return static_cast<uint64_t>(us) * 1000ull;
+}
+
 // Per-device set-up, once: the error word's device address and the device's
 // compute capability.
 DeviceState* device_state(int* dev_out) {
@@ -296,6 +308,7 @@ extern "C" attn_status_t attn_fwd(const void* q, const void* k, const void* v,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.return_lse = return_lse ? 1 : 0;
   p.timeout_ns = wait_timeout_ns();
+  p.epilogue_delay_ns = test_epilogue_delay_ns();
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool c = causal != 0;

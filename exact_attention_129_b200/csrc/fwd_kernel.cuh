@@ -69,7 +69,17 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e)
   int return_lse;
   uint64_t timeout_ns;
+  // test hook (0 in normal use): the softmax warps idle this long before their
+  // final wait, so the tile's last P.V is sure to have completed by then
+  uint64_t epilogue_delay_ns;
 };
+
+__device__ __forceinline__ void fwd_test_delay(const FwdParams& p) {
+  if (p.epilogue_delay_ns == 0) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < p.epilogue_delay_ns) {
+  }
+}
 
 template <int D>
 struct FwdCfg {
@@ -109,8 +119,9 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
   static constexpr int OFF_BAR = OFF_RING + NSLOT * CHUNK;
-  // barriers: q_full[NQ] kv_full[NSTAGE] kv_empty[NSTAGE] s_full[NSS] p_full[NSS] o_ready[NQ]
-  static constexpr int NBAR = NQ + 2 * NSTAGE + 2 * NSS + NQ;
+  // barriers: q_full[NQ] kv_full[NSTAGE] kv_empty[NSTAGE] s_full[NSS] p_full[NSS]
+  // o_ready[NQ] o_final[NQ]
+  static constexpr int NBAR = NQ + 2 * NSTAGE + 2 * NSS + 2 * NQ;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // row-split exchange: [tile][block parity][half][row] fp32
   static constexpr int OFF_XCH = OFF_MISC + 64;
@@ -132,7 +143,8 @@ struct FwdSmem {
   uint64_t* kv_empty;
   uint64_t* s_full;
   uint64_t* p_full;
-  uint64_t* o_ready;
+  uint64_t* o_ready;  // one phase per P.V (rescales wait on the previous one)
+  uint64_t* o_final;  // one phase per CTA: the tile's last P.V is done
   uint32_t* tmem_base;
   volatile int* abort;
   float* xch;
@@ -151,6 +163,7 @@ __device__ __forceinline__ FwdSmem fwd_smem(uint8_t* base) {
   s.s_full = s.kv_empty + C::NSTAGE;
   s.p_full = s.s_full + C::NSS;
   s.o_ready = s.p_full + C::NSS;
+  s.o_final = s.o_ready + C::NQ;
   s.tmem_base = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
   s.abort = reinterpret_cast<volatile int*>(base + C::OFF_MISC + 4);
   s.xch = reinterpret_cast<float*>(base + C::OFF_XCH);
@@ -401,6 +414,7 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
       m.release_stages(1);
       TRACE(tr + 4);
     }
+    mma_commit(&s.o_final[qt]);
   } else {
     // one query tile, two S slots alternating over key blocks; one chunk per stage
     constexpr int P = C::PANELS;
@@ -432,6 +446,7 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
         m.release_stages(P);
       }
     }
+    mma_commit(&s.o_final[0]);
   }
 }
 
@@ -589,7 +604,10 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     l_run += lsum;
     if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 3);
     if (__any_sync(0xffffffffu, rescale)) {
-      // O must not be rescaled while the previous P.V MMA may still write it
+      // O must not be rescaled while the previous P.V MMA may still write it.
+      // o_ready has completed j-1 or j phases here (S(j), just read, was issued
+      // after P.V(j-2), and P.V(j) needs this block's P), so the parity of
+      // phase j-1 is unambiguous.
       if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (j - 1) & 1, s.abort, p.err,
                                              ERR_FWD_SOFTMAX | 2, p.timeout_ns))) {
         ok = false;
@@ -625,16 +643,14 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
   uint8_t* stage = s.q + qt * C::Q_BYTES;
   constexpr int CPR = D / 8;  // 16-byte chunks per row
-  // The last S this warpgroup read was issued before the second-to-last P.V, so
-  // that P.V may still be running: wait for its phase first, then the last one
-  // (a single parity wait could match a phase two behind).
-  if (ok && n > 1) {
-    if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (n - 2) & 1, s.abort, p.err,
-                                           ERR_FWD_SOFTMAX | 3, p.timeout_ns)))
-      ok = false;
-  }
+  // Wait for the tile's last P.V on its own single-phase barrier.  A parity
+  // wait on o_ready cannot do it: the last S this warpgroup read was issued
+  // before the second-to-last P.V, so o_ready may be anywhere from two phases
+  // short of the end to already past it, and a parity test cannot tell a phase
+  // two behind from the current one.
+  fwd_test_delay(p);
   if (ok && n > 0) {
-    if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (n - 1) & 1, s.abort, p.err,
+    if (!__all_sync(0xffffffffu, mbar_wait(&s.o_final[qt], 0, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 3, p.timeout_ns)))
       ok = false;
   }
@@ -801,7 +817,10 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
       l_run += (a0 + a1) + (a2 + a3);
     }
     if (__any_sync(0xffffffffu, rescale)) {
-      // O must not be rescaled while the previous P.V MMA may still write it
+      // O must not be rescaled while the previous P.V MMA may still write it.
+      // o_ready has completed j-1 or j phases here (S(j), just read, was issued
+      // after P.V(j-2), and P.V(j) needs this block's P), so the parity of
+      // phase j-1 is unambiguous.
       if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (j - 1) & 1, s.abort, p.err,
                                              ERR_FWD_SOFTMAX | 2, p.timeout_ns))) {
         ok = false;
@@ -834,12 +853,10 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
   const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
   uint8_t* stage = s.q + qt * C::Q_BYTES;
   constexpr int CPR = D / 8;  // 16-byte chunks per row
-  // the last S read was issued before the second-to-last P.V: wait for both
-  if (ok && n > 1)
-    ok = __all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (n - 2) & 1, s.abort, p.err,
-                                           ERR_FWD_SOFTMAX | 3, p.timeout_ns));
+  // the tile's last P.V, on its single-phase barrier (see fwd_softmax)
+  fwd_test_delay(p);
   if (ok && n > 0)
-    ok = __all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (n - 1) & 1, s.abort, p.err,
+    ok = __all_sync(0xffffffffu, mbar_wait(&s.o_final[qt], 0, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 3, p.timeout_ns));
   if (ok) {
     tc_fence_after();
@@ -915,7 +932,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.p_full[i], 4 * C::ROW_SPLIT);  // one arrival per softmax warp of the tile
     }
-    for (int i = 0; i < C::NQ; ++i) mbar_init(&s.o_ready[i], 1);
+    for (int i = 0; i < C::NQ; ++i) {
+      mbar_init(&s.o_ready[i], 1);
+      mbar_init(&s.o_final[i], 1);
+    }
     *s.abort = 0;
     fence_mbar_init();
   }

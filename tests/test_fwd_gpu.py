@@ -76,6 +76,17 @@ def test_lse_flag_does_not_change_out(d):
     assert torch.equal(o1, o2)
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_epilogue_after_last_pv(d, monkeypatch):
+    """The softmax warps reach their final wait only after the tile's last P.V
+    has completed (the test hook holds them 200 us).  A parity wait on the
+    per-P.V barrier would then name a phase two behind and never return; the
+    single-phase final barrier must let every tile finish."""
+    monkeypatch.setenv("ATTN_TEST_EPILOGUE_DELAY_US", "200")
+    for causal in (False, True):
+        check_full(si.Workload(f"late_epilogue_d{d}", [1000, 257, 96], 4, 2, d, causal, seed=9))
+
+
 def test_deterministic():
     wl = si.Workload("det", [777, 1500], 4, 2, 128, True, seed=8)
     outs = [run_fwd(wl)[1:] for _ in range(3)]
