@@ -56,11 +56,19 @@ def _load(mutation: int = 0, out_dir: str | None = None):
             ip = ctypes.POINTER(ctypes.c_int32)
             lp = ctypes.POINTER(ctypes.c_int64)
             i, d = ctypes.c_int, ctypes.c_double
+            lg = ctypes.c_long
             lib.oracle_fwd.argtypes = [dp, dp, dp, ip, ip, i, i, i, i, d, i, dp, dp]
             lib.oracle_bwd.argtypes = [dp, dp, dp, dp, ip, ip, i, i, i, i, d, i, dp, dp, dp]
             lib.oracle_rows.argtypes = [dp, dp, dp, dp, ip, ip, i, i, i, i, d, i, i, ip, lp,
                                         dp, dp, dp]
-            for fn in (lib.oracle_fwd, lib.oracle_bwd, lib.oracle_rows):
+            lib.oracle_fwd_ex.argtypes = [dp, dp, dp, ip, ip, i, i, i, i, d, i, lg, lg, d, dp,
+                                          dp]
+            lib.oracle_bwd_ex.argtypes = [dp, dp, dp, dp, ip, ip, i, i, i, i, d, i, lg, lg, d,
+                                          dp, dp, dp]
+            lib.oracle_rows_ex.argtypes = [dp, dp, dp, dp, ip, ip, i, i, i, i, d, i, lg, lg, d,
+                                           i, ip, lp, dp, dp, dp]
+            for fn in (lib.oracle_fwd, lib.oracle_bwd, lib.oracle_rows, lib.oracle_fwd_ex,
+                       lib.oracle_bwd_ex, lib.oracle_rows_ex):
                 fn.restype = ctypes.c_int
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_mutation.restype = ctypes.c_int
@@ -99,25 +107,39 @@ def num_threads(mutation: int = 0) -> int:
     return int(_load(mutation).oracle_num_threads())
 
 
-def fwd(q, k, v, cu_q, cu_k, scale, causal, *, mutation: int = 0, lib_dir=None):
-    """O [Tq,Hq,D] and LSE [Hq,Tq] (natural log of the scaled scores), float64."""
+def _mask_args(window, softcap):
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    return wl, wr, float(softcap or 0.0)
+
+
+def fwd(q, k, v, cu_q, cu_k, scale, causal, *, window=None, softcap=0.0, mutation: int = 0,
+        lib_dir=None):
+    """O [Tq,Hq,D] and LSE [Hq,Tq] (natural log of the scaled scores), float64.
+
+    ``window`` = (left, right) key-distance bounds around the bottom-right
+    aligned diagonal (negative = no bound); ``softcap`` > 0 caps the scaled
+    scores at c * tanh(s / c)."""
+    wl, wr, cap = _mask_args(window, softcap)
     q, k, v = _f64(q), _f64(k), _f64(v)
     cu_q, cu_k = _i32(cu_q), _i32(cu_k)
     Tq, Hq, Tk, Hkv, D, B = _dims(q, k, cu_q)
     assert int(cu_q[-1]) == Tq and int(cu_k[-1]) == Tk
     out = np.zeros((Tq, Hq, D), np.float64)
     lse = np.zeros((Hq, Tq), np.float64)
-    rc = _load(mutation, lib_dir).oracle_fwd(
+    rc = _load(mutation, lib_dir).oracle_fwd_ex(
         _ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double),
         _ptr(cu_q, ctypes.c_int32), _ptr(cu_k, ctypes.c_int32), B, Hq, Hkv, D,
-        float(scale), int(bool(causal)), _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
+        float(scale), int(bool(causal)), wl, wr, cap, _ptr(out, ctypes.c_double),
+        _ptr(lse, ctypes.c_double))
     if rc != 0:
         raise ValueError(f"oracle_fwd rejected its arguments (code {rc})")
     return out, lse
 
 
-def bwd(q, k, v, dout, cu_q, cu_k, scale, causal, *, mutation: int = 0, lib_dir=None):
+def bwd(q, k, v, dout, cu_q, cu_k, scale, causal, *, window=None, softcap=0.0,
+        mutation: int = 0, lib_dir=None):
     """dQ [Tq,Hq,D], dK, dV [Tk,Hkv,D] of L = sum(dout * O), float64."""
+    wl, wr, cap = _mask_args(window, softcap)
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     cu_q, cu_k = _i32(cu_q), _i32(cu_k)
     Tq, Hq, Tk, Hkv, D, B = _dims(q, k, cu_q)
@@ -125,10 +147,10 @@ def bwd(q, k, v, dout, cu_q, cu_k, scale, causal, *, mutation: int = 0, lib_dir=
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
-    rc = _load(mutation, lib_dir).oracle_bwd(
+    rc = _load(mutation, lib_dir).oracle_bwd_ex(
         _ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double),
         _ptr(dout, ctypes.c_double), _ptr(cu_q, ctypes.c_int32), _ptr(cu_k, ctypes.c_int32),
-        B, Hq, Hkv, D, float(scale), int(bool(causal)), _ptr(dq, ctypes.c_double),
+        B, Hq, Hkv, D, float(scale), int(bool(causal)), wl, wr, cap, _ptr(dq, ctypes.c_double),
         _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double))
     if rc != 0:
         raise ValueError(f"oracle_bwd rejected its arguments (code {rc})")
@@ -136,12 +158,13 @@ def bwd(q, k, v, dout, cu_q, cu_k, scale, causal, *, mutation: int = 0, lib_dir=
 
 
 def rows(q, k, v, cu_q, cu_k, scale, causal, heads, row_index, dout=None, *,
-         mutation: int = 0, lib_dir=None):
+         window=None, softcap=0.0, mutation: int = 0, lib_dir=None):
     """O, LSE (and dQ if ``dout`` is given) for chosen (head, global row) pairs.
 
     Exact at any length: a row needs only its own scores.  Returns
     ``(out [n,D], lse [n], dq [n,D] or None)``.
     """
+    wl, wr, cap = _mask_args(window, softcap)
     q, k, v = _f64(q), _f64(k), _f64(v)
     dptr = None
     if dout is not None:
@@ -156,10 +179,11 @@ def rows(q, k, v, cu_q, cu_k, scale, causal, heads, row_index, dout=None, *,
     out = np.zeros((n, D), np.float64)
     lse = np.zeros((n,), np.float64)
     dq = np.zeros((n, D), np.float64) if dout is not None else None
-    rc = _load(mutation, lib_dir).oracle_rows(
+    rc = _load(mutation, lib_dir).oracle_rows_ex(
         _ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double), dptr,
         _ptr(cu_q, ctypes.c_int32), _ptr(cu_k, ctypes.c_int32), B, Hq, Hkv, D, float(scale),
-        int(bool(causal)), n, _ptr(heads, ctypes.c_int32), _ptr(row_index, ctypes.c_int64),
+        int(bool(causal)), wl, wr, cap, n, _ptr(heads, ctypes.c_int32),
+        _ptr(row_index, ctypes.c_int64),
         _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double),
         _ptr(dq, ctypes.c_double) if dq is not None else None)
     if rc != 0:

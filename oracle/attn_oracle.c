@@ -10,14 +10,19 @@
  *   For segment b (query rows [cu_q[b], cu_q[b+1]), key rows [cu_k[b], cu_k[b+1])),
  *   query head h and its key/value head hk = floor(h / G), G = Hq / Hkv:
  *     s_ij  = scale * sum_d q_id k_jd                    for every key j of the segment
- *     key j is allowed for row i  iff  !causal || j <= i + (s_k - s_q)
+ *             (with a softcap c > 0: s_ij = c * tanh(scale * sum_d q_id k_jd / c))
+ *     key j is allowed for row i  iff, with delta = s_k - s_q,
+ *             (!causal || j <= i + delta)
+ *          && (window_left  < 0 || j >= i + delta - window_left)
+ *          && (window_right < 0 || j <= i + delta + window_right)
  *     LSE_i = log sum_{allowed j} exp(s_ij)              (natural log, scaled scores)
  *     P_ij  = exp(s_ij - LSE_i) for allowed j, else 0
  *     O_i   = sum_j P_ij v_j
  *   and, given dO:
  *     D_i   = sum_d dO_id O_id
  *     dP_ij = sum_d dO_id v_jd
- *     dS_ij = P_ij (dP_ij - D_i)
+ *     dS_ij = P_ij (dP_ij - D_i) * g_ij,  g_ij = 1 - (s_ij / c)^2 with a softcap
+ *             (the derivative of c tanh(x / c) at x = scale q_i.k_j), else 1
  *     dQ_i  = scale * sum_j dS_ij k_j
  *     dK_j  = scale * sum_{h in group(hk)} sum_i dS_ij q_i
  *     dV_j  =         sum_{h in group(hk)} sum_i P_ij dO_i
@@ -38,6 +43,11 @@
  *   - a row with no allowed key: O_i = 0, LSE_i = -inf, and it contributes
  *     nothing to any gradient.
  *   - zero-length segments are allowed and produce nothing.
+ *   - local (sliding-window) masks and the softcap: the FA4 repository guide
+ *     (Public API) names window_size_left/right and softcap as parameters but
+ *     states no formula; the reading above is the plainest one (the window
+ *     bounds are inclusive distances from the bottom-right aligned diagonal, a
+ *     negative bound means none; the cap applies to the scaled score).
  *
  * Layouts (row-major, last index fastest):
  *   q, out, dout, dq : [Tq][Hq][D]      k, v, dk, dv : [Tk][Hkv][D]
@@ -98,12 +108,47 @@ static int kv_head_of(int h, int Hq, int Hkv) {
 #endif
 }
 
-static int key_allowed(long i, long j, long sq, long sk, int causal) {
-  if (!causal) return 1;
+typedef struct {
+  int causal;
+  long wl, wr;     /* window bounds, < 0 = none */
+  double softcap;  /* <= 0 = none */
+} mask_t;
+
+static int key_allowed(const mask_t* mk, long i, long j, long sq, long sk) {
+  const long diag = i + (sk - sq);
 #if ORACLE_MUTATION == 3
-  return j < i + (sk - sq); /* planted: diagonal excluded */
+  if (mk->causal && !(j < diag)) return 0; /* planted: diagonal excluded */
 #else
-  return j <= i + (sk - sq);
+  if (mk->causal && !(j <= diag)) return 0;
+#endif
+#if ORACLE_MUTATION == 8
+  if (mk->wl >= 0 && !(j > diag - mk->wl)) return 0; /* planted: window edge excluded */
+#else
+  if (mk->wl >= 0 && !(j >= diag - mk->wl)) return 0;
+#endif
+  if (mk->wr >= 0 && !(j <= diag + mk->wr)) return 0;
+  return 1;
+}
+
+/* the score of row q_i and key k_j (scaled, then capped if a softcap is set) */
+static double score(const mask_t* mk, double scale, double qk) {
+  if (mk->softcap <= 0.0) return scale * qk;
+#if ORACLE_MUTATION == 10
+  return mk->softcap * tanh(qk / mk->softcap); /* planted: cap of the unscaled score */
+#else
+  return mk->softcap * tanh(scale * qk / mk->softcap);
+#endif
+}
+
+/* d score / d (scale q.k), from the (capped) score itself */
+static double score_grad(const mask_t* mk, double s) {
+#if ORACLE_MUTATION == 9
+  (void)s;
+  return 1.0; /* planted: the cap's derivative is dropped */
+#else
+  if (mk->softcap <= 0.0) return 1.0;
+  const double t = s / mk->softcap;
+  return 1.0 - t * t;
 #endif
 }
 
@@ -122,7 +167,7 @@ typedef struct {
   const double *q, *k, *v, *dout;
   int Hq, Hkv, D;
   double scale;
-  int causal;
+  mask_t mk;
 } problem_t;
 
 static int row_forward(const problem_t* pb, int h, long qrow, long i, long k0, long sq,
@@ -133,9 +178,9 @@ static int row_forward(const problem_t* pb, int h, long qrow, long i, long k0, l
   int n_allowed = 0;
   double m = -INFINITY;
   for (long j = 0; j < sk; ++j) {
-    if (!key_allowed(i, j, sq, sk, pb->causal)) { s[j] = -INFINITY; continue; }
+    if (!key_allowed(&pb->mk, i, j, sq, sk)) { s[j] = -INFINITY; continue; }
     const double* kj = pb->k + ((size_t)(k0 + j) * pb->Hkv + hk) * D;
-    s[j] = pb->scale * dot(qi, kj, D);
+    s[j] = score(&pb->mk, pb->scale, dot(qi, kj, D));
     if (s[j] > m) m = s[j];
     ++n_allowed;
   }
@@ -176,9 +221,9 @@ static double row_delta(const problem_t* pb, int h, long qrow, const double* o) 
 #endif
 }
 
-/* dS_ij for one row, given P_ij and D_i */
+/* dS_ij for one row, given its scores s_ij, P_ij and D_i */
 static void row_dscores(const problem_t* pb, int h, long qrow, long k0, long sk,
-                        const double* p, double delta, double* ds) {
+                        const double* s, const double* p, double delta, double* ds) {
   const int D = pb->D;
   const int hk = kv_head_of(h, pb->Hq, pb->Hkv);
   const double* doi = pb->dout + ((size_t)qrow * pb->Hq + h) * D;
@@ -191,6 +236,7 @@ static void row_dscores(const problem_t* pb, int h, long qrow, long k0, long sk,
 #else
     ds[j] = p[j] * (dp - delta);
 #endif
+    ds[j] *= score_grad(&pb->mk, s[j]);
   }
 }
 
@@ -232,15 +278,18 @@ int oracle_num_threads(void) {
 
 int oracle_mutation(void) { return ORACLE_MUTATION; }
 
-/* Full forward: out [Tq][Hq][D], lse [Hq][Tq] (lse may be NULL). */
-int oracle_fwd(const double* q, const double* k, const double* v, const int32_t* cu_q,
-               const int32_t* cu_k, int batch, int Hq, int Hkv, int D, double scale,
-               int causal, double* out, double* lse) {
+/* Full forward: out [Tq][Hq][D], lse [Hq][Tq] (lse may be NULL).  window_left /
+ * window_right < 0 mean no bound, softcap <= 0 means none. */
+int oracle_fwd_ex(const double* q, const double* k, const double* v, const int32_t* cu_q,
+                  const int32_t* cu_k, int batch, int Hq, int Hkv, int D, double scale,
+                  int causal, long window_left, long window_right, double softcap,
+                  double* out, double* lse) {
   int rc = check_args(cu_q, cu_k, batch, Hq, Hkv, D);
   if (rc) return rc;
   if (!q || !k || !v || !out) return -1;
   if (batch == 0) return 0;
-  const problem_t pb = {q, k, v, NULL, Hq, Hkv, D, scale, causal};
+  const problem_t pb = {q, k, v, NULL, Hq, Hkv, D, scale,
+                        {causal, window_left, window_right, softcap}};
   const long Tq = cu_q[batch];
   const long msk = max_seg_len(cu_k, batch);
   const long n_units = (long)Hq * Tq;
@@ -265,18 +314,27 @@ int oracle_fwd(const double* q, const double* k, const double* v, const int32_t*
   return 0;
 }
 
+int oracle_fwd(const double* q, const double* k, const double* v, const int32_t* cu_q,
+               const int32_t* cu_k, int batch, int Hq, int Hkv, int D, double scale,
+               int causal, double* out, double* lse) {
+  return oracle_fwd_ex(q, k, v, cu_q, cu_k, batch, Hq, Hkv, D, scale, causal, -1, -1, 0.0,
+                       out, lse);
+}
+
 /*
  * Full backward from first principles: recomputes P from the definition
  * (it takes no O or LSE from anywhere else).  dq like q, dk/dv like k.
  */
-int oracle_bwd(const double* q, const double* k, const double* v, const double* dout,
-               const int32_t* cu_q, const int32_t* cu_k, int batch, int Hq, int Hkv,
-               int D, double scale, int causal, double* dq, double* dk, double* dv) {
+int oracle_bwd_ex(const double* q, const double* k, const double* v, const double* dout,
+                  const int32_t* cu_q, const int32_t* cu_k, int batch, int Hq, int Hkv,
+                  int D, double scale, int causal, long window_left, long window_right,
+                  double softcap, double* dq, double* dk, double* dv) {
   int rc = check_args(cu_q, cu_k, batch, Hq, Hkv, D);
   if (rc) return rc;
   if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
   if (batch == 0) return 0;
-  const problem_t pb = {q, k, v, dout, Hq, Hkv, D, scale, causal};
+  const problem_t pb = {q, k, v, dout, Hq, Hkv, D, scale,
+                        {causal, window_left, window_right, softcap}};
   const long Tq = cu_q[batch], Tk = cu_k[batch];
   const long msk = max_seg_len(cu_k, batch);
   const int G = Hq / Hkv;
@@ -303,7 +361,7 @@ int oracle_bwd(const double* q, const double* k, const double* v, const double* 
       const double delta = row_delta(&pb, h, r, o);
       lse_all[(size_t)h * Tq + r] = l;
       delta_all[(size_t)h * Tq + r] = delta;
-      row_dscores(&pb, h, r, cu_k[b], sk, p, delta, ds);
+      row_dscores(&pb, h, r, cu_k[b], sk, s, p, delta, ds);
       row_dq(&pb, h, cu_k[b], sk, ds, dq + ((size_t)r * Hq + h) * D);
     }
     free(s); free(p); free(ds); free(o);
@@ -326,18 +384,20 @@ int oracle_bwd(const double* q, const double* k, const double* v, const double* 
     for (int h = 0; h < Hq; ++h) {
       if (kv_head_of(h, Hq, Hkv) != hk) continue;
       for (long i = 0; i < sq; ++i) {
-        if (!key_allowed(i, j, sq, sk, causal)) continue;
+        if (!key_allowed(&pb.mk, i, j, sq, sk)) continue;
         const long r = cu_q[b] + i;
         const double l = lse_all[(size_t)h * Tq + r];
         if (l == -INFINITY) continue;
         const double* qi = q + ((size_t)r * Hq + h) * D;
         const double* doi = dout + ((size_t)r * Hq + h) * D;
-        const double pij = exp(scale * dot(qi, kj, D) - l);
+        const double sij = score(&pb.mk, scale, dot(qi, kj, D));
+        const double pij = exp(sij - l);
 #if ORACLE_MUTATION == 2
-        const double dsij = pij * (delta_all[(size_t)h * Tq + r] - dot(doi, vj, D));
+        double dsij = pij * (delta_all[(size_t)h * Tq + r] - dot(doi, vj, D));
 #else
-        const double dsij = pij * (dot(doi, vj, D) - delta_all[(size_t)h * Tq + r]);
+        double dsij = pij * (dot(doi, vj, D) - delta_all[(size_t)h * Tq + r]);
 #endif
+        dsij *= score_grad(&pb.mk, sij);
         for (int d = 0; d < D; ++d) {
 #if ORACLE_MUTATION == 6
           dkj[d] += scale * dsij * doi[d]; /* planted: wrong operand */
@@ -355,22 +415,30 @@ int oracle_bwd(const double* q, const double* k, const double* v, const double* 
   return 0;
 }
 
+int oracle_bwd(const double* q, const double* k, const double* v, const double* dout,
+               const int32_t* cu_q, const int32_t* cu_k, int batch, int Hq, int Hkv,
+               int D, double scale, int causal, double* dq, double* dk, double* dv) {
+  return oracle_bwd_ex(q, k, v, dout, cu_q, cu_k, batch, Hq, Hkv, D, scale, causal, -1, -1,
+                       0.0, dq, dk, dv);
+}
+
 /*
  * Sampled rows: for n (head, global query row) pairs, the row's O, LSE and,
  * when dout is not NULL, its dQ.  Each row needs only its own scores, so this
  * is exact at any sequence length.  out_rows/dq_rows are [n][D].
  */
-int oracle_rows(const double* q, const double* k, const double* v, const double* dout,
-                const int32_t* cu_q, const int32_t* cu_k, int batch, int Hq, int Hkv,
-                int D, double scale, int causal, int n, const int32_t* row_head,
-                const int64_t* row_index, double* out_rows, double* lse_rows,
-                double* dq_rows) {
+int oracle_rows_ex(const double* q, const double* k, const double* v, const double* dout,
+                   const int32_t* cu_q, const int32_t* cu_k, int batch, int Hq, int Hkv,
+                   int D, double scale, int causal, long window_left, long window_right,
+                   double softcap, int n, const int32_t* row_head, const int64_t* row_index,
+                   double* out_rows, double* lse_rows, double* dq_rows) {
   int rc = check_args(cu_q, cu_k, batch, Hq, Hkv, D);
   if (rc) return rc;
   if (!q || !k || !v || !row_head || !row_index || !out_rows || !lse_rows) return -1;
   if (dq_rows && !dout) return -1;
   if (batch == 0 || n == 0) return 0;
-  const problem_t pb = {q, k, v, dout, Hq, Hkv, D, scale, causal};
+  const problem_t pb = {q, k, v, dout, Hq, Hkv, D, scale,
+                        {causal, window_left, window_right, softcap}};
   const long Tq = cu_q[batch];
   for (int t = 0; t < n; ++t)
     if (row_head[t] < 0 || row_head[t] >= Hq || row_index[t] < 0 || row_index[t] >= Tq)
@@ -391,11 +459,20 @@ int oracle_rows(const double* q, const double* k, const double* v, const double*
       row_forward(&pb, h, r, r - cu_q[b], cu_k[b], sq, sk, s, p, o, &lse_rows[t]);
       if (dq_rows) {
         const double delta = row_delta(&pb, h, r, o);
-        row_dscores(&pb, h, r, cu_k[b], sk, p, delta, ds);
+        row_dscores(&pb, h, r, cu_k[b], sk, s, p, delta, ds);
         row_dq(&pb, h, cu_k[b], sk, ds, dq_rows + (size_t)t * D);
       }
     }
     free(s); free(p); free(ds);
   }
   return 0;
+}
+
+int oracle_rows(const double* q, const double* k, const double* v, const double* dout,
+                const int32_t* cu_q, const int32_t* cu_k, int batch, int Hq, int Hkv,
+                int D, double scale, int causal, int n, const int32_t* row_head,
+                const int64_t* row_index, double* out_rows, double* lse_rows,
+                double* dq_rows) {
+  return oracle_rows_ex(q, k, v, dout, cu_q, cu_k, batch, Hq, Hkv, D, scale, causal, -1, -1,
+                        0.0, n, row_head, row_index, out_rows, lse_rows, dq_rows);
 }

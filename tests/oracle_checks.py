@@ -16,7 +16,12 @@ with one planted mistake.  The facts used:
 * gradient identities: sum_j dK_j = 0 (each row of dS sums to zero) and
   sum_j dV_j = sum over the group's rows of dO (each row of P sums to one);
 * structure: a packed varlen batch equals independent dense calls, and GQA
-  equals MHA with K/V repeated per group (dK/dV then sum over the group).
+  equals MHA with K/V repeated per group (dK/dV then sum over the group);
+* local masks and the softcap: window (0, 0) leaves one key (O = v_j, LSE = the
+  capped score, a closed form); a window wider than the segment is no window;
+  (-1, 0) is causal; a huge cap is no cap; a windowed row equals unmasked
+  attention over its key slice; plus the torch reference and finite
+  differences on windowed and capped cases.
 """
 from __future__ import annotations
 
@@ -58,8 +63,13 @@ def _close(a, b, tol):
 # --------------------------------------------------------------------------
 # independent torch fp64 implementation (explicit mask, autograd)
 # --------------------------------------------------------------------------
-def torch_reference(q, k, v, dout, lengths_q, lengths_k, scale, causal):
-    """Dense per-segment softmax(scale QK^T + mask) V with autograd (fp64 CPU)."""
+def torch_reference(q, k, v, dout, lengths_q, lengths_k, scale, causal, window=None,
+                    softcap=0.0):
+    """Dense per-segment softmax(scale QK^T + mask) V with autograd (fp64 CPU).
+
+    ``window`` (left, right) and ``softcap`` follow the reading stated in the
+    oracle's header: inclusive key distances around the bottom-right diagonal,
+    and c * tanh(s / c) of the scaled score; autograd supplies the derivatives."""
     tq = torch.tensor(q, dtype=torch.float64, requires_grad=True)
     tk = torch.tensor(k, dtype=torch.float64, requires_grad=True)
     tv = torch.tensor(v, dtype=torch.float64, requires_grad=True)
@@ -72,9 +82,16 @@ def torch_reference(q, k, v, dout, lengths_q, lengths_k, scale, causal):
         ks = tk[ok_:ok_ + sk].permute(1, 0, 2).repeat_interleave(G, 0)
         vs = tv[ok_:ok_ + sk].permute(1, 0, 2).repeat_interleave(G, 0)
         s = scale * qs @ ks.transpose(1, 2)                       # [Hq, sq, sk]
+        if softcap and softcap > 0:
+            s = softcap * torch.tanh(s / softcap)
         i = torch.arange(sq).view(-1, 1)
         j = torch.arange(sk).view(1, -1)
-        allowed = (j <= i + (sk - sq)) if causal else torch.ones(sq, sk, dtype=torch.bool)
+        diag = i + (sk - sq)
+        allowed = (j <= diag) if causal else torch.ones(sq, sk, dtype=torch.bool)
+        if window is not None and window[0] >= 0:
+            allowed = allowed & (j >= diag - window[0])
+        if window is not None and window[1] >= 0:
+            allowed = allowed & (j <= diag + window[1])
         s = s.masked_fill(~allowed, float("-inf"))
         lse = torch.logsumexp(s, dim=-1)                          # [Hq, sq]
         p = torch.exp(s - lse.unsqueeze(-1))
@@ -347,7 +364,138 @@ def check_fully_masked_rows(mutation=0):
     return True, "ok"
 
 
+# --------------------------------------------------------------------------
+# local (sliding-window) masks and the softcap
+# --------------------------------------------------------------------------
+def check_window_softcap_closed_forms(mutation=0):
+    Hq, Hkv, D = 2, 1, 8
+    lq, lk = [7, 5], [9, 5]          # s_k - s_q = 2 and 0
+    cq, ck = _cu(lq), _cu(lk)
+    q, k, v = _rand((12, Hq, D), 90), _rand((14, Hkv, D), 91), _rand((14, Hkv, D), 92)
+    scale = 0.6
+    # window (0, 0): row i sees exactly key i + (s_k - s_q): O = v_j, LSE = s_ij
+    for cap in (0.0, 2.5):
+        o, lse = oracle.fwd(q, k, v, cq, ck, scale, False, window=(0, 0), softcap=cap,
+                            mutation=mutation)
+        oq = ok_ = 0
+        for sq, sk in zip(lq, lk):
+            for i in range(sq):
+                j = i + sk - sq
+                for h in range(Hq):
+                    a = scale * float(q[oq + i, h] @ k[ok_ + j, 0])
+                    want = cap * np.tanh(a / cap) if cap > 0 else a
+                    if not np.allclose(o[oq + i, h], v[ok_ + j, 0], atol=1e-14):
+                        return False, f"window (0,0) cap={cap}: O is not v_(i+delta)"
+                    if abs(lse[h, oq + i] - want) > 1e-12:
+                        return False, f"window (0,0) cap={cap}: LSE {lse[h, oq + i]} vs {want}"
+            oq += sq
+            ok_ += sk
+    # bounds at least as wide as the segment change nothing; (-1, 0) is causal
+    o0, l0 = oracle.fwd(q, k, v, cq, ck, scale, False, mutation=mutation)
+    o1, l1 = oracle.fwd(q, k, v, cq, ck, scale, False, window=(20, 20), mutation=mutation)
+    if not (_close(o1, o0, 1e-14)[0] and _close(l1, l0, 1e-14)[0]):
+        return False, "a window wider than the segment changed the result"
+    oc_, lc = oracle.fwd(q, k, v, cq, ck, scale, True, mutation=mutation)
+    ow, lw = oracle.fwd(q, k, v, cq, ck, scale, False, window=(-1, 0), mutation=mutation)
+    if not (_close(ow, oc_, 1e-14)[0] and _close(lw, lc, 1e-14)[0]):
+        return False, "window (-1, 0) differs from causal"
+    # a huge cap is no cap (tanh(x) = x to O(x^3))
+    oh, lh = oracle.fwd(q, k, v, cq, ck, scale, False, softcap=1e7, mutation=mutation)
+    if not (_close(oh, o0, 1e-9)[0] and _close(lh, l0, 1e-9)[0]):
+        return False, "softcap 1e7 differs from no softcap"
+    return True, "ok"
+
+
+def check_window_is_a_slice(mutation=0):
+    """Row i under window (L, R) equals unmasked attention over the key slice
+    [i + delta - L, i + delta + R] (clipped to the segment), computed by the
+    unmasked oracle on that slice alone."""
+    Hq, Hkv, D = 2, 2, 4
+    sq, sk = 9, 12
+    q, k, v = _rand((sq, Hq, D), 93), _rand((sk, Hkv, D), 94), _rand((sk, Hkv, D), 95)
+    for (L, R) in ((2, 1), (0, 3), (4, 0), (3, -1), (-1, 2)):
+        o, lse = oracle.fwd(q, k, v, _cu([sq]), _cu([sk]), 0.8, False, window=(L, R),
+                            mutation=mutation)
+        for i in range(sq):
+            d = i + sk - sq
+            lo = 0 if L < 0 else max(0, d - L)
+            hi = sk - 1 if R < 0 else min(sk - 1, d + R)
+            if hi < lo:
+                if not (np.all(o[i] == 0) and np.all(np.isneginf(lse[:, i]))):
+                    return False, f"window {(L, R)} row {i}: empty window not O=0, LSE=-inf"
+                continue
+            os_, ls_ = oracle.fwd(q[i:i + 1], k[lo:hi + 1], v[lo:hi + 1], _cu([1]),
+                                  _cu([hi + 1 - lo]), 0.8, False, mutation=mutation)
+            if not (_close(o[i:i + 1], os_, 1e-13)[0] and _close(lse[:, i:i + 1], ls_, 1e-13)[0]):
+                return False, f"window {(L, R)} row {i} differs from its key slice"
+    return True, "ok"
+
+
+MASK_CASES = [
+    # (lengths_q, lengths_k, Hq, Hkv, D, causal, window, softcap)
+    ([7], [7], 2, 1, 4, False, (2, 1), 0.0),
+    ([6, 4], [8, 4], 2, 1, 4, True, (3, -1), 0.0),
+    ([7], [7], 2, 2, 4, False, (-1, -1), 1.5),
+    ([5, 6], [5, 7], 4, 2, 4, True, (2, 0), 2.0),
+]
+
+
+def check_torch_reference_masks(mutation=0, tol=1e-12):
+    for ci, (lq, lk, Hq, Hkv, D, causal, win, cap) in enumerate(MASK_CASES):
+        Tq, Tk = sum(lq), sum(lk)
+        q, k, v = _rand((Tq, Hq, D), 150 + ci), _rand((Tk, Hkv, D), 160 + ci), _rand((Tk, Hkv, D), 170 + ci)
+        do = _rand((Tq, Hq, D), 180 + ci)
+        scale = 0.9
+        cq, ck = _cu(lq), _cu(lk)
+        o, lse = oracle.fwd(q, k, v, cq, ck, scale, causal, window=win, softcap=cap,
+                            mutation=mutation)
+        dq, dk, dv = oracle.bwd(q, k, v, do, cq, ck, scale, causal, window=win, softcap=cap,
+                                mutation=mutation)
+        ro, rlse, (rdq, rdk, rdv) = torch_reference(q, k, v, do, lq, lk, scale, causal,
+                                                    window=win, softcap=cap)
+        for name, a, b in (("O", o, ro), ("LSE", lse, rlse), ("dQ", dq, rdq),
+                           ("dK", dk, rdk), ("dV", dv, rdv)):
+            ok, msg = _close(a, b, tol)
+            if not ok:
+                return False, f"torch mask case {ci} {name}: {msg}"
+    return True, "ok"
+
+
+def check_finite_differences_masks(mutation=0, eps=1e-6, tol=1e-6):
+    for ci, (lq, lk, Hq, Hkv, D, causal, win, cap) in enumerate(MASK_CASES):
+        Tq, Tk = sum(lq), sum(lk)
+        q, k, v = _rand((Tq, Hq, D), 110 + ci), _rand((Tk, Hkv, D), 120 + ci), _rand((Tk, Hkv, D), 130 + ci)
+        do = _rand((Tq, Hq, D), 140 + ci)
+        scale = 0.7
+        cq, ck = _cu(lq), _cu(lk)
+        dq, dk, dv = oracle.bwd(q, k, v, do, cq, ck, scale, causal, window=win, softcap=cap,
+                                mutation=mutation)
+
+        def loss():
+            o, _ = oracle.fwd(q, k, v, cq, ck, scale, causal, window=win, softcap=cap,
+                              mutation=mutation)
+            return float(np.sum(o * do))
+
+        for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            num = np.zeros_like(x)
+            flat = x.reshape(-1)
+            for t in range(flat.size):
+                old = flat[t]
+                flat[t] = old + eps
+                lp = loss()
+                flat[t] = old - eps
+                lm = loss()
+                flat[t] = old
+                num.reshape(-1)[t] = (lp - lm) / (2 * eps)
+            ok, msg = _close(g, num, tol)
+            if not ok:
+                return False, f"FD mask case {ci} d{name}: {msg}"
+    return True, "ok"
+
+
 ALL_CHECKS = [
+    check_window_softcap_closed_forms,
+    check_window_is_a_slice,
     check_closed_forms,
     check_lse_logsumexp,
     check_gradient_identities,
@@ -355,5 +503,7 @@ ALL_CHECKS = [
     check_rows_match_full,
     check_fully_masked_rows,
     check_torch_reference,
+    check_torch_reference_masks,
     check_finite_differences,
+    check_finite_differences_masks,
 ]

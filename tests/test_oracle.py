@@ -84,6 +84,9 @@ MUTATIONS = {
     5: "LSE drops the max term",
     6: "dK multiplies dS by dO instead of Q",
     7: "D_i drops the O factor",
+    8: "the window's far edge is excluded",
+    9: "the softcap's derivative is dropped from dS",
+    10: "the softcap is applied to the unscaled score",
 }
 
 
