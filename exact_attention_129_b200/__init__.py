@@ -8,7 +8,7 @@ missing or the tensors are not on a CUDA device, calls raise.
 Functions
 ---------
 attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, ...)
-    -> (out, lse)
+    -> (out, lse); causal, window=(left, right) and softcap options
 attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, ...)
     -> (dq, dk, dv)
 attention(...)  autograd-aware forward (backward through attn_bwd)
@@ -28,9 +28,9 @@ __all__ = ["attn_fwd", "attn_bwd", "attention", "bwd_workspace_size", "last_devi
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED",
           3: "ATTN_ERR_CUDA", 4: "ATTN_ERR_TIMEOUT", 5: "ATTN_ERR_SCRATCH_TOO_SMALL"}
-EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_last_device_error",
-            "attn_set_timing_events", "attn_bwd_static_scratch", "attn_watchdog_selftest",
-            "attn_version")
+EXPORTED = ("attn_fwd", "attn_bwd", "attn_fwd_ex", "attn_bwd_ex", "attn_bwd_workspace_size",
+            "attn_last_device_error", "attn_set_timing_events", "attn_bwd_static_scratch",
+            "attn_watchdog_selftest", "attn_version")
 KERNEL_FWD, KERNEL_BWD_MAIN = 0, 1
 
 
@@ -58,6 +58,13 @@ def library() -> ctypes.CDLL:
         lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                  i32, i32, f32, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
         lib.attn_bwd.restype = ctypes.c_int
+        lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                    i32, f32, i32, i32, i32, f32, i32, vp, vp, vp]
+        lib.attn_fwd_ex.restype = ctypes.c_int
+        lib.attn_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                    i32, i32, i32, f32, i32, i32, i32, f32, vp, vp, vp, vp,
+                                    ctypes.c_size_t, vp]
+        lib.attn_bwd_ex.restype = ctypes.c_int
         lib.attn_bwd_workspace_size.argtypes = [i32, i32, i32, i32]
         lib.attn_bwd_workspace_size.restype = ctypes.c_size_t
         lib.attn_last_device_error.argtypes = [vp, ctypes.c_char_p, ctypes.c_size_t]
@@ -96,9 +103,21 @@ def _check_layout(name, t, dtype):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _window(window):
+    if window is None:
+        return -1, -1
+    left, right = window
+    return (-1 if left is None else int(left)), (-1 if right is None else int(right))
+
+
 def attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
-             scale=None, causal=False, return_lse=True, out=None, lse=None):
-    """Forward pass. q [Tq,Hq,D], k/v [Tk,Hkv,D] bf16; returns (out, lse or None)."""
+             scale=None, causal=False, window=None, softcap=0.0, return_lse=True, out=None,
+             lse=None):
+    """Forward pass. q [Tq,Hq,D], k/v [Tk,Hkv,D] bf16; returns (out, lse or None).
+
+    ``window`` = (left, right): with delta = s_k - s_q, row i sees keys
+    [i + delta - left, i + delta + right]; None or a negative side = no bound.
+    ``softcap`` > 0 caps each scaled score at softcap * tanh(s / softcap)."""
     _check_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k, out, lse)
     for n, t in (("q", q), ("k", k), ("v", v)):
         _check_layout(n, t, torch.bfloat16)
@@ -112,11 +131,12 @@ def attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
         out = torch.empty_like(q)
     if return_lse and lse is None:
         lse = torch.empty((hq, tq), device=q.device, dtype=torch.float32)
-    rc = library().attn_fwd(
+    wl, wr = _window(window)
+    rc = library().attn_fwd_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
         cu_seqlens_q.numel() - 1, tq, tk, int(max_seqlen_q), int(max_seqlen_k), hq, hkv, d,
-        float(scale), int(bool(causal)), int(bool(return_lse)), _ptr(out),
-        _ptr(lse) if return_lse else None, _stream(q.device))
+        float(scale), int(bool(causal)), wl, wr, float(softcap or 0.0),
+        int(bool(return_lse)), _ptr(out), _ptr(lse) if return_lse else None, _stream(q.device))
     if rc != 0:
         raise AttnError("attn_fwd", rc)
     return out, (lse if return_lse else None)
@@ -127,8 +147,10 @@ def bwd_workspace_size(batch, total_q, nheads_q, head_dim) -> int:
 
 
 def attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-             *, scale=None, causal=False, dq=None, dk=None, dv=None, workspace=None):
-    """Backward pass; returns (dq, dk, dv) in the layouts of q, k, v."""
+             *, scale=None, causal=False, window=None, softcap=0.0, dq=None, dk=None, dv=None,
+             workspace=None):
+    """Backward pass; returns (dq, dk, dv) in the layouts of q, k, v.  ``causal``,
+    ``window`` and ``softcap`` must match the forward call."""
     _check_cuda(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, dq, dk, dv, workspace)
     for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
         _check_layout(n, t, torch.bfloat16)
@@ -144,11 +166,13 @@ def attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, 
     need = bwd_workspace_size(batch, tq, hq, d)
     if workspace is None:
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
-    rc = library().attn_bwd(
+    wl, wr = _window(window)
+    rc = library().attn_bwd_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(cu_seqlens_q),
         _ptr(cu_seqlens_k), batch, tq, tk, int(max_seqlen_q), int(max_seqlen_k), hq, hkv, d,
-        float(scale), int(bool(causal)), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(q.device))
+        float(scale), int(bool(causal)), wl, wr, float(softcap or 0.0), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(q.device))
     if rc != 0:
         raise AttnError("attn_bwd", rc)
     return dq, dk, dv
@@ -176,26 +200,28 @@ def last_device_error(stream=None):
 
 class _Attention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, scale, causal):
+    def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, scale, causal, window, softcap):
         out, lse = attn_fwd(q, k, v, cu_q, cu_k, max_q, max_k, scale=scale, causal=causal,
-                            return_lse=True)
+                            window=window, softcap=softcap, return_lse=True)
         ctx.save_for_backward(q, k, v, out, lse, cu_q, cu_k)
-        ctx.args = (max_q, max_k, scale, causal)
+        ctx.args = (max_q, max_k, scale, causal, window, softcap)
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, out, lse, cu_q, cu_k = ctx.saved_tensors
-        max_q, max_k, scale, causal = ctx.args
+        max_q, max_k, scale, causal, window, softcap = ctx.args
         dq, dk, dv = attn_bwd(q, k, v, out, lse, dout.contiguous(), cu_q, cu_k, max_q, max_k,
-                              scale=scale, causal=causal)
-        return dq, dk, dv, None, None, None, None, None, None
+                              scale=scale, causal=causal, window=window, softcap=softcap)
+        return dq, dk, dv, None, None, None, None, None, None, None, None
 
 
 def attention(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
-              scale=None, causal=False):
-    """Differentiable exact attention over packed variable-length segments."""
+              scale=None, causal=False, window=None, softcap=0.0):
+    """Differentiable exact attention over packed variable-length segments, with
+    an optional local window (left, right) and softcap (see attn_fwd)."""
     if scale is None:
         scale = q.shape[-1] ** -0.5
     return _Attention.apply(q, k, v, cu_seqlens_q, cu_seqlens_k, int(max_seqlen_q),
-                            int(max_seqlen_k), float(scale), bool(causal))
+                            int(max_seqlen_k), float(scale), bool(causal), window,
+                            float(softcap or 0.0))

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -159,7 +160,34 @@ attn_status_t check_common(const void* q, const void* k, const void* v,
   return ATTN_OK;
 }
 
-template <int D, bool CAUSAL>
+// Window and softcap arguments turned into the kernels' form.  With delta =
+// s_k - s_q, row i sees keys [i + delta - lo_off, i + delta + hi_off].
+struct MaskArgs {
+  bool upper;    // an upper key bound exists (causal or window_right >= 0)
+  int hi_off;
+  int lo_off;    // kNoBound: none
+  bool softcap;
+  float cap_k;   // scale / c
+  float cap_log2;  // c * log2(e)
+};
+
+attn_status_t mask_args(int32_t causal, int32_t window_left, int32_t window_right,
+                        float softcap, float scale, MaskArgs* m) {
+  if (!std::isfinite(softcap) || softcap < 0.f) return ATTN_ERR_INVALID_ARG;
+  // bounds past any possible segment length mean no bound
+  const int32_t kFar = kNoBound - 1;
+  const int32_t wl = window_left < 0 ? -1 : std::min(window_left, kFar);
+  const int32_t wr = window_right < 0 ? -1 : std::min(window_right, kFar);
+  m->upper = causal != 0 || wr >= 0;
+  m->hi_off = causal ? (wr >= 0 ? std::min(wr, 0) : 0) : (wr >= 0 ? wr : kNoBound);
+  m->lo_off = wl >= 0 ? wl : kNoBound;
+  m->softcap = softcap > 0.f;
+  m->cap_k = m->softcap ? scale / softcap : 0.f;
+  m->cap_log2 = m->softcap ? softcap * 1.4426950408889634f : 0.f;
+  return ATTN_OK;
+}
+
+template <int D, bool CAUSAL, bool SOFTCAP>
 attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_q, int total_k,
                          int hkv, const FwdParams& p, int batch, int hq, int max_q,
                          cudaStream_t stream) {
@@ -175,7 +203,7 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_
   cudaGetDevice(&dev);
   cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once[dev], [&] {
-    attr_err = cudaFuncSetAttribute(attn_fwd_kernel<D, CAUSAL>,
+    attr_err = cudaFuncSetAttribute(attn_fwd_kernel<D, CAUSAL, SOFTCAP>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
@@ -183,13 +211,14 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_
   if (m_tiles == 0) return ATTN_OK;
   dim3 grid(m_tiles, hq, batch);
   record_start(ATTN_KERNEL_FWD, stream);
-  attn_fwd_kernel<D, CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  attn_fwd_kernel<D, CAUSAL, SOFTCAP><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv,
+                                                                                  p);
   const cudaError_t e = cudaGetLastError();
   record_stop(ATTN_KERNEL_FWD, stream);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SOFTCAP>
 attn_status_t launch_bwd_main(const BwdArgs& a, const BwdParams& bp, cudaStream_t stream) {
   using C = BwdCfg<D>;
   static std::once_flag attr_once[kMaxDevices];
@@ -197,7 +226,7 @@ attn_status_t launch_bwd_main(const BwdArgs& a, const BwdParams& bp, cudaStream_
   cudaGetDevice(&dev);
   cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once[dev], [&] {
-    attr_err = cudaFuncSetAttribute(attn_bwd_main_kernel<D, CAUSAL>,
+    attr_err = cudaFuncSetAttribute(attn_bwd_main_kernel<D, CAUSAL, SOFTCAP>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
@@ -212,8 +241,8 @@ attn_status_t launch_bwd_main(const BwdArgs& a, const BwdParams& bp, cudaStream_
   if (n_blocks == 0) return ATTN_OK;
   dim3 grid(n_blocks * C::NSPLIT, a.hkv, a.batch);
   record_start(ATTN_KERNEL_BWD_MAIN, stream);
-  attn_bwd_main_kernel<D, CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mk, mv, mq, mo, mdq,
-                                                                                bp);
+  attn_bwd_main_kernel<D, CAUSAL, SOFTCAP><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
+      mk, mv, mq, mo, mdq, bp);
   const cudaError_t e = cudaGetLastError();
   record_stop(ATTN_KERNEL_BWD_MAIN, stream);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -247,10 +276,19 @@ attn_status_t bwd_launch_d(const BwdArgs& a, cudaStream_t stream) {
   bp.nheads_kv = a.hkv;
   bp.scale = a.scale;
   bp.scale_log2 = a.scale * 1.4426950408889634f;
+  bp.hi_off = a.hi_off;
+  bp.lo_off = a.lo_off;
+  bp.cap_k = a.cap_k;
+  bp.cap_log2 = a.cap_log2;
   bp.timeout_ns = a.timeout_ns;
   if (a.total_k > 0) {
-    attn_status_t st = a.causal ? launch_bwd_main<D, true>(a, bp, stream)
-                                : launch_bwd_main<D, false>(a, bp, stream);
+    attn_status_t st;
+    if (a.softcap)
+      st = a.upper ? launch_bwd_main<D, true, true>(a, bp, stream)
+                   : launch_bwd_main<D, false, true>(a, bp, stream);
+    else
+      st = a.upper ? launch_bwd_main<D, true, false>(a, bp, stream)
+                   : launch_bwd_main<D, false, false>(a, bp, stream);
     if (st != ATTN_OK) return st;
   }
   if (n_rh > 0) {
@@ -277,16 +315,20 @@ attn_status_t bwd_launch(const BwdArgs& a, cudaStream_t stream) {
 
 using namespace attn;
 
-extern "C" attn_status_t attn_fwd(const void* q, const void* k, const void* v,
-                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
-                                  int32_t batch, int32_t total_q, int32_t total_k,
-                                  int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t nheads_q,
-                                  int32_t nheads_kv, int32_t head_dim, float scale,
-                                  int32_t causal, int32_t return_lse, void* out, float* lse,
-                                  attn_stream_t stream) {
+extern "C" attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v,
+                                     const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                     int32_t batch, int32_t total_q, int32_t total_k,
+                                     int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                     int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                                     float scale, int32_t causal, int32_t window_left,
+                                     int32_t window_right, float softcap, int32_t return_lse,
+                                     void* out, float* lse, attn_stream_t stream) {
   attn_status_t st = check_common(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
                                   max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim,
                                   scale);
+  if (st != ATTN_OK) return st;
+  MaskArgs mk;
+  st = mask_args(causal, window_left, window_right, softcap, scale, &mk);
   if (st != ATTN_OK) return st;
   if (!out || !aligned16(out)) return ATTN_ERR_INVALID_ARG;
   if (return_lse && (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u))) return ATTN_ERR_INVALID_ARG;
@@ -307,22 +349,54 @@ extern "C" attn_status_t attn_fwd(const void* q, const void* k, const void* v,
   p.nheads_kv = nheads_kv;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.return_lse = return_lse ? 1 : 0;
+  p.hi_off = mk.hi_off;
+  p.lo_off = mk.lo_off;
+  p.cap_k = mk.cap_k;
+  p.cap_log2 = mk.cap_log2;
   p.timeout_ns = wait_timeout_ns();
   p.epilogue_delay_ns = test_epilogue_delay_ns();
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool c = causal != 0;
   auto run = [&](auto launch) {
     return launch(q, k, v, total_q, total_k, nheads_kv, p, batch, nheads_q, max_seqlen_q, s);
   };
+  // the kernel's CAUSAL parameter means "rows have an upper key bound"
+  const int variant = (mk.upper ? 1 : 0) | (mk.softcap ? 2 : 0);
   switch (head_dim) {
     case 64:
-      return c ? run(launch_fwd<64, true>) : run(launch_fwd<64, false>);
+      switch (variant) {
+        case 0: return run(launch_fwd<64, false, false>);
+        case 1: return run(launch_fwd<64, true, false>);
+        case 2: return run(launch_fwd<64, false, true>);
+        default: return run(launch_fwd<64, true, true>);
+      }
     case 128:
-      return c ? run(launch_fwd<128, true>) : run(launch_fwd<128, false>);
+      switch (variant) {
+        case 0: return run(launch_fwd<128, false, false>);
+        case 1: return run(launch_fwd<128, true, false>);
+        case 2: return run(launch_fwd<128, false, true>);
+        default: return run(launch_fwd<128, true, true>);
+      }
     default:
-      return c ? run(launch_fwd<256, true>) : run(launch_fwd<256, false>);
+      switch (variant) {
+        case 0: return run(launch_fwd<256, false, false>);
+        case 1: return run(launch_fwd<256, true, false>);
+        case 2: return run(launch_fwd<256, false, true>);
+        default: return run(launch_fwd<256, true, true>);
+      }
   }
+}
+
+extern "C" attn_status_t attn_fwd(const void* q, const void* k, const void* v,
+                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                  int32_t batch, int32_t total_q, int32_t total_k,
+                                  int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t nheads_q,
+                                  int32_t nheads_kv, int32_t head_dim, float scale,
+                                  int32_t causal, int32_t return_lse, void* out, float* lse,
+                                  attn_stream_t stream) {
+  return attn_fwd_ex(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                     max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim, scale, causal,
+                     -1, -1, 0.f, return_lse, out, lse, stream);
 }
 
 extern "C" size_t attn_bwd_workspace_size(int32_t batch, int32_t total_q, int32_t nheads_q,
@@ -331,17 +405,22 @@ extern "C" size_t attn_bwd_workspace_size(int32_t batch, int32_t total_q, int32_
   return bwd_workspace_bytes(batch, total_q, nheads_q, head_dim);
 }
 
-extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
-                                  const float* lse, const void* dout,
-                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
-                                  int32_t batch, int32_t total_q, int32_t total_k,
-                                  int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t nheads_q,
-                                  int32_t nheads_kv, int32_t head_dim, float scale,
-                                  int32_t causal, void* dq, void* dk, void* dv, void* workspace,
-                                  size_t workspace_bytes, attn_stream_t stream) {
+extern "C" attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v,
+                                     const void* out, const float* lse, const void* dout,
+                                     const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                     int32_t batch, int32_t total_q, int32_t total_k,
+                                     int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                     int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                                     float scale, int32_t causal, int32_t window_left,
+                                     int32_t window_right, float softcap, void* dq, void* dk,
+                                     void* dv, void* workspace, size_t workspace_bytes,
+                                     attn_stream_t stream) {
   attn_status_t st = check_common(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
                                   max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim,
                                   scale);
+  if (st != ATTN_OK) return st;
+  MaskArgs mk;
+  st = mask_args(causal, window_left, window_right, softcap, scale, &mk);
   if (st != ATTN_OK) return st;
   if (!out || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
@@ -360,11 +439,26 @@ extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, c
   a.batch = batch; a.total_q = total_q; a.total_k = total_k;
   a.max_q = max_seqlen_q; a.max_k = max_seqlen_k;
   a.hq = nheads_q; a.hkv = nheads_kv; a.d = head_dim;
-  a.scale = scale; a.causal = causal != 0;
+  a.scale = scale;
+  a.upper = mk.upper; a.hi_off = mk.hi_off; a.lo_off = mk.lo_off;
+  a.softcap = mk.softcap; a.cap_k = mk.cap_k; a.cap_log2 = mk.cap_log2;
   a.dq = dq; a.dk = dk; a.dv = dv; a.workspace = workspace;
   a.err = ds->err;
   a.timeout_ns = wait_timeout_ns();
   return bwd_launch(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                                  const float* lse, const void* dout,
+                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                  int32_t batch, int32_t total_q, int32_t total_k,
+                                  int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t nheads_q,
+                                  int32_t nheads_kv, int32_t head_dim, float scale,
+                                  int32_t causal, void* dq, void* dk, void* dv, void* workspace,
+                                  size_t workspace_bytes, attn_stream_t stream) {
+  return attn_bwd_ex(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, batch, total_q,
+                     total_k, max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim, scale,
+                     causal, -1, -1, 0.f, dq, dk, dv, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -32,6 +32,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "attn.h"
 #include "ptx.cuh"
@@ -50,7 +51,10 @@ struct BwdArgs {
   const int32_t *cu_q, *cu_k;
   int batch, total_q, total_k, max_q, max_k, hq, hkv, d;
   float scale;
-  bool causal;
+  bool upper;              // rows have an upper key bound (causal or a right window)
+  int hi_off, lo_off;      // window offsets, as in BwdParams
+  bool softcap;
+  float cap_k, cap_log2;
   void *dq, *dk, *dv, *workspace;
   uint32_t* err;
   uint64_t timeout_ns;
@@ -78,6 +82,14 @@ struct BwdParams {
   int nheads_kv;
   float scale;
   float scale_log2;
+  // keys allowed for segment-local query row i, with delta = s_k - s_q:
+  // [i + delta - lo_off, i + delta + hi_off] (kNoBound = none; the upper
+  // bound exists iff the kernel's CAUSAL parameter is set)
+  int hi_off;
+  int lo_off;
+  // softcap c: scores c tanh(s / c); cap_k = scale / c, cap_log2 = c log2(e)
+  float cap_k;
+  float cap_log2;
   uint64_t timeout_ns;
 };
 
@@ -196,15 +208,15 @@ __device__ __forceinline__ bool bwd_tile(const BwdParams& p, BwdTile& t) {
   t.sk = p.cu_k[b + 1] - t.k0;
   t.n_base = nb * C::BN;
   if (t.n_base >= t.sk) return false;
-  t.m_hi = (t.sq + C::BM - 1) / C::BM;
-  t.m_lo = 0;
-  if (CAUSAL) {
-    // query row i sees key j iff j <= i + (sk - sq): the first row that sees
-    // this block's first key is n_base - (sk - sq)
-    const int first = t.n_base - (t.sk - t.sq);
-    t.m_lo = first > 0 ? first / C::BM : 0;
-  }
-  if (t.m_lo > t.m_hi) t.m_lo = t.m_hi;
+  // query rows that see a key of [n_base, n_base + BN): row i sees key j iff
+  // i + delta - lo_off <= j <= i + delta + hi_off
+  const int delta = t.sk - t.sq;
+  int row_lo = 0, row_hi = t.sq;  // [row_lo, row_hi)
+  if (CAUSAL) row_lo = max(0, t.n_base - delta - p.hi_off);
+  if (p.lo_off < kNoBound) row_hi = min(t.sq, t.n_base + C::BN - delta + p.lo_off);
+  t.m_lo = row_lo / C::BM;
+  t.m_hi = (row_hi + C::BM - 1) / C::BM;
+  if (row_hi <= row_lo || t.m_lo > t.m_hi) t.m_hi = t.m_lo;
   t.n_iter = t.G * (t.m_hi - t.m_lo);
   return true;
 }
@@ -489,7 +501,7 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, const BwdTile& t, co
 // ---------------------------------------------------------------------------
 // elementwise warps: thread = key row
 // ---------------------------------------------------------------------------
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SOFTCAP>
 __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, const BwdSmem& s,
                                          uint32_t tmem, const CUtensorMap* tmDQ) {
   // two warpgroups: warpgroup wg handles query columns [32 wg, 32 wg + 32) of
@@ -578,11 +590,18 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     if (tid == 0 && i < 200) TRACE(i * 8 + 1);
     __syncwarp();
     if (lane == 0) mbar_arrive(s.dp_free);
-    // causal: query column x of this block sees this key iff m0 + x >= kr - causal_off
-    const int jmin = CAUSAL ? (kr - causal_off - m0 - qc0) : 0;
+    // query column x of this block (row m0 + qc0 + x) sees this key iff
+    // x in [xmin, xmax]: kr <= row + delta + hi_off and kr >= row + delta - lo_off
+    const int xmin = CAUSAL ? (kr - causal_off - p.hi_off - m0 - qc0) : -kNoBound;
+    const int xmax = (p.lo_off < kNoBound) ? (kr - causal_off + p.lo_off - m0 - qc0) : kNoBound;
     uint32_t pk[16];
     uint4 dsk[4];
     const uint64_t c2 = f2_pack(c, c);
+    // most threads have all 32 of their query columns allowed: only the others
+    // run the per-element mask
+    const bool all_in = key_ok && xmin <= 0 && xmax >= 31;
+    auto pairs = [&](auto masked_tag) {
+    constexpr bool MASKED = decltype(masked_tag)::value;
 #pragma unroll
     for (int x4 = 0; x4 < 8; ++x4) {
       const float4 l4 = reinterpret_cast<const float4*>(lse2)[x4];
@@ -591,14 +610,26 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
       for (int hp = 0; hp < 2; ++hp) {
         const int x = x4 * 4 + hp * 2;
         float e0, e1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[x]), __uint_as_float(sr[x + 1])), c2,
-                         hp ? f2_pack(-l4.z, -l4.w) : f2_pack(-l4.x, -l4.y)),
-                  e0, e1);
+        float g0 = 1.f, g1 = 1.f;  // d(capped score) / d(scaled score)
+        if constexpr (SOFTCAP) {
+          const float t0 = tanhf(__uint_as_float(sr[x]) * p.cap_k);
+          const float t1 = tanhf(__uint_as_float(sr[x + 1]) * p.cap_k);
+          e0 = p.cap_log2 * t0 - (hp ? l4.z : l4.x);
+          e1 = p.cap_log2 * t1 - (hp ? l4.w : l4.y);
+          g0 = 1.f - t0 * t0;
+          g1 = 1.f - t1 * t1;
+        } else {
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[x]), __uint_as_float(sr[x + 1])), c2,
+                           hp ? f2_pack(-l4.z, -l4.w) : f2_pack(-l4.x, -l4.y)),
+                    e0, e1);
+        }
         float p0 = ex2(e0), p1 = ex2(e1);
-        if (!key_ok || (CAUSAL && x < jmin)) p0 = 0.f;
-        if (!key_ok || (CAUSAL && x + 1 < jmin)) p1 = 0.f;
+        if (MASKED) {
+          if (!key_ok || x < xmin || x > xmax) p0 = 0.f;
+          if (!key_ok || x + 1 < xmin || x + 1 > xmax) p1 = 0.f;
+        }
         float d0, d1;
-        f2_unpack(f2_mul(f2_pack(p0, p1),
+        f2_unpack(f2_mul(f2_pack(p0 * g0, p1 * g1),
                          f2_add(f2_pack(__uint_as_float(dr[x]), __uint_as_float(dr[x + 1])),
                                 hp ? f2_pack(-d4.z, -d4.w) : f2_pack(-d4.x, -d4.y))),
                   d0, d1);
@@ -611,6 +642,11 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
         else dsk[x >> 3].w = dpk;
       }
     }
+    };
+    if (all_in)
+      pairs(std::integral_constant<bool, false>());
+    else
+      pairs(std::integral_constant<bool, true>());
     // P (bf16 pairs) goes over the first 16 of this warpgroup's own 32 score
     // columns, which this warpgroup has already read: the other warpgroup may
     // still be reading its own columns
@@ -674,7 +710,7 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SOFTCAP>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
@@ -733,7 +769,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *s.tmem_base;
   if (warp < 8) {
-    bwd_elem<D, CAUSAL>(p, t, s, tmem, &tmDQ);
+    bwd_elem<D, CAUSAL, SOFTCAP>(p, t, s, tmem, &tmDQ);
   } else if (warp == C::LOAD_WARP) {
     bwd_load<D>(p, t, s, &tmK, &tmV, &tmQ, &tmO);
   } else {

@@ -68,11 +68,26 @@ struct FwdParams {
   int nheads_kv;
   float scale_log2;  // scale * log2(e)
   int return_lse;
+  // keys allowed for segment-local query row i, with delta = s_k - s_q:
+  //   [i + delta - lo_off, i + delta + hi_off]  (kNoBound = no bound; the
+  //   upper bound exists iff the kernel's CAUSAL parameter is set)
+  int hi_off;
+  int lo_off;
+  // softcap c: scores become c tanh(s / c); cap_k = scale / c, cap_log2 = c log2(e)
+  float cap_k;
+  float cap_log2;
   uint64_t timeout_ns;
   // test hook (0 in normal use): the softmax warps idle this long before their
   // final wait, so the tile's last P.V is sure to have completed by then
   uint64_t epilogue_delay_ns;
 };
+
+// softcap of one score (fp32 bits): c tanh(s scale / c) in the log2 domain,
+// i.e. c log2(e) tanh(s cap_k); masked scores (-inf) stay -inf
+__device__ __forceinline__ uint32_t fwd_cap(const FwdParams& p, uint32_t bits) {
+  const float x = __uint_as_float(bits);
+  return x == -INFINITY ? bits : __float_as_uint(p.cap_log2 * tanhf(x * p.cap_k));
+}
 
 __device__ __forceinline__ void fwd_test_delay(const FwdParams& p) {
   if (p.epilogue_delay_ns == 0) return;
@@ -174,7 +189,8 @@ __device__ __forceinline__ FwdSmem fwd_smem(uint8_t* base) {
 struct FwdTile {
   int q0, sq, k0, sk;   // segment offsets / lengths
   int m_base;           // first segment-local row of the CTA
-  int n_blocks;         // key blocks to visit
+  int n_lo;             // first key block to visit
+  int n_blocks;         // key blocks to visit: [n_lo, n_lo + n_blocks)
   int h, hk;
 };
 
@@ -192,12 +208,16 @@ __device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t) {
   const int m_tile = CAUSAL ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
   t.m_base = m_tile * C::BM * C::NQ;
   if (t.m_base >= t.sq) return false;
+  // the union of the rows' allowed key ranges
+  const int delta = t.sk - t.sq;
   int n_end = t.sk;
   if (CAUSAL) {
     const int last_row = min(t.sq, t.m_base + C::BM * C::NQ) - 1;
-    n_end = min(t.sk, last_row + (t.sk - t.sq) + 1);
+    n_end = min(t.sk, last_row + delta + p.hi_off + 1);
   }
-  t.n_blocks = n_end > 0 ? (n_end + C::BN - 1) / C::BN : 0;
+  const int n_beg = (p.lo_off < kNoBound) ? max(0, t.m_base + delta - p.lo_off) : 0;
+  t.n_lo = n_beg / C::BN;
+  t.n_blocks = n_end > n_beg ? (n_end + C::BN - 1) / C::BN - t.n_lo : 0;
   return true;
 }
 
@@ -245,13 +265,13 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, c
   };
   // K block j: one chunk per 64-column panel (BN rows, K-major)
   auto load_k = [&](uint8_t* dst, uint64_t* full, int j, int c) {
-    tma_load_3d(dst, tmK, full, c * 64, t.hk, t.k0 + j * C::BN);
+    tma_load_3d(dst, tmK, full, c * 64, t.hk, t.k0 + (t.n_lo + j) * C::BN);
   };
   // rows [c*VROWS, (c+1)*VROWS) of V block j: all D columns, panel by panel
   auto load_v = [&](uint8_t* dst, uint64_t* full, int j, int c) {
     for (int pn = 0; pn < C::PANELS; ++pn)
       tma_load_3d(dst + pn * (C::VROWS * 128), tmV, full, pn * 64, t.hk,
-                  t.k0 + j * C::BN + c * C::VROWS);
+                  t.k0 + (t.n_lo + j) * C::BN + c * C::VROWS);
   };
   const int n = t.n_blocks;
   uint8_t* base;
@@ -453,7 +473,7 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
 // ---------------------------------------------------------------------------
 // softmax warpgroup: one thread per query row
 // ---------------------------------------------------------------------------
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SOFTCAP>
 __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t,
                                             const FwdSmem& s, uint32_t tmem, int qt) {
   using C = FwdCfg<D>;
@@ -463,13 +483,18 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   const int row = t.m_base + qt * C::BM + row_in_tile;  // segment-local query row
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
   const int n = t.n_blocks;
-  const float c = p.scale_log2;
-  // keys [0, key_lim) are allowed for this row
-  const int key_lim = CAUSAL ? min(t.sk, row + (t.sk - t.sq) + 1) : t.sk;
-  // block j needs element masks for this warpgroup when it crosses the causal
-  // diagonal of the tile's first row or the end of the keys
+  // with a softcap the scores are turned into capped log2-domain values first
+  const float c = SOFTCAP ? 1.f : p.scale_log2;
+  // keys [key_lo, key_lim) are allowed for this row
+  const int delta = t.sk - t.sq;
+  const int key_lim = CAUSAL ? min(t.sk, row + delta + p.hi_off + 1) : t.sk;
+  const int key_lo = row + delta - p.lo_off;
+  // a block needs element masks for this warpgroup when it crosses the upper
+  // bound of the tile's first row (or the end of the keys) or the lower bound
+  // of its last row
   const int tile_row0 = t.m_base + qt * C::BM;
-  const int mask_from = CAUSAL ? min(t.sk, tile_row0 + (t.sk - t.sq) + 1) : t.sk;
+  const int mask_from = CAUSAL ? min(t.sk, tile_row0 + delta + p.hi_off + 1) : t.sk;
+  const int lo_until = tile_row0 + (C::BM - 1) + delta - p.lo_off;
 
   // With two query tiles, warp w of each tile shares an SM sub-partition and
   // its special-function unit: their exp phases take turns (tile 0 first in
@@ -513,12 +538,17 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     if constexpr (NCOL == 128) tmem_ld128(s_addr, sr);
     else tmem_ld64(s_addr, sr);
     if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 1);
-    const bool masked = (j + 1) * C::BN > mask_from;
+    const int kb = (t.n_lo + j) * C::BN;  // segment-local key of column 0
+    const bool masked = (kb + C::BN > mask_from) || (kb < lo_until);
     if (masked) {
-      const int lim = key_lim - j * C::BN;
+      const int lim = key_lim - kb, lo = key_lo - kb;
 #pragma unroll
       for (int i = 0; i < NCOL; ++i)
-        if (i >= lim) sr[i] = 0xff800000u;  // -inf
+        if (i >= lim || i < lo) sr[i] = 0xff800000u;  // -inf
+    }
+    if constexpr (SOFTCAP) {
+#pragma unroll
+      for (int i = 0; i < NCOL; ++i) sr[i] = fwd_cap(p, sr[i]);
     }
     // row max: 8 independent chains of three-input max, then a short tree
     float mx;
@@ -712,7 +742,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
 // row sums.  Every thread meets every barrier, also after a timed-out wait
 // (then it only plays the barriers), so its partner never blocks for good.
 // ---------------------------------------------------------------------------
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SOFTCAP>
 __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdTile& t,
                                                   const FwdSmem& s, uint32_t tmem, int qt,
                                                   int hf) {
@@ -726,10 +756,13 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
   const int row = t.m_base + qt * C::BM + row_in_tile;
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
   const int n = t.n_blocks;
-  const float c = p.scale_log2;
-  const int key_lim = CAUSAL ? min(t.sk, row + (t.sk - t.sq) + 1) : t.sk;
+  const float c = SOFTCAP ? 1.f : p.scale_log2;
+  const int delta = t.sk - t.sq;
+  const int key_lim = CAUSAL ? min(t.sk, row + delta + p.hi_off + 1) : t.sk;
+  const int key_lo = row + delta - p.lo_off;
   const int tile_row0 = t.m_base + qt * C::BM;
-  const int mask_from = CAUSAL ? min(t.sk, tile_row0 + (t.sk - t.sq) + 1) : t.sk;
+  const int mask_from = CAUSAL ? min(t.sk, tile_row0 + delta + p.hi_off + 1) : t.sk;
+  const int lo_until = tile_row0 + (C::BM - 1) + delta - p.lo_off;
   const int pair_bar = 3 + qt * 4 + quad;
   float* xch = s.xch + qt * (2 * 2 * C::BM);  // [block parity][half][row]
 
@@ -747,19 +780,26 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
     const uint32_t s_addr = tmem + lane_base + slot * C::BN;
     uint32_t sa[32], sb[16];  // keys 32 hf + i, then 64 + 16 hf + i
     float mx = -INFINITY;
-    const bool masked = (j + 1) * C::BN > mask_from;
+    const int kb = (t.n_lo + j) * C::BN;  // segment-local key of column 0
+    const bool masked = (kb + C::BN > mask_from) || (kb < lo_until);
     TRACE(tr);
     if (ok) {
       tc_fence_after();
       tmem_ld32_16(s_addr + hf * 32, sa, s_addr + 64 + hf * 16, sb);
       if (masked) {
-        const int lim = key_lim - j * C::BN;
+        const int lim = key_lim - kb, lo = key_lo - kb;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (hf * 32 + i >= lim) sa[i] = 0xff800000u;  // -inf
+          if (hf * 32 + i >= lim || hf * 32 + i < lo) sa[i] = 0xff800000u;  // -inf
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          if (64 + hf * 16 + i >= lim) sb[i] = 0xff800000u;
+          if (64 + hf * 16 + i >= lim || 64 + hf * 16 + i < lo) sb[i] = 0xff800000u;
+      }
+      if constexpr (SOFTCAP) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sa[i] = fwd_cap(p, sa[i]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sb[i] = fwd_cap(p, sb[i]);
       }
       float ch[8];
 #pragma unroll
@@ -906,7 +946,7 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SOFTCAP>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK,
@@ -958,9 +998,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int qt = grp / C::ROW_SPLIT;
     if (t.m_base + qt * C::BM < t.sq) {
       if constexpr (C::ROW_SPLIT == 2)
-        fwd_softmax_split<D, CAUSAL>(p, t, s, tmem, qt, grp % 2);
+        fwd_softmax_split<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt, grp % 2);
       else
-        fwd_softmax<D, CAUSAL>(p, t, s, tmem, qt);
+        fwd_softmax<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt);
     }
   } else if (warp == C::LOAD_WARP) {
     if (lane_id() == 0) fwd_load<D>(p, t, s, &tmQ, &tmK, &tmV);

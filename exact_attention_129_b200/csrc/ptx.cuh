@@ -382,6 +382,9 @@ __device__ __forceinline__ void fence_async_smem() {
 }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// a local-mask (window) bound that no key distance reaches: no bound
+constexpr int kNoBound = 1 << 29;
+
 // Debug builds only (-DATTN_TRACE): per-role SM-clock timestamps of the first
 // CTAs, written to a buffer set with attn_debug_set_trace.  The product build
 // compiles none of it.

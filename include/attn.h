@@ -107,6 +107,35 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v,
                        void* out, float* lse, attn_stream_t stream);
 
 /*
+ * Forward pass with a local (sliding-window) mask and a softcap (FA4
+ * repository guide, Public API: window_size_left/right and softcap are
+ * parameters of the varlen entry point; the page gives no formula, and this
+ * library takes the plainest reading):
+ *
+ *   window_left, window_right  with delta = s_k - s_q of the segment, key j is
+ *                  allowed for query row i iff j >= i + delta - window_left
+ *                  (when window_left >= 0) and j <= i + delta + window_right
+ *                  (when window_right >= 0); a negative bound means none.
+ *                  causal = 1 adds j <= i + delta as before.  Rows left with
+ *                  no allowed key get O = 0 and LSE = -inf.
+ *   softcap        0: none; > 0: every scaled score s = scale * q_i . k_j
+ *                  becomes softcap * tanh(s / softcap) before the softmax (the
+ *                  LSE is over the capped scores).  Negative or non-finite
+ *                  values return ATTN_ERR_INVALID_ARG.
+ *
+ * Every other argument is as for attn_fwd; attn_fwd is attn_fwd_ex with
+ * window_left = window_right = -1 and softcap = 0.
+ */
+attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v,
+                          const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                          int32_t batch, int32_t total_q, int32_t total_k,
+                          int32_t max_seqlen_q, int32_t max_seqlen_k,
+                          int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                          float scale, int32_t causal, int32_t window_left,
+                          int32_t window_right, float softcap, int32_t return_lse,
+                          void* out, float* lse, attn_stream_t stream);
+
+/*
  * Bytes of device workspace attn_bwd needs for these sizes (a pure function of
  * its arguments; 0 for invalid sizes).  The workspace holds the fp32 dQ
  * accumulator and the fp32 row-dot D_i = dO_i . O_i.
@@ -139,6 +168,25 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        float scale, int32_t causal,
                        void* dq, void* dk, void* dv,
                        void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * Backward pass with a local mask and a softcap: the gradient of attn_fwd_ex
+ * with the same window_left, window_right and softcap (which must match the
+ * forward call that produced out and lse).  With a softcap, dS carries the
+ * derivative of the cap, 1 - (s' / softcap)^2 at the capped score s'.  Every
+ * other argument is as for attn_bwd; attn_bwd is attn_bwd_ex with
+ * window_left = window_right = -1 and softcap = 0.
+ */
+attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const void* out,
+                          const float* lse, const void* dout,
+                          const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                          int32_t batch, int32_t total_q, int32_t total_k,
+                          int32_t max_seqlen_q, int32_t max_seqlen_k,
+                          int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                          float scale, int32_t causal, int32_t window_left,
+                          int32_t window_right, float softcap,
+                          void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
  * Backward pass that allocates nothing and takes no workspace.

@@ -66,6 +66,19 @@ def test_fwd_rejects_bad_arguments_without_launching(lib, bad, code):
     assert _fwd(lib, **bad) == code
 
 
+@pytest.mark.parametrize("cap", [-1.0, float("nan"), float("inf")])
+def test_fwd_ex_rejects_bad_softcap(lib, cap):
+    # validated on the host, before any device call
+    vp = ctypes.c_void_p
+    rc = lib.attn_fwd_ex(vp(16), vp(16), vp(16), vp(16), vp(16), 1, 128, 128, 128, 128, 4, 2,
+                         128, 0.088, 0, -1, -1, cap, 1, vp(16), vp(16), None)
+    assert rc == 1
+    rc = lib.attn_bwd_ex(vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), 1, 128,
+                         128, 128, 128, 4, 2, 128, 0.088, 0, -1, -1, cap, vp(16), vp(16),
+                         vp(16), vp(256), 1 << 30, None)
+    assert rc == 1
+
+
 def test_bwd_rejects_small_workspace(lib):
     vp = ctypes.c_void_p
     need = lib.attn_bwd_workspace_size(1, 128, 4, 128)

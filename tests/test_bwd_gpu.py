@@ -12,10 +12,10 @@ pytestmark = pytest.mark.gpu
 ea = pytest.importorskip("exact_attention_129_b200")
 
 
-def run_fwd_bwd(wl, guard=True):
+def run_fwd_bwd(wl, guard=True, window=None, softcap=0.0):
     host, (q, k, v, do), cu_q, cu_k = to_dev(wl)
     out, lse = ea.attn_fwd(q, k, v, cu_q, cu_k, wl.max_q, wl.max_k, scale=wl.scale,
-                           causal=wl.causal, return_lse=True)
+                           causal=wl.causal, window=window, softcap=softcap, return_lse=True)
     dev = q.device
     bufs = []
     grads = []
@@ -27,8 +27,8 @@ def run_fwd_bwd(wl, guard=True):
         else:
             grads.append(torch.empty_like(like))
     dq, dk, dv = ea.attn_bwd(q, k, v, out, lse, do, cu_q, cu_k, wl.max_q, wl.max_k,
-                             scale=wl.scale, causal=wl.causal, dq=grads[0], dk=grads[1],
-                             dv=grads[2])
+                             scale=wl.scale, causal=wl.causal, window=window, softcap=softcap,
+                             dq=grads[0], dk=grads[1], dv=grads[2])
     rc, msg = ea.last_device_error()
     assert rc == 0, msg
     for buf, g in bufs:
@@ -45,10 +45,11 @@ def rel_err(got, ref):
     return float(np.max(np.abs(got - ref))) / scale
 
 
-def check_full(wl):
-    host, _, grads = run_fwd_bwd(wl)
+def check_full(wl, window=None, softcap=0.0):
+    host, _, grads = run_fwd_bwd(wl, window=window, softcap=softcap)
     q, k, v, do = host
-    ref = oracle.bwd(q, k, v, do, wl.cu_q, wl.cu_k, wl.scale, wl.causal)
+    ref = oracle.bwd(q, k, v, do, wl.cu_q, wl.cu_k, wl.scale, wl.causal, window=window,
+                     softcap=softcap)
     for name, g, r in zip(("dQ", "dK", "dV"), grads, ref):
         gn = g.float().cpu().numpy()
         assert np.isfinite(gn).all(), f"{wl.name}: {name} not finite"
@@ -58,6 +59,27 @@ def check_full(wl):
 
 def test_tiny_config():
     check_full(si.tiny())
+
+
+WINDOWS = [(0, 0), (1, 0), (63, 64), (100, 37), (-1, 17), (200, -1), (130, 0)]
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_local_window(d, causal):
+    for wi, win in enumerate(WINDOWS):
+        wl = si.Workload(f"window{win}_d{d}", [300, 1, 515, 129], 4, 2, d, causal,
+                         lengths_k=[400, 1, 515, 64], seed=40 + wi)
+        check_full(wl, window=win)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("cap", [1.5, 30.0])
+def test_softcap(d, cap):
+    check_full(si.Workload(f"softcap{cap}_d{d}", [300, 129, 64], 4, 2, d, False, seed=51),
+               softcap=cap)
+    check_full(si.Workload(f"softcap{cap}_causal_d{d}", [515, 70], 4, 1, d, True, seed=52),
+               softcap=cap, window=(150, 0))
 
 
 RAGGED = [1, 127, 128, 129, 300, 0, 515, 64]

@@ -13,13 +13,14 @@ pytestmark = pytest.mark.gpu
 ea = pytest.importorskip("exact_attention_129_b200")
 
 
-def run_fwd(wl, return_lse=True, guard=True):
+def run_fwd(wl, return_lse=True, guard=True, window=None, softcap=0.0):
     host, (q, k, v, _), cu_q, cu_k = to_dev(wl, with_dout=False)
     dev = q.device
     obuf, out, og = guarded_empty(q.shape, torch.bfloat16, dev)
     lbuf, lse, lg = guarded_empty((wl.hq, wl.total_q), torch.float32, dev)
     ea.attn_fwd(q, k, v, cu_q, cu_k, wl.max_q, wl.max_k, scale=wl.scale, causal=wl.causal,
-                return_lse=return_lse, out=out, lse=lse if return_lse else None)
+                window=window, softcap=softcap, return_lse=return_lse, out=out,
+                lse=lse if return_lse else None)
     rc, msg = ea.last_device_error()
     assert rc == 0, msg
     assert guards_intact(obuf, og), "out guard band overwritten"
@@ -27,16 +28,25 @@ def run_fwd(wl, return_lse=True, guard=True):
     return host, out, lse
 
 
-def check_full(wl):
-    host, out, lse = run_fwd(wl)
+def few_key_o_tol(v):
+    """O bound when rows see only a few keys (the large-scores test derives it):
+    the bf16 rounding of P, the fp32-normaliser vs rounded-P mismatch and the bf16
+    rounding of O no longer average out, each reaching 2^-9 * max|v|."""
+    return max(O_TOL, 3 * 2.0 ** -9 * float(np.abs(np.asarray(v, np.float64)).max()))
+
+
+def check_full(wl, window=None, softcap=0.0, o_tol=None):
+    host, out, lse = run_fwd(wl, window=window, softcap=softcap)
     q, k, v, _ = host
-    ref_o, ref_lse = oracle.fwd(q, k, v, wl.cu_q, wl.cu_k, wl.scale, wl.causal)
+    ref_o, ref_lse = oracle.fwd(q, k, v, wl.cu_q, wl.cu_k, wl.scale, wl.causal, window=window,
+                                softcap=softcap)
     got_o = out.float().cpu().numpy()
     got_lse = lse.cpu().numpy()
     assert np.isfinite(got_o).all()
     eo = max_abs(got_o, ref_o)
     el = lse_err(got_lse, ref_lse)
-    assert eo <= O_TOL, f"{wl.name}: max |O err| {eo:.3e}"
+    tol = O_TOL if o_tol is None else o_tol
+    assert eo <= tol, f"{wl.name}: max |O err| {eo:.3e} (tol {tol:.3e})"
     assert el <= LSE_TOL, f"{wl.name}: max |LSE err| {el:.3e}"
     return eo, el
 
@@ -87,6 +97,33 @@ def test_epilogue_after_last_pv(d, monkeypatch):
         check_full(si.Workload(f"late_epilogue_d{d}", [1000, 257, 96], 4, 2, d, causal, seed=9))
 
 
+# local (sliding-window) masks: bounds below, at and above the block sizes,
+# one-sided windows, and segments with s_q != s_k
+WINDOWS = [(0, 0), (1, 0), (63, 64), (100, 37), (-1, 17), (200, -1), (130, 0)]
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_local_window(d, causal):
+    for wi, win in enumerate(WINDOWS):
+        wl = si.Workload(f"window{win}_d{d}", [300, 1, 515, 129], 4, 2, d, causal,
+                         lengths_k=[400, 1, 515, 64], seed=20 + wi)
+        # windows are outside the stated workloads, and every window (like the
+        # first rows under causal) leaves some rows with only a few keys: the
+        # bound for those rows applies
+        check_full(wl, window=win, o_tol=few_key_o_tol(wl.tensors(False)[2].float()))
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("cap", [1.5, 30.0])
+def test_softcap(d, cap):
+    check_full(si.Workload(f"softcap{cap}_d{d}", [300, 129, 64], 4, 2, d, False, seed=31),
+               softcap=cap)
+    wl = si.Workload(f"softcap{cap}_causal_d{d}", [515, 70], 4, 1, d, True, seed=32)
+    check_full(wl, softcap=cap, window=(150, 0),
+               o_tol=few_key_o_tol(wl.tensors(False)[2].float()))
+
+
 def test_deterministic():
     wl = si.Workload("det", [777, 1500], 4, 2, 128, True, seed=8)
     outs = [run_fwd(wl)[1:] for _ in range(3)]
@@ -105,7 +142,7 @@ def test_large_scores_stay_finite():
     # P no longer averages out: each of P's rounding, the mismatch between the
     # fp32 normaliser and the rounded P, and the bf16 rounding of O can reach
     # 2^-9 * max|v|.  Outside the stated workloads, so the bound is derived here.
-    tol = 3 * 2.0 ** -9 * float(host[2].float().abs().max())
+    tol = few_key_o_tol(host[2].float())
     assert max_abs(out.float().cpu().numpy(), ref_o) <= tol
     # |LSE| ~ 100 here: allow the same relative error as at |LSE| ~ 1
     assert lse_err(lse.cpu().numpy(), ref_l) <= LSE_TOL * max(1.0, np.abs(ref_l).max() / 10)
