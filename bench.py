@@ -41,12 +41,15 @@ METRIC = "attention fwd & fwd+bwd TFLOP/s (bf16) and % of B200 dense bf16 peak"
 WORKLOADS = {
     "varlen_gqa": lambda: si.varlen_gqa(),
     "gqa_16k": lambda: si.single_gqa(16384),
+    "gqa_16k_causal": lambda: si.single_gqa(16384, True),
     "gqa_64k": lambda: si.single_gqa(65536),
     "d64_mha": lambda: si.d64_mha(),
     "d256_mha_16k": lambda: si.d256_mha(16384, False),
     "d256_mha_16k_causal": lambda: si.d256_mha(16384, True),
     "d256_gqa8_128k": lambda: si.d256_gqa8(131072, False),
     "d256_gqa8_128k_causal": lambda: si.d256_gqa8(131072, True),
+    "gqa_16k_swa": lambda: si.gqa_sliding_window(16384, 4096),
+    "gqa_16k_softcap": lambda: si.gqa_softcap(16384, 50.0),
     "tiny": lambda: si.tiny(),
 }
 
@@ -182,27 +185,32 @@ def oracle_sample(wl: si.Workload, seconds: float):
     import oracle
     G = wl.hq // wl.hkv
     # calibrate the oracle's rate on a 256-token segment of this head group
-    cal = si.Workload("cal", [256], G, 1, wl.d, wl.causal, seed=wl.seed)
+    cal = si.Workload("cal", [256], G, 1, wl.d, wl.causal, seed=wl.seed, window=wl.window,
+                      softcap=wl.softcap)
     q, k, v, do = cal.tensors()
     t0 = time.perf_counter()
-    oracle.fwd(q, k, v, cal.cu_q, cal.cu_k, cal.scale, cal.causal)
-    oracle.bwd(q, k, v, do, cal.cu_q, cal.cu_k, cal.scale, cal.causal)
+    oracle.fwd(q, k, v, cal.cu_q, cal.cu_k, cal.scale, cal.causal, window=cal.window,
+               softcap=cal.softcap)
+    oracle.bwd(q, k, v, do, cal.cu_q, cal.cu_k, cal.scale, cal.causal, window=cal.window,
+               softcap=cal.softcap)
     rate = 3.5 * cal.fwd_flops() / max(time.perf_counter() - t0, 1e-6)
     lengths = []
     budget = seconds * rate
     for s in wl.lengths_q:
         trial = lengths + [s]
-        f = 3.5 * si.Workload("t", trial, G, 1, wl.d, wl.causal).fwd_flops()
+        f = 3.5 * si.Workload("t", trial, G, 1, wl.d, wl.causal, window=wl.window).fwd_flops()
         if lengths and f > budget:
             break
         lengths = trial
         if f > budget:
             break
-    if len(lengths) == 1 and 3.5 * si.Workload("t", lengths, G, 1, wl.d, wl.causal).fwd_flops() > 4 * budget:
+    if len(lengths) == 1 and 3.5 * si.Workload("t", lengths, G, 1, wl.d, wl.causal,
+                                                window=wl.window).fwd_flops() > 4 * budget:
         # one segment is far over budget: take a shorter prefix of it
         s = int(np.sqrt(budget / (3.5 * 4 * G * wl.d * (0.5 if wl.causal else 1.0))))
         lengths = [max(64, s)]
-    sample = si.Workload(f"{wl.name}_oracle_sample", lengths, G, 1, wl.d, wl.causal, seed=wl.seed)
+    sample = si.Workload(f"{wl.name}_oracle_sample", lengths, G, 1, wl.d, wl.causal, seed=wl.seed,
+                         window=wl.window, softcap=wl.softcap)
     desc = (f"{len(lengths)} segment(s) {lengths[:6]}{'...' if len(lengths) > 6 else ''} "
             f"of the workload, {G} query heads / 1 key-value head, head_dim {wl.d}, "
             f"{'causal' if wl.causal else 'non-causal'}: full oracle forward + backward")
@@ -213,8 +221,10 @@ def time_oracle(sample: si.Workload):
     import oracle
     q, k, v, do = sample.tensors()
     t0 = time.perf_counter()
-    oracle.fwd(q, k, v, sample.cu_q, sample.cu_k, sample.scale, sample.causal)
-    oracle.bwd(q, k, v, do, sample.cu_q, sample.cu_k, sample.scale, sample.causal)
+    oracle.fwd(q, k, v, sample.cu_q, sample.cu_k, sample.scale, sample.causal,
+               window=sample.window, softcap=sample.softcap)
+    oracle.bwd(q, k, v, do, sample.cu_q, sample.cu_k, sample.scale, sample.causal,
+               window=sample.window, softcap=sample.softcap)
     return time.perf_counter() - t0
 
 
@@ -256,6 +266,8 @@ def run_reference(args, wl, world, rank):
 def config_of(wl, l2):
     return {"workload": wl.name, "segments": len(wl.lengths_q), "total_tokens": wl.total_q,
             "nheads_q": wl.hq, "nheads_kv": wl.hkv, "head_dim": wl.d, "causal": wl.causal,
+            "window": list(wl.window) if wl.window is not None else None,
+            "softcap": wl.softcap or None,
             "softmax_scale": wl.scale, "l2": l2, "parallelism": "replicas"}
 
 
@@ -281,9 +293,10 @@ def run_ours(args, wl, world, rank, local):
 
     def step():
         ea.attn_fwd(q, k, v, cu_q, cu_k, wl.max_q, wl.max_k, scale=wl.scale, causal=wl.causal,
-                    return_lse=True, out=out, lse=lse)
+                    window=wl.window, softcap=wl.softcap, return_lse=True, out=out, lse=lse)
         ea.attn_bwd(q, k, v, out, lse, do, cu_q, cu_k, wl.max_q, wl.max_k, scale=wl.scale,
-                    causal=wl.causal, dq=dq, dk=dk, dv=dv, workspace=ws)
+                    causal=wl.causal, window=wl.window, softcap=wl.softcap, dq=dq, dk=dk, dv=dv,
+                    workspace=ws)
 
     for _ in range(args.warmup):
         step()

@@ -167,7 +167,7 @@ struct MaskArgs {
   int hi_off;
   int lo_off;    // kNoBound: none
   bool softcap;
-  float cap_k;   // scale / c
+  float cap_k2;    // 2 log2(e) scale / c
   float cap_log2;  // c * log2(e)
 };
 
@@ -182,7 +182,7 @@ attn_status_t mask_args(int32_t causal, int32_t window_left, int32_t window_righ
   m->hi_off = causal ? (wr >= 0 ? std::min(wr, 0) : 0) : (wr >= 0 ? wr : kNoBound);
   m->lo_off = wl >= 0 ? wl : kNoBound;
   m->softcap = softcap > 0.f;
-  m->cap_k = m->softcap ? scale / softcap : 0.f;
+  m->cap_k2 = m->softcap ? 2.f * 1.4426950408889634f * scale / softcap : 0.f;
   m->cap_log2 = m->softcap ? softcap * 1.4426950408889634f : 0.f;
   return ATTN_OK;
 }
@@ -278,7 +278,7 @@ attn_status_t bwd_launch_d(const BwdArgs& a, cudaStream_t stream) {
   bp.scale_log2 = a.scale * 1.4426950408889634f;
   bp.hi_off = a.hi_off;
   bp.lo_off = a.lo_off;
-  bp.cap_k = a.cap_k;
+  bp.cap_k2 = a.cap_k2;
   bp.cap_log2 = a.cap_log2;
   bp.timeout_ns = a.timeout_ns;
   if (a.total_k > 0) {
@@ -351,7 +351,7 @@ extern "C" attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v
   p.return_lse = return_lse ? 1 : 0;
   p.hi_off = mk.hi_off;
   p.lo_off = mk.lo_off;
-  p.cap_k = mk.cap_k;
+  p.cap_k2 = mk.cap_k2;
   p.cap_log2 = mk.cap_log2;
   p.timeout_ns = wait_timeout_ns();
   p.epilogue_delay_ns = test_epilogue_delay_ns();
@@ -441,7 +441,7 @@ extern "C" attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v
   a.hq = nheads_q; a.hkv = nheads_kv; a.d = head_dim;
   a.scale = scale;
   a.upper = mk.upper; a.hi_off = mk.hi_off; a.lo_off = mk.lo_off;
-  a.softcap = mk.softcap; a.cap_k = mk.cap_k; a.cap_log2 = mk.cap_log2;
+  a.softcap = mk.softcap; a.cap_k2 = mk.cap_k2; a.cap_log2 = mk.cap_log2;
   a.dq = dq; a.dk = dk; a.dv = dv; a.workspace = workspace;
   a.err = ds->err;
   a.timeout_ns = wait_timeout_ns();

@@ -54,7 +54,7 @@ struct BwdArgs {
   bool upper;              // rows have an upper key bound (causal or a right window)
   int hi_off, lo_off;      // window offsets, as in BwdParams
   bool softcap;
-  float cap_k, cap_log2;
+  float cap_k2, cap_log2;
   void *dq, *dk, *dv, *workspace;
   uint32_t* err;
   uint64_t timeout_ns;
@@ -87,8 +87,9 @@ struct BwdParams {
   // bound exists iff the kernel's CAUSAL parameter is set)
   int hi_off;
   int lo_off;
-  // softcap c: scores c tanh(s / c); cap_k = scale / c, cap_log2 = c log2(e)
-  float cap_k;
+  // softcap c: scores c tanh(s scale / c); cap_k2 = 2 log2(e) scale / c,
+  // cap_log2 = c log2(e)
+  float cap_k2;
   float cap_log2;
   uint64_t timeout_ns;
 };
@@ -612,8 +613,8 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
         float e0, e1;
         float g0 = 1.f, g1 = 1.f;  // d(capped score) / d(scaled score)
         if constexpr (SOFTCAP) {
-          const float t0 = tanhf(__uint_as_float(sr[x]) * p.cap_k);
-          const float t1 = tanhf(__uint_as_float(sr[x + 1]) * p.cap_k);
+          const float t0 = tanh_from_ex2(__uint_as_float(sr[x]) * p.cap_k2);
+          const float t1 = tanh_from_ex2(__uint_as_float(sr[x + 1]) * p.cap_k2);
           e0 = p.cap_log2 * t0 - (hp ? l4.z : l4.x);
           e1 = p.cap_log2 * t1 - (hp ? l4.w : l4.y);
           g0 = 1.f - t0 * t0;

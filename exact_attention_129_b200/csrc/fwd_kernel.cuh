@@ -73,8 +73,9 @@ struct FwdParams {
   //   upper bound exists iff the kernel's CAUSAL parameter is set)
   int hi_off;
   int lo_off;
-  // softcap c: scores become c tanh(s / c); cap_k = scale / c, cap_log2 = c log2(e)
-  float cap_k;
+  // softcap c: scores become c tanh(s scale / c); cap_k2 = 2 log2(e) scale / c,
+  // cap_log2 = c log2(e)
+  float cap_k2;
   float cap_log2;
   uint64_t timeout_ns;
   // test hook (0 in normal use): the softmax warps idle this long before their
@@ -83,10 +84,10 @@ struct FwdParams {
 };
 
 // softcap of one score (fp32 bits): c tanh(s scale / c) in the log2 domain,
-// i.e. c log2(e) tanh(s cap_k); masked scores (-inf) stay -inf
+// i.e. c log2(e) tanh(s scale / c); masked scores (-inf) stay -inf
 __device__ __forceinline__ uint32_t fwd_cap(const FwdParams& p, uint32_t bits) {
   const float x = __uint_as_float(bits);
-  return x == -INFINITY ? bits : __float_as_uint(p.cap_log2 * tanhf(x * p.cap_k));
+  return x == -INFINITY ? bits : __float_as_uint(p.cap_log2 * tanh_from_ex2(x * p.cap_k2));
 }
 
 __device__ __forceinline__ void fwd_test_delay(const FwdParams& p) {

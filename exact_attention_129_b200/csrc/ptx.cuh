@@ -364,6 +364,17 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// tanh(x) from the identity tanh(x) = 1 - 2 / (e^(2x) + 1), with e^(2x) taken as
+// 2^(x * k2) where k2 = 2 log2(e) (folded into the caller's scale): one ex2 and
+// one reciprocal.  Absolute error ~1e-7; +-inf and large |x| give +-1.
+__device__ __forceinline__ float tanh_from_ex2(float x_times_k2) {
+  return 1.f - 2.f * rcp_approx(ex2(x_times_k2) + 1.f);
+}
 // two floats -> packed bf16x2, `lo` in the low half (round to nearest even)
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;

@@ -75,6 +75,8 @@ class Workload:
     causal: bool
     lengths_k: list = field(default=None)
     seed: int = 0
+    window: tuple = None      # (left, right) key-distance bounds; None = no window
+    softcap: float = 0.0      # > 0: scores capped at softcap * tanh(s / softcap)
 
     def __post_init__(self):
         if self.lengths_k is None:
@@ -113,9 +115,25 @@ class Workload:
                             self.seed, with_dout)
 
     def fwd_flops(self) -> float:
-        """Forward FLOPs: 4 * s_q * s_k * Hq * D per segment, halved when causal."""
-        f = sum(4.0 * a * b * self.hq * self.d for a, b in zip(self.lengths_q, self.lengths_k))
-        return f / 2 if self.causal else f
+        """Forward FLOPs: 4 * s_q * s_k * Hq * D per segment, halved when causal
+        (the pages' convention).  With a local window: 4 * Hq * D per allowed
+        (row, key) pair, counted exactly."""
+        if self.window is None or (self.window[0] < 0 and self.window[1] < 0):
+            f = sum(4.0 * a * b * self.hq * self.d
+                    for a, b in zip(self.lengths_q, self.lengths_k))
+            return f / 2 if self.causal else f
+        left, right = self.window
+        pairs = 0
+        for sq, sk in zip(self.lengths_q, self.lengths_k):
+            diag = np.arange(sq, dtype=np.int64) + (sk - sq)
+            hi = np.full(sq, sk - 1, np.int64)
+            if self.causal:
+                hi = np.minimum(hi, diag)
+            if right >= 0:
+                hi = np.minimum(hi, diag + right)
+            lo = np.zeros(sq, np.int64) if left < 0 else np.maximum(0, diag - left)
+            pairs += int(np.maximum(0, hi - lo + 1).sum())
+        return 4.0 * pairs * self.hq * self.d
 
 
 # The five problem families of the pages, by name.
@@ -131,6 +149,19 @@ def varlen_gqa(total: int = 16384, seed: int = 0) -> Workload:
 def single_gqa(seqlen: int, causal: bool = False) -> Workload:
     return Workload(f"gqa_s{seqlen}_hq32_hkv8_d128{'_causal' if causal else ''}",
                     [seqlen], 32, 8, 128, causal)
+
+
+def gqa_sliding_window(seqlen: int = 16384, window: int = 4096) -> Workload:
+    """The GQA head_dim-128 family with a causal sliding window of `window` keys
+    (each row sees itself and the window - 1 keys before it)."""
+    return Workload(f"gqa_s{seqlen}_hq32_hkv8_d128_causal_window{window}", [seqlen], 32, 8,
+                    128, True, window=(window - 1, 0))
+
+
+def gqa_softcap(seqlen: int = 16384, cap: float = 50.0) -> Workload:
+    """The GQA head_dim-128 family, causal, with the scores soft-capped."""
+    return Workload(f"gqa_s{seqlen}_hq32_hkv8_d128_causal_softcap{cap:g}", [seqlen], 32, 8, 128,
+                    True, softcap=cap)
 
 
 def d64_mha() -> Workload:
