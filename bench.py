@@ -49,6 +49,7 @@ WORKLOADS = {
     "d256_gqa8_128k": lambda: si.d256_gqa8(131072, False),
     "d256_gqa8_128k_causal": lambda: si.d256_gqa8(131072, True),
     "gqa_16k_swa": lambda: si.gqa_sliding_window(16384, 4096),
+    "decode_64x64k": lambda: si.decode_gqa(64, 65536),
     "gqa_16k_softcap": lambda: si.gqa_softcap(16384, 50.0),
     "tiny": lambda: si.tiny(),
 }
@@ -263,8 +264,9 @@ def run_reference(args, wl, world, rank):
     }
 
 
-def config_of(wl, l2):
+def config_of(wl, l2, num_splits=1):
     return {"workload": wl.name, "segments": len(wl.lengths_q), "total_tokens": wl.total_q,
+            "total_keys": wl.total_k, "num_splits": num_splits,
             "nheads_q": wl.hq, "nheads_kv": wl.hkv, "head_dim": wl.d, "causal": wl.causal,
             "window": list(wl.window) if wl.window is not None else None,
             "softcap": wl.softcap or None,
@@ -288,12 +290,17 @@ def run_ours(args, wl, world, rank, local):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(ea.bwd_workspace_size(len(wl.lengths_q), wl.total_q, wl.hq, wl.d),
                      device=dev, dtype=torch.uint8)
+    fws = None
+    if args.num_splits > 1:
+        fws = torch.empty(ea.fwd_split_workspace_size(wl.total_q, wl.hq, wl.d, args.num_splits),
+                          device=dev, dtype=torch.uint8)
     flush = torch.empty(L2_FLUSH_BYTES, device=dev, dtype=torch.uint8)
     F = wl.fwd_flops()
 
     def step():
         ea.attn_fwd(q, k, v, cu_q, cu_k, wl.max_q, wl.max_k, scale=wl.scale, causal=wl.causal,
-                    window=wl.window, softcap=wl.softcap, return_lse=True, out=out, lse=lse)
+                    window=wl.window, softcap=wl.softcap, return_lse=True, out=out, lse=lse,
+                    num_splits=args.num_splits, workspace=fws)
         ea.attn_bwd(q, k, v, out, lse, do, cu_q, cu_k, wl.max_q, wl.max_k, scale=wl.scale,
                     causal=wl.causal, window=wl.window, softcap=wl.softcap, dq=dq, dk=dk, dv=dv,
                     workspace=ws)
@@ -394,7 +401,7 @@ def run_ours(args, wl, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16; varlen lengths seeded uniform)",
-        "config": config_of(wl, "flushed between steps (512 MiB write)"),
+        "config": config_of(wl, "flushed between steps (512 MiB write)", args.num_splits),
         "fwd_tflops": F / (fwd_ms * 1e-3) / 1e12,
         "fwd_ms": fwd_ms, "bwd_main_ms": bwd_main_ms,
         "pct_of_2250": {"fwd": 100 * F / (fwd_ms * 1e-3) / 1e12 / PAGE_PEAK_TFLOPS,
@@ -419,6 +426,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="varlen_gqa")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--num-splits", type=int, default=1,
+                    help="SplitKV parts of the forward (1: plain forward)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

@@ -21,14 +21,16 @@ import os
 
 import torch
 
-__all__ = ["attn_fwd", "attn_bwd", "attention", "bwd_workspace_size", "last_device_error",
+__all__ = ["attn_fwd", "attn_bwd", "attention", "bwd_workspace_size", "fwd_split_workspace_size",
+           "last_device_error",
            "set_timing_events", "KERNEL_FWD", "KERNEL_BWD_MAIN",
            "library", "LIB_PATH", "AttnError", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED",
           3: "ATTN_ERR_CUDA", 4: "ATTN_ERR_TIMEOUT", 5: "ATTN_ERR_SCRATCH_TOO_SMALL"}
-EXPORTED = ("attn_fwd", "attn_bwd", "attn_fwd_ex", "attn_bwd_ex", "attn_bwd_workspace_size",
+EXPORTED = ("attn_fwd", "attn_bwd", "attn_fwd_ex", "attn_bwd_ex", "attn_fwd_split",
+            "attn_fwd_split_workspace_size", "attn_bwd_workspace_size",
             "attn_last_device_error", "attn_set_timing_events", "attn_bwd_static_scratch",
             "attn_watchdog_selftest", "attn_version")
 KERNEL_FWD, KERNEL_BWD_MAIN = 0, 1
@@ -65,6 +67,12 @@ def library() -> ctypes.CDLL:
                                     i32, i32, i32, f32, i32, i32, i32, f32, vp, vp, vp, vp,
                                     ctypes.c_size_t, vp]
         lib.attn_bwd_ex.restype = ctypes.c_int
+        lib.attn_fwd_split.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                       i32, f32, i32, i32, i32, f32, i32, i32, vp, vp, vp,
+                                       ctypes.c_size_t, vp]
+        lib.attn_fwd_split.restype = ctypes.c_int
+        lib.attn_fwd_split_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.attn_fwd_split_workspace_size.restype = ctypes.c_size_t
         lib.attn_bwd_workspace_size.argtypes = [i32, i32, i32, i32]
         lib.attn_bwd_workspace_size.restype = ctypes.c_size_t
         lib.attn_last_device_error.argtypes = [vp, ctypes.c_char_p, ctypes.c_size_t]
@@ -110,14 +118,20 @@ def _window(window):
     return (-1 if left is None else int(left)), (-1 if right is None else int(right))
 
 
+def fwd_split_workspace_size(total_q, nheads_q, head_dim, num_splits) -> int:
+    return int(library().attn_fwd_split_workspace_size(total_q, nheads_q, head_dim, num_splits))
+
+
 def attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
              scale=None, causal=False, window=None, softcap=0.0, return_lse=True, out=None,
-             lse=None):
+             lse=None, num_splits=1, workspace=None):
     """Forward pass. q [Tq,Hq,D], k/v [Tk,Hkv,D] bf16; returns (out, lse or None).
 
     ``window`` = (left, right): with delta = s_k - s_q, row i sees keys
     [i + delta - left, i + delta + right]; None or a negative side = no bound.
-    ``softcap`` > 0 caps each scaled score at softcap * tanh(s / softcap)."""
+    ``softcap`` > 0 caps each scaled score at softcap * tanh(s / softcap).
+    ``num_splits`` > 1 runs the SplitKV forward (key range of every query tile
+    cut into that many parts, merged by LSE) in ``workspace`` (allocated if None)."""
     _check_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k, out, lse)
     for n, t in (("q", q), ("k", k), ("v", v)):
         _check_layout(n, t, torch.bfloat16)
@@ -132,6 +146,20 @@ def attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
     if return_lse and lse is None:
         lse = torch.empty((hq, tq), device=q.device, dtype=torch.float32)
     wl, wr = _window(window)
+    if int(num_splits) > 1:
+        need = fwd_split_workspace_size(tq, hq, d, int(num_splits))
+        if workspace is None:
+            workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
+        _check_cuda(workspace)
+        rc = library().attn_fwd_split(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+            cu_seqlens_q.numel() - 1, tq, tk, int(max_seqlen_q), int(max_seqlen_k), hq, hkv, d,
+            float(scale), int(bool(causal)), wl, wr, float(softcap or 0.0), int(num_splits),
+            int(bool(return_lse)), _ptr(out), _ptr(lse) if return_lse else None,
+            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(q.device))
+        if rc != 0:
+            raise AttnError("attn_fwd_split", rc)
+        return out, (lse if return_lse else None)
     rc = library().attn_fwd_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
         cu_seqlens_q.numel() - 1, tq, tk, int(max_seqlen_q), int(max_seqlen_k), hq, hkv, d,

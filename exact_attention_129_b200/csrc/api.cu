@@ -315,14 +315,23 @@ attn_status_t bwd_launch(const BwdArgs& a, cudaStream_t stream) {
 
 using namespace attn;
 
-extern "C" attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v,
-                                     const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
-                                     int32_t batch, int32_t total_q, int32_t total_k,
-                                     int32_t max_seqlen_q, int32_t max_seqlen_k,
-                                     int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
-                                     float scale, int32_t causal, int32_t window_left,
-                                     int32_t window_right, float softcap, int32_t return_lse,
-                                     void* out, float* lse, attn_stream_t stream) {
+namespace {
+constexpr int kMaxSplits = 128;
+
+size_t fwd_split_workspace_bytes(int32_t total_q, int32_t nheads_q, int32_t head_dim,
+                                 int32_t num_splits) {
+  const size_t rows = static_cast<size_t>(num_splits) * (total_q > 0 ? total_q : 1) * nheads_q;
+  return bwd_align256(rows * head_dim * 4) + bwd_align256(rows * 4);
+}
+
+// the forward with num_splits SplitKV parts (1: plain) and its combine
+attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                       const int32_t* cu_seqlens_k, int32_t batch, int32_t total_q,
+                       int32_t total_k, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                       int32_t nheads_q, int32_t nheads_kv, int32_t head_dim, float scale,
+                       int32_t causal, int32_t window_left, int32_t window_right, float softcap,
+                       int32_t num_splits, int32_t return_lse, void* out, float* lse,
+                       void* workspace, size_t workspace_bytes, attn_stream_t stream) {
   attn_status_t st = check_common(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
                                   max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim,
                                   scale);
@@ -332,6 +341,13 @@ extern "C" attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v
   if (st != ATTN_OK) return st;
   if (!out || !aligned16(out)) return ATTN_ERR_INVALID_ARG;
   if (return_lse && (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u))) return ATTN_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > kMaxSplits ||
+      static_cast<int64_t>(batch) * num_splits > 65535)
+    return ATTN_ERR_INVALID_ARG;
+  if (num_splits > 1 &&
+      (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+       workspace_bytes < fwd_split_workspace_bytes(total_q, nheads_q, head_dim, num_splits)))
+    return ATTN_ERR_INVALID_ARG;
   int dev = 0;
   DeviceState* ds = device_state(&dev);
   if (!ds) return ATTN_ERR_CUDA;
@@ -353,12 +369,43 @@ extern "C" attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v
   p.lo_off = mk.lo_off;
   p.cap_k2 = mk.cap_k2;
   p.cap_log2 = mk.cap_log2;
+  p.num_splits = num_splits;
+  p.o_part = nullptr;
+  p.lse_part = nullptr;
+  if (num_splits > 1) {
+    p.o_part = static_cast<float*>(workspace);
+    p.lse_part = reinterpret_cast<float*>(
+        static_cast<uint8_t*>(workspace) +
+        bwd_align256(static_cast<size_t>(num_splits) * total_q * nheads_q * head_dim * 4));
+  }
   p.timeout_ns = wait_timeout_ns();
   p.epilogue_delay_ns = test_epilogue_delay_ns();
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int grid_z = batch * num_splits;
   auto run = [&](auto launch) {
-    return launch(q, k, v, total_q, total_k, nheads_kv, p, batch, nheads_q, max_seqlen_q, s);
+    attn_status_t r =
+        launch(q, k, v, total_q, total_k, nheads_kv, p, grid_z, nheads_q, max_seqlen_q, s);
+    if (r != ATTN_OK || num_splits == 1) return r;
+    const long long warps = static_cast<long long>(total_q) * nheads_q;
+    const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+    switch (head_dim) {
+      case 64:
+        attn_fwd_combine_kernel<64><<<blocks, 256, 0, s>>>(
+            p.o_part, p.lse_part, static_cast<uint16_t*>(out), lse, total_q, nheads_q,
+            num_splits, return_lse);
+        break;
+      case 128:
+        attn_fwd_combine_kernel<128><<<blocks, 256, 0, s>>>(
+            p.o_part, p.lse_part, static_cast<uint16_t*>(out), lse, total_q, nheads_q,
+            num_splits, return_lse);
+        break;
+      default:
+        attn_fwd_combine_kernel<256><<<blocks, 256, 0, s>>>(
+            p.o_part, p.lse_part, static_cast<uint16_t*>(out), lse, total_q, nheads_q,
+            num_splits, return_lse);
+    }
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
   };
   // the kernel's CAUSAL parameter means "rows have an upper key bound"
   const int variant = (mk.upper ? 1 : 0) | (mk.softcap ? 2 : 0);
@@ -385,6 +432,44 @@ extern "C" attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v
         default: return run(launch_fwd<256, true, true>);
       }
   }
+}
+
+}  // namespace
+
+extern "C" attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v,
+                                     const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                     int32_t batch, int32_t total_q, int32_t total_k,
+                                     int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                     int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                                     float scale, int32_t causal, int32_t window_left,
+                                     int32_t window_right, float softcap, int32_t return_lse,
+                                     void* out, float* lse, attn_stream_t stream) {
+  return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, nheads_q, nheads_kv, head_dim, scale, causal, window_left,
+                  window_right, softcap, 1, return_lse, out, lse, nullptr, 0, stream);
+}
+
+extern "C" size_t attn_fwd_split_workspace_size(int32_t total_q, int32_t nheads_q,
+                                                int32_t head_dim, int32_t num_splits) {
+  if (total_q < 0 || nheads_q < 1 || head_dim < 1 || num_splits < 1 || num_splits > kMaxSplits)
+    return 0;
+  return fwd_split_workspace_bytes(total_q, nheads_q, head_dim, num_splits);
+}
+
+extern "C" attn_status_t attn_fwd_split(const void* q, const void* k, const void* v,
+                                        const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                        int32_t batch, int32_t total_q, int32_t total_k,
+                                        int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                        int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                                        float scale, int32_t causal, int32_t window_left,
+                                        int32_t window_right, float softcap, int32_t num_splits,
+                                        int32_t return_lse, void* out, float* lse,
+                                        void* workspace, size_t workspace_bytes,
+                                        attn_stream_t stream) {
+  return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, nheads_q, nheads_kv, head_dim, scale, causal, window_left,
+                  window_right, softcap, num_splits, return_lse, out, lse, workspace,
+                  workspace_bytes, stream);
 }
 
 extern "C" attn_status_t attn_fwd(const void* q, const void* k, const void* v,

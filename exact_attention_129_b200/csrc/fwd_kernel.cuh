@@ -77,6 +77,12 @@ struct FwdParams {
   // cap_log2 = c log2(e)
   float cap_k2;
   float cap_log2;
+  // SplitKV: num_splits > 1 splits every CTA's key-block range into that many
+  // contiguous parts (grid.z = batch * num_splits); each part writes its own
+  // normalised O and LSE to o_part / lse_part for the combine kernel
+  int num_splits;
+  float* o_part;    // fp32 [num_splits][total_q][nheads_q][D]
+  float* lse_part;  // fp32 [num_splits][nheads_q][total_q]
   uint64_t timeout_ns;
   // test hook (0 in normal use): the softmax warps idle this long before their
   // final wait, so the tile's last P.V is sure to have completed by then
@@ -193,12 +199,35 @@ struct FwdTile {
   int n_lo;             // first key block to visit
   int n_blocks;         // key blocks to visit: [n_lo, n_lo + n_blocks)
   int h, hk;
+  int split;            // SplitKV part of this CTA (0 without SplitKV)
 };
+
+// SplitKV: 32 columns (from col0) of a row's normalised O into the fp32 partial
+// buffer of this CTA's split, and the row's partial LSE
+template <int D>
+__device__ __forceinline__ void fwd_store_part(const FwdParams& p, const FwdTile& t, int row,
+                                               int col0, const uint32_t (&r)[32], float inv_l) {
+  if (row >= t.sq) return;
+  float* dst = p.o_part +
+               ((static_cast<size_t>(t.split) * p.total_q + t.q0 + row) * p.nheads_q + t.h) * D +
+               col0;
+#pragma unroll
+  for (int g = 0; g < 8; ++g)
+    reinterpret_cast<float4*>(dst)[g] =
+        make_float4(__uint_as_float(r[4 * g]) * inv_l, __uint_as_float(r[4 * g + 1]) * inv_l,
+                    __uint_as_float(r[4 * g + 2]) * inv_l, __uint_as_float(r[4 * g + 3]) * inv_l);
+}
+__device__ __forceinline__ void fwd_store_part_lse(const FwdParams& p, const FwdTile& t, int row,
+                                                   float lse) {
+  if (row < t.sq)
+    p.lse_part[(static_cast<size_t>(t.split) * p.nheads_q + t.h) * p.total_q + t.q0 + row] = lse;
+}
 
 template <int D, bool CAUSAL>
 __device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t) {
   using C = FwdCfg<D>;
-  const int b = blockIdx.z;
+  const int b = blockIdx.z / p.num_splits;
+  t.split = blockIdx.z % p.num_splits;
   t.h = blockIdx.y;
   t.hk = t.h / (p.nheads_q / p.nheads_kv);
   t.q0 = p.cu_q[b];
@@ -219,6 +248,14 @@ __device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t) {
   const int n_beg = (p.lo_off < kNoBound) ? max(0, t.m_base + delta - p.lo_off) : 0;
   t.n_lo = n_beg / C::BN;
   t.n_blocks = n_end > n_beg ? (n_end + C::BN - 1) / C::BN - t.n_lo : 0;
+  if (p.num_splits > 1) {
+    // this CTA's contiguous share; a share past the end has no blocks and
+    // writes O = 0, LSE = -inf for the combine
+    const int per = (t.n_blocks + p.num_splits - 1) / p.num_splits;
+    const int first = t.split * per;
+    t.n_lo += first;
+    t.n_blocks = max(0, min(per, t.n_blocks - first));
+  }
   return true;
 }
 
@@ -697,6 +734,10 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
 #pragma unroll
         for (int i = 0; i < 32; ++i) r[i] = 0u;
       }
+      if (p.num_splits > 1) {  // SplitKV: fp32 partial, straight from registers
+        fwd_store_part<D>(p, t, row, cc * 32, r, inv_l);
+        continue;
+      }
 #pragma unroll
       for (int g = 0; g < 4; ++g) {  // 4 chunks of 8 columns
         uint4 v;
@@ -711,7 +752,11 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     }
   }
   named_bar_sync(1 + qt, 128);
-  if (ok) {
+  if (ok && p.num_splits > 1) {
+    fwd_store_part_lse(p, t, row,
+                       (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f
+                                     : -INFINITY);
+  } else if (ok) {
     const int rows_left = t.sq - tile_row0;
     uint8_t* out = static_cast<uint8_t*>(p.out);
     const int tid = threadIdx.x & 127;
@@ -911,6 +956,10 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
 #pragma unroll
         for (int i = 0; i < 32; ++i) r[i] = 0u;
       }
+      if (p.num_splits > 1) {  // SplitKV: fp32 partial, straight from registers
+        fwd_store_part<D>(p, t, row, hf * OC + cc * 32, r, inv_l);
+        continue;
+      }
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         uint4 v;
@@ -925,7 +974,12 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
     }
   }
   named_bar_sync(1 + qt, 256);  // both halves of the tile
-  if (ok) {
+  if (ok && p.num_splits > 1) {
+    if (hf == 0)
+      fwd_store_part_lse(p, t, row,
+                         (l_tot > 0.f) ? (m_run + __log2f(l_tot)) * 0.69314718055994530942f
+                                       : -INFINITY);
+  } else if (ok) {
     const int rows_left = t.sq - tile_row0;
     uint8_t* out = static_cast<uint8_t*>(p.out);
     const int tid = hf * 128 + row_in_tile;
@@ -1016,6 +1070,59 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// ---------------------------------------------------------------------------
+// SplitKV combine (the FA4 repository guide, Forward Kernels: a combine kernel
+// merges the SplitKV partial results).  Split s of a row holds O_s (normalised
+// over its own keys) and LSE_s; over all splits LSE = log sum_s exp(LSE_s) and
+// O = sum_s exp(LSE_s - LSE) O_s.  One warp per (row, head); a row whose
+// splits all saw no key gets O = 0 and LSE = -inf.  HBM-bound.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+    attn_fwd_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                            uint16_t* __restrict__ out, float* __restrict__ lse, int total_q,
+                            int nheads_q, int num_splits, int return_lse) {
+  constexpr int VPL = D / 32;  // columns per lane: 2, 4 or 8
+  const long long w = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<long long>(total_q) * nheads_q) return;  // whole warps leave together
+  const int row = static_cast<int>(w / nheads_q), h = static_cast<int>(w % nheads_q);
+  auto lse_of = [&](int sp) {
+    return lse_part[(static_cast<size_t>(sp) * nheads_q + h) * total_q + row];
+  };
+  float m = -INFINITY;
+  for (int sp = lane; sp < num_splits; sp += 32) m = fmaxf(m, lse_of(sp));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+  float sum = 0.f;
+  if (m != -INFINITY) {
+    for (int sp = 0; sp < num_splits; ++sp) {
+      const float l = lse_of(sp);
+      if (l == -INFINITY) continue;
+      const float wgt = expf(l - m);
+      sum += wgt;
+      const float* src =
+          o_part + ((static_cast<size_t>(sp) * total_q + row) * nheads_q + h) * D + lane * VPL;
+#pragma unroll
+      for (int i = 0; i < VPL; i += 2) {
+        const float2 v = *reinterpret_cast<const float2*>(src + i);
+        acc[i] += wgt * v.x;
+        acc[i + 1] += wgt * v.y;
+      }
+    }
+  }
+  const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
+  uint32_t* dst = reinterpret_cast<uint32_t*>(
+      out + (static_cast<size_t>(row) * nheads_q + h) * D + lane * VPL);
+#pragma unroll
+  for (int i = 0; i < VPL; i += 2) dst[i / 2] = pack_bf16(acc[i] * inv, acc[i + 1] * inv);
+  if (return_lse && lane == 0)
+    lse[static_cast<size_t>(h) * total_q + row] = (sum > 0.f) ? m + logf(sum) : -INFINITY;
 }
 
 }  // namespace attn

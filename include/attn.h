@@ -136,6 +136,42 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v,
                           void* out, float* lse, attn_stream_t stream);
 
 /*
+ * SplitKV forward (FA4 repository guide, Forward Kernels: the Blackwell forward
+ * supports SplitKV, and a combine kernel merges the SplitKV partial results).
+ * For short query segments against long key segments (decode-like shapes) the
+ * plain grid has too few CTAs; here every CTA's range of key blocks is cut into
+ * num_splits contiguous parts, each run by its own CTA, which writes its part's
+ * O (normalised over its own keys) and LSE to the workspace; a second kernel
+ * merges them: LSE = log sum_s exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s.
+ *
+ *   num_splits     1..128; batch * num_splits <= 65535.  1 computes exactly
+ *                  what attn_fwd_ex computes (and needs no workspace).
+ *   workspace      device memory of at least attn_fwd_split_workspace_size(...)
+ *                  bytes, 256-byte aligned (may be NULL when num_splits == 1);
+ *                  clobbered.  Calls sharing a workspace must not overlap on
+ *                  the GPU.
+ * Every other argument is as for attn_fwd_ex.  The result equals the
+ * unsplit one up to fp32 rounding of the merge (O is still rounded to bf16
+ * once, at the end).
+ */
+attn_status_t attn_fwd_split(const void* q, const void* k, const void* v,
+                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                             int32_t batch, int32_t total_q, int32_t total_k,
+                             int32_t max_seqlen_q, int32_t max_seqlen_k,
+                             int32_t nheads_q, int32_t nheads_kv, int32_t head_dim,
+                             float scale, int32_t causal, int32_t window_left,
+                             int32_t window_right, float softcap, int32_t num_splits,
+                             int32_t return_lse, void* out, float* lse, void* workspace,
+                             size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * Bytes of device workspace attn_fwd_split needs (fp32 partial O and LSE of
+ * every split; 0 for invalid sizes).
+ */
+size_t attn_fwd_split_workspace_size(int32_t total_q, int32_t nheads_q, int32_t head_dim,
+                                     int32_t num_splits);
+
+/*
  * Bytes of device workspace attn_bwd needs for these sizes (a pure function of
  * its arguments; 0 for invalid sizes).  The workspace holds the fp32 dQ
  * accumulator and the fp32 row-dot D_i = dO_i . O_i.

@@ -116,13 +116,17 @@ class Workload:
 
     def fwd_flops(self) -> float:
         """Forward FLOPs: 4 * s_q * s_k * Hq * D per segment, halved when causal
-        (the pages' convention).  With a local window: 4 * Hq * D per allowed
-        (row, key) pair, counted exactly."""
-        if self.window is None or (self.window[0] < 0 and self.window[1] < 0):
+        (the pages' convention, for s_q = s_k).  With a local window, or causal
+        with s_q != s_k: 4 * Hq * D per allowed (row, key) pair, counted exactly."""
+        square = all(a == b for a, b in zip(self.lengths_q, self.lengths_k))
+        no_window = self.window is None or (self.window[0] < 0 and self.window[1] < 0)
+        if no_window and (square or not self.causal):
             f = sum(4.0 * a * b * self.hq * self.d
                     for a, b in zip(self.lengths_q, self.lengths_k))
             return f / 2 if self.causal else f
-        left, right = self.window
+        # windows, and causal segments with s_q != s_k (where halving does not
+        # describe the mask): count the allowed (row, key) pairs
+        left, right = self.window if not no_window else (-1, -1)
         pairs = 0
         for sq, sk in zip(self.lengths_q, self.lengths_k):
             diag = np.arange(sq, dtype=np.int64) + (sk - sq)
@@ -156,6 +160,13 @@ def gqa_sliding_window(seqlen: int = 16384, window: int = 4096) -> Workload:
     (each row sees itself and the window - 1 keys before it)."""
     return Workload(f"gqa_s{seqlen}_hq32_hkv8_d128_causal_window{window}", [seqlen], 32, 8,
                     128, True, window=(window - 1, 0))
+
+
+def decode_gqa(q_rows: int = 64, seqlen_k: int = 65536) -> Workload:
+    """A short query segment (the last q_rows positions) against a long key
+    segment: the SplitKV shape.  GQA 32/8, head_dim 128, causal (bottom-right)."""
+    return Workload(f"decode_q{q_rows}_k{seqlen_k}_hq32_hkv8_d128_causal", [q_rows], 32, 8, 128,
+                    True, lengths_k=[seqlen_k])
 
 
 def gqa_softcap(seqlen: int = 16384, cap: float = 50.0) -> Workload:

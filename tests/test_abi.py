@@ -79,6 +79,32 @@ def test_fwd_ex_rejects_bad_softcap(lib, cap):
     assert rc == 1
 
 
+def _fwd_split(lib, splits, ws=256, ws_bytes=1 << 30, batch=1):
+    vp = ctypes.c_void_p
+    return lib.attn_fwd_split(vp(16), vp(16), vp(16), vp(16), vp(16), batch, 128, 128, 128, 128,
+                              4, 2, 128, 0.088, 0, -1, -1, 0.0, splits, 1, vp(16), vp(16),
+                              vp(ws) if ws else None, ws_bytes, None)
+
+
+@pytest.mark.parametrize("splits,kw", [
+    (0, {}), (129, {}),                   # split count out of range
+    (2, {"batch": 40000}),                # batch * splits beyond the grid's z limit
+    (2, {"ws": 0}),                       # no workspace
+    (2, {"ws": 272}),                     # workspace not 256-byte aligned
+    (2, {"ws_bytes": 1024}),              # workspace too small
+])
+def test_fwd_split_rejects_bad_arguments(lib, splits, kw):
+    assert _fwd_split(lib, splits, **kw) == 1
+
+
+def test_fwd_split_workspace_size(lib):
+    assert lib.attn_fwd_split_workspace_size(128, 4, 128, 0) == 0
+    assert lib.attn_fwd_split_workspace_size(128, 4, 128, 129) == 0
+    one = lib.attn_fwd_split_workspace_size(128, 4, 128, 1)
+    four = lib.attn_fwd_split_workspace_size(128, 4, 128, 4)
+    assert one >= 128 * 4 * 128 * 4 and four >= 4 * 128 * 4 * 128 * 4 and four > one
+
+
 def test_bwd_rejects_small_workspace(lib):
     vp = ctypes.c_void_p
     need = lib.attn_bwd_workspace_size(1, 128, 4, 128)

@@ -13,14 +13,14 @@ pytestmark = pytest.mark.gpu
 ea = pytest.importorskip("exact_attention_129_b200")
 
 
-def run_fwd(wl, return_lse=True, guard=True, window=None, softcap=0.0):
+def run_fwd(wl, return_lse=True, guard=True, window=None, softcap=0.0, num_splits=1):
     host, (q, k, v, _), cu_q, cu_k = to_dev(wl, with_dout=False)
     dev = q.device
     obuf, out, og = guarded_empty(q.shape, torch.bfloat16, dev)
     lbuf, lse, lg = guarded_empty((wl.hq, wl.total_q), torch.float32, dev)
     ea.attn_fwd(q, k, v, cu_q, cu_k, wl.max_q, wl.max_k, scale=wl.scale, causal=wl.causal,
                 window=window, softcap=softcap, return_lse=return_lse, out=out,
-                lse=lse if return_lse else None)
+                lse=lse if return_lse else None, num_splits=num_splits)
     rc, msg = ea.last_device_error()
     assert rc == 0, msg
     assert guards_intact(obuf, og), "out guard band overwritten"
@@ -35,8 +35,8 @@ def few_key_o_tol(v):
     return max(O_TOL, 3 * 2.0 ** -9 * float(np.abs(np.asarray(v, np.float64)).max()))
 
 
-def check_full(wl, window=None, softcap=0.0, o_tol=None):
-    host, out, lse = run_fwd(wl, window=window, softcap=softcap)
+def check_full(wl, window=None, softcap=0.0, o_tol=None, num_splits=1):
+    host, out, lse = run_fwd(wl, window=window, softcap=softcap, num_splits=num_splits)
     q, k, v, _ = host
     ref_o, ref_lse = oracle.fwd(q, k, v, wl.cu_q, wl.cu_k, wl.scale, wl.causal, window=window,
                                 softcap=softcap)
@@ -122,6 +122,32 @@ def test_softcap(d, cap):
     wl = si.Workload(f"softcap{cap}_causal_d{d}", [515, 70], 4, 1, d, True, seed=32)
     check_full(wl, softcap=cap, window=(150, 0),
                o_tol=few_key_o_tol(wl.tensors(False)[2].float()))
+
+
+# SplitKV: short query segments against long key segments, split counts from 1
+# to more than there are key blocks (the extra splits see no key)
+DECODE = dict(lengths_q=[1, 3, 64, 130], lengths_k=[2000, 5000, 300, 1024])
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("splits", [1, 2, 3, 7, 64, 128])
+def test_splitkv(d, splits):
+    for causal in (False, True):
+        wl = si.Workload(f"decode_d{d}_s{splits}", DECODE["lengths_q"], 8, 2, d, causal,
+                         lengths_k=DECODE["lengths_k"], seed=60)
+        check_full(wl, num_splits=splits)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_splitkv_window_softcap_no_lse(d):
+    wl = si.Workload(f"decode_mask_d{d}", DECODE["lengths_q"], 4, 1, d, True,
+                     lengths_k=DECODE["lengths_k"], seed=61)
+    check_full(wl, num_splits=5, window=(700, 0), softcap=20.0,
+               o_tol=few_key_o_tol(wl.tensors(False)[2].float()))
+    # return_lse off: O must not change
+    _, o1, _ = run_fwd(wl, num_splits=5, window=(700, 0), softcap=20.0)
+    _, o2, _ = run_fwd(wl, return_lse=False, num_splits=5, window=(700, 0), softcap=20.0)
+    assert torch.equal(o1, o2)
 
 
 def test_deterministic():
