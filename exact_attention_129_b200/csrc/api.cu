@@ -87,6 +87,24 @@ uint64_t test_epilogue_delay_ns() {
   return static_cast<uint64_t>(us) * 1000ull;
 }
 
+// Packed GQA for the forward: a CTA serves all G query heads of a key/value head
+// (tile row r = query row r / G of head r % G), so short query segments fill
+// its tiles and K/V is loaded once per group.  Used when G is a power of two in
+// [2, 16] and the longest query segment would leave a tile mostly empty
+// (max_seqlen_q < 128).  ATTN_PACK_GQA=0 / 1 forces it off / on (where G allows),
+// read on every call so tests can exercise both.  Returns log2 G or 0.
+int pack_gqa_shift(int group, int max_seqlen_q) {
+  if (group < 2 || group > 16 || (group & (group - 1)) != 0) return 0;
+  const char* e = std::getenv("ATTN_PACK_GQA");
+  bool on = max_seqlen_q < 128;
+  if (e && e[0] == '0') on = false;
+  if (e && e[0] == '1') on = true;
+  if (!on) return 0;
+  int sh = 0;
+  while ((1 << sh) < group) ++sh;
+  return sh;
+}
+
 // Per-device set-up, once: the error word's device address and the device's
 // compute capability.
 DeviceState* device_state(int* dev_out) {
@@ -128,14 +146,16 @@ bool make_map_f32(CUtensorMap* map, const void* ptr, int rows, int heads, int d,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_map(CUtensorMap* map, const void* ptr, int rows, int heads, int d, int box_rows) {
+bool make_map(CUtensorMap* map, const void* ptr, int rows, int heads, int d, int box_rows,
+              int box_heads = 1) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
                               static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                                  static_cast<cuuint64_t>(heads) * d * 2};
-  const cuuint32_t box[3] = {64u, 1u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_heads),
+                             static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -195,7 +215,10 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_
   // Q: one 128-row box per 64-column panel; K: one BN-row box per panel;
   // V: VROWS rows per box, all panels of a chunk together
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, total_q, hq, D, C::BM) || !make_map(&mk, k, total_k, hkv, D, C::BN) ||
+  // packed GQA: one box holds BM/G query rows of all G heads of a group
+  const int g = 1 << p.pack_shift;
+  if (!make_map(&mq, q, total_q, hq, D, C::BM / g, g) ||
+      !make_map(&mk, k, total_k, hkv, D, C::BN) ||
       !make_map(&mv, v, total_k, hkv, D, C::VROWS))
     return ATTN_ERR_CUDA;
   static std::once_flag attr_once[kMaxDevices];
@@ -207,9 +230,10 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
-  const int m_tiles = (max_q + C::BM * C::NQ - 1) / (C::BM * C::NQ);
+  const int rows_per_cta = (C::BM * C::NQ) >> p.pack_shift;
+  const int m_tiles = (max_q + rows_per_cta - 1) / rows_per_cta;
   if (m_tiles == 0) return ATTN_OK;
-  dim3 grid(m_tiles, hq, batch);
+  dim3 grid(m_tiles, p.pack_shift > 0 ? hkv : hq, batch);
   record_start(ATTN_KERNEL_FWD, stream);
   attn_fwd_kernel<D, CAUSAL, SOFTCAP><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv,
                                                                                   p);
@@ -378,6 +402,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
         static_cast<uint8_t*>(workspace) +
         bwd_align256(static_cast<size_t>(num_splits) * total_q * nheads_q * head_dim * 4));
   }
+  p.pack_shift = pack_gqa_shift(nheads_q / nheads_kv, max_seqlen_q);
   p.timeout_ns = wait_timeout_ns();
   p.epilogue_delay_ns = test_epilogue_delay_ns();
 

@@ -83,6 +83,10 @@ struct FwdParams {
   int num_splits;
   float* o_part;    // fp32 [num_splits][total_q][nheads_q][D]
   float* lse_part;  // fp32 [num_splits][nheads_q][total_q]
+  // packed GQA (pack_shift > 0): a CTA serves one key/value head and all
+  // G = 1 << pack_shift query heads of its group; tile row r is query row
+  // r >> pack_shift of head (r & (G - 1)), and grid.y runs over key/value heads
+  int pack_shift;
   uint64_t timeout_ns;
   // test hook (0 in normal use): the softmax warps idle this long before their
   // final wait, so the tile's last P.V is sure to have completed by then
@@ -195,7 +199,8 @@ __device__ __forceinline__ FwdSmem fwd_smem(uint8_t* base) {
 // Number of key blocks a CTA visits and the rows it covers.
 struct FwdTile {
   int q0, sq, k0, sk;   // segment offsets / lengths
-  int m_base;           // first segment-local row of the CTA
+  int m_base;           // first segment-local query row of the CTA
+  int rows;             // query rows per tile: BM, or BM / G when packing GQA
   int n_lo;             // first key block to visit
   int n_blocks;         // key blocks to visit: [n_lo, n_lo + n_blocks)
   int h, hk;
@@ -206,10 +211,11 @@ struct FwdTile {
 // buffer of this CTA's split, and the row's partial LSE
 template <int D>
 __device__ __forceinline__ void fwd_store_part(const FwdParams& p, const FwdTile& t, int row,
-                                               int col0, const uint32_t (&r)[32], float inv_l) {
+                                               int head, int col0, const uint32_t (&r)[32],
+                                               float inv_l) {
   if (row >= t.sq) return;
   float* dst = p.o_part +
-               ((static_cast<size_t>(t.split) * p.total_q + t.q0 + row) * p.nheads_q + t.h) * D +
+               ((static_cast<size_t>(t.split) * p.total_q + t.q0 + row) * p.nheads_q + head) * D +
                col0;
 #pragma unroll
   for (int g = 0; g < 8; ++g)
@@ -218,9 +224,9 @@ __device__ __forceinline__ void fwd_store_part(const FwdParams& p, const FwdTile
                     __uint_as_float(r[4 * g + 2]) * inv_l, __uint_as_float(r[4 * g + 3]) * inv_l);
 }
 __device__ __forceinline__ void fwd_store_part_lse(const FwdParams& p, const FwdTile& t, int row,
-                                                   float lse) {
+                                                   int head, float lse) {
   if (row < t.sq)
-    p.lse_part[(static_cast<size_t>(t.split) * p.nheads_q + t.h) * p.total_q + t.q0 + row] = lse;
+    p.lse_part[(static_cast<size_t>(t.split) * p.nheads_q + head) * p.total_q + t.q0 + row] = lse;
 }
 
 template <int D, bool CAUSAL>
@@ -228,21 +234,27 @@ __device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t) {
   using C = FwdCfg<D>;
   const int b = blockIdx.z / p.num_splits;
   t.split = blockIdx.z % p.num_splits;
-  t.h = blockIdx.y;
-  t.hk = t.h / (p.nheads_q / p.nheads_kv);
+  if (p.pack_shift > 0) {
+    t.hk = blockIdx.y;
+    t.h = t.hk << p.pack_shift;  // first query head of the group
+  } else {
+    t.h = blockIdx.y;
+    t.hk = t.h / (p.nheads_q / p.nheads_kv);
+  }
+  t.rows = C::BM >> p.pack_shift;
   t.q0 = p.cu_q[b];
   t.sq = p.cu_q[b + 1] - t.q0;
   t.k0 = p.cu_k[b];
   t.sk = p.cu_k[b + 1] - t.k0;
   // causal: heaviest tiles (bottom of the segment) first
   const int m_tile = CAUSAL ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
-  t.m_base = m_tile * C::BM * C::NQ;
+  t.m_base = m_tile * t.rows * C::NQ;
   if (t.m_base >= t.sq) return false;
   // the union of the rows' allowed key ranges
   const int delta = t.sk - t.sq;
   int n_end = t.sk;
   if (CAUSAL) {
-    const int last_row = min(t.sq, t.m_base + C::BM * C::NQ) - 1;
+    const int last_row = min(t.sq, t.m_base + t.rows * C::NQ) - 1;
     n_end = min(t.sk, last_row + delta + p.hi_off + 1);
   }
   const int n_beg = (p.lo_off < kNoBound) ? max(0, t.m_base + delta - p.lo_off) : 0;
@@ -269,18 +281,19 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, c
   using C = FwdCfg<D>;
   if (t.n_blocks == 0) return;  // nothing to attend to: no copy may outlive the CTA
   for (int qt = 0; qt < C::NQ; ++qt) {
-    if (t.m_base + qt * C::BM >= t.sq) break;
+    if (t.m_base + qt * t.rows >= t.sq) break;
     mbar_expect_tx(&s.q_full[qt], C::Q_BYTES);
+    // one box per panel: t.rows query rows x (packed: all G heads) x 64 columns
     for (int pn = 0; pn < C::PANELS; ++pn)
       tma_load_3d(s.q + qt * C::Q_BYTES + pn * C::QPANEL, tmQ, &s.q_full[qt], pn * 64, t.h,
-                  t.q0 + t.m_base + qt * C::BM);
+                  t.q0 + t.m_base + qt * t.rows);
   }
   uint32_t ring = 0;  // stages issued so far
   // on the way out after a timed-out wait elsewhere: let every copy this CTA
   // issued land before its shared memory is released
   auto drain = [&]() {
     for (int qt = 0; qt < C::NQ; ++qt)
-      if (t.m_base + qt * C::BM < t.sq) mbar_wait_drain(&s.q_full[qt], 0, 100000000ull);
+      if (t.m_base + qt * t.rows < t.sq) mbar_wait_drain(&s.q_full[qt], 0, 100000000ull);
     const uint32_t first = ring > (uint32_t)C::NSTAGE ? ring - C::NSTAGE : 0u;
     for (uint32_t r = first; r < ring; ++r)
       mbar_wait_drain(&s.kv_full[r % C::NSTAGE], (r / C::NSTAGE) & 1, 100000000ull);
@@ -518,7 +531,9 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   const int warp = (threadIdx.x >> 5) & 3;  // warp within the warpgroup = TMEM lane quadrant
   const int lane = lane_id();
   const int row_in_tile = warp * 32 + lane;
-  const int row = t.m_base + qt * C::BM + row_in_tile;  // segment-local query row
+  // segment-local query row and query head of this thread's tile row
+  const int row = t.m_base + qt * t.rows + (row_in_tile >> p.pack_shift);
+  const int head = t.h + (row_in_tile & ((1 << p.pack_shift) - 1));
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
   const int n = t.n_blocks;
   // with a softcap the scores are turned into capped log2-domain values first
@@ -530,16 +545,16 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   // a block needs element masks for this warpgroup when it crosses the upper
   // bound of the tile's first row (or the end of the keys) or the lower bound
   // of its last row
-  const int tile_row0 = t.m_base + qt * C::BM;
+  const int tile_row0 = t.m_base + qt * t.rows;
   const int mask_from = CAUSAL ? min(t.sk, tile_row0 + delta + p.hi_off + 1) : t.sk;
-  const int lo_until = tile_row0 + (C::BM - 1) + delta - p.lo_off;
+  const int lo_until = tile_row0 + (t.rows - 1) + delta - p.lo_off;
 
   // With two query tiles, warp w of each tile shares an SM sub-partition and
   // its special-function unit: their exp phases take turns (tile 0 first in
   // each block) through a pair of named barriers, so one warp's loads, max and
   // stores overlap the other's exps.  A warp that gives up on a timed-out wait
   // still plays its remaining turns, so its partner never waits forever.
-  const bool pingpong = C::DBUF && C::ROW_SPLIT == 1 && (t.m_base + C::BM < t.sq);
+  const bool pingpong = C::DBUF && C::ROW_SPLIT == 1 && (t.m_base + t.rows < t.sq);
   const int bar_t0 = 3 + 2 * warp, bar_t1 = 4 + 2 * warp;  // "tile 0 / tile 1 may start"
   auto turn_begin = [&](int k) {
     if (qt == 0) {
@@ -735,7 +750,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
         for (int i = 0; i < 32; ++i) r[i] = 0u;
       }
       if (p.num_splits > 1) {  // SplitKV: fp32 partial, straight from registers
-        fwd_store_part<D>(p, t, row, cc * 32, r, inv_l);
+        fwd_store_part<D>(p, t, row, head, cc * 32, r, inv_l);
         continue;
       }
 #pragma unroll
@@ -753,7 +768,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   }
   named_bar_sync(1 + qt, 128);
   if (ok && p.num_splits > 1) {
-    fwd_store_part_lse(p, t, row,
+    fwd_store_part_lse(p, t, row, head,
                        (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f
                                      : -INFINITY);
   } else if (ok) {
@@ -763,17 +778,18 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
 #pragma unroll 4
     for (int q = tid; q < C::BM * CPR; q += 128) {
       const int r = q / CPR, ch = q % CPR;
-      if (r < rows_left) {
+      if ((r >> p.pack_shift) < rows_left) {
         const uint4 v =
             *reinterpret_cast<const uint4*>(stage + r * (D * 2) + ((ch ^ (r & 7)) * 16));
-        const size_t grow = static_cast<size_t>(t.q0 + tile_row0 + r);
-        *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + t.h) * D) * 2 + ch * 16) = v;
+        const size_t grow = static_cast<size_t>(t.q0 + tile_row0 + (r >> p.pack_shift));
+        const int gh = t.h + (r & ((1 << p.pack_shift) - 1));
+        *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + gh) * D) * 2 + ch * 16) = v;
       }
     }
     if (p.return_lse && row_valid) {
       const float lse =
           (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
-      p.lse[static_cast<size_t>(t.h) * p.total_q + t.q0 + row] = lse;
+      p.lse[static_cast<size_t>(head) * p.total_q + t.q0 + row] = lse;
     }
   }
 }
@@ -799,16 +815,17 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
   const int quad = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant
   const int lane = lane_id();
   const int row_in_tile = quad * 32 + lane;
-  const int row = t.m_base + qt * C::BM + row_in_tile;
+  const int row = t.m_base + qt * t.rows + (row_in_tile >> p.pack_shift);
+  const int head = t.h + (row_in_tile & ((1 << p.pack_shift) - 1));
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
   const int n = t.n_blocks;
   const float c = SOFTCAP ? 1.f : p.scale_log2;
   const int delta = t.sk - t.sq;
   const int key_lim = CAUSAL ? min(t.sk, row + delta + p.hi_off + 1) : t.sk;
   const int key_lo = row + delta - p.lo_off;
-  const int tile_row0 = t.m_base + qt * C::BM;
+  const int tile_row0 = t.m_base + qt * t.rows;
   const int mask_from = CAUSAL ? min(t.sk, tile_row0 + delta + p.hi_off + 1) : t.sk;
-  const int lo_until = tile_row0 + (C::BM - 1) + delta - p.lo_off;
+  const int lo_until = tile_row0 + (t.rows - 1) + delta - p.lo_off;
   const int pair_bar = 3 + qt * 4 + quad;
   float* xch = s.xch + qt * (2 * 2 * C::BM);  // [block parity][half][row]
 
@@ -957,7 +974,7 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
         for (int i = 0; i < 32; ++i) r[i] = 0u;
       }
       if (p.num_splits > 1) {  // SplitKV: fp32 partial, straight from registers
-        fwd_store_part<D>(p, t, row, hf * OC + cc * 32, r, inv_l);
+        fwd_store_part<D>(p, t, row, head, hf * OC + cc * 32, r, inv_l);
         continue;
       }
 #pragma unroll
@@ -976,7 +993,7 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
   named_bar_sync(1 + qt, 256);  // both halves of the tile
   if (ok && p.num_splits > 1) {
     if (hf == 0)
-      fwd_store_part_lse(p, t, row,
+      fwd_store_part_lse(p, t, row, head,
                          (l_tot > 0.f) ? (m_run + __log2f(l_tot)) * 0.69314718055994530942f
                                        : -INFINITY);
   } else if (ok) {
@@ -986,17 +1003,18 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
 #pragma unroll 4
     for (int q = tid; q < C::BM * CPR; q += 256) {
       const int r = q / CPR, ch = q % CPR;
-      if (r < rows_left) {
+      if ((r >> p.pack_shift) < rows_left) {
         const uint4 v =
             *reinterpret_cast<const uint4*>(stage + r * (D * 2) + ((ch ^ (r & 7)) * 16));
-        const size_t grow = static_cast<size_t>(t.q0 + tile_row0 + r);
-        *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + t.h) * D) * 2 + ch * 16) = v;
+        const size_t grow = static_cast<size_t>(t.q0 + tile_row0 + (r >> p.pack_shift));
+        const int gh = t.h + (r & ((1 << p.pack_shift) - 1));
+        *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + gh) * D) * 2 + ch * 16) = v;
       }
     }
     if (p.return_lse && row_valid && hf == 0) {
       const float lse =
           (l_tot > 0.f) ? (m_run + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
-      p.lse[static_cast<size_t>(t.h) * p.total_q + t.q0 + row] = lse;
+      p.lse[static_cast<size_t>(head) * p.total_q + t.q0 + row] = lse;
     }
   }
 }
@@ -1018,7 +1036,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NQ; ++i) mbar_init(&s.q_full[i], 1);
     // every MMA warp with a query tile releases each ring stage once
-    const int n_mma = (t.m_base + C::BM < t.sq && C::NQ == 2) ? 2 : 1;
+    const int n_mma = (t.m_base + t.rows < t.sq && C::NQ == 2) ? 2 : 1;
     for (int i = 0; i < C::NSTAGE; ++i) {
       mbar_init(&s.kv_full[i], 1);
       mbar_init(&s.kv_empty[i], n_mma);
@@ -1051,7 +1069,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   if (warp < C::SOFTMAX_WARPS) {
     const int grp = warp / 4;
     const int qt = grp / C::ROW_SPLIT;
-    if (t.m_base + qt * C::BM < t.sq) {
+    if (t.m_base + qt * t.rows < t.sq) {
       if constexpr (C::ROW_SPLIT == 2)
         fwd_softmax_split<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt, grp % 2);
       else
@@ -1061,7 +1079,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     if (lane_id() == 0) fwd_load<D>(p, t, s, &tmQ, &tmK, &tmV);
   } else {
     const int qt = warp - C::MMA_WARP;
-    if (lane_id() == 0 && t.m_base + qt * C::BM < t.sq) fwd_mma<D>(p, t, s, tmem, qt);
+    if (lane_id() == 0 && t.m_base + qt * t.rows < t.sq) fwd_mma<D>(p, t, s, tmem, qt);
     __syncwarp();
   }
   tc_fence_before();

@@ -150,6 +150,38 @@ def test_splitkv_window_softcap_no_lse(d):
     assert torch.equal(o1, o2)
 
 
+# packed GQA: the G query heads of a key/value head share the tile rows
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("group", [2, 4, 8, 16])
+def test_pack_gqa_forced(d, group, monkeypatch):
+    monkeypatch.setenv("ATTN_PACK_GQA", "1")
+    hkv = 2 if group <= 8 else 1
+    for causal in (False, True):
+        wl = si.Workload(f"pack_g{group}_d{d}", [300, 1, 515, 129], group * hkv, hkv, d, causal,
+                         lengths_k=[400, 1, 515, 64], seed=70 + group)
+        # causal: the first rows of a segment see one or two keys (few-key bound)
+        check_full(wl, o_tol=few_key_o_tol(wl.tensors(False)[2].float()) if causal else None)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_pack_gqa_masks_and_splits(d, monkeypatch):
+    monkeypatch.setenv("ATTN_PACK_GQA", "1")
+    wl = si.Workload(f"pack_mask_d{d}", [77, 200, 5], 8, 2, d, True, lengths_k=[900, 200, 3000],
+                     seed=80)
+    tol = few_key_o_tol(wl.tensors(False)[2].float())
+    check_full(wl, window=(300, 0), softcap=10.0, o_tol=tol)
+    check_full(wl, num_splits=4, window=(300, 0), o_tol=tol)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_decode_shapes_default_path(d):
+    # max_seqlen_q < 128 with G = 4: packed by default, with and without SplitKV
+    wl = si.Workload(f"decode_small_d{d}", [1, 16, 100], 8, 2, d, True,
+                     lengths_k=[3000, 700, 4100], seed=81)
+    for splits in (1, 6):
+        check_full(wl, num_splits=splits)
+
+
 def test_deterministic():
     wl = si.Workload("det", [777, 1500], 4, 2, 128, True, seed=8)
     outs = [run_fwd(wl)[1:] for _ in range(3)]
