@@ -134,7 +134,17 @@ struct BwdCfg {
   // its own barriers while the other keeps the tensor pipe busy
   static constexpr int ELEM_THREADS = 256;
   static constexpr bool TWO_ISSUERS = (NSPLIT == 1);
-  static constexpr int THREADS = TWO_ISSUERS ? 352 : 320;
+  // head_dim 64/128: warps 12-15 read dQ^T out of tensor memory and issue its
+  // TMA reduce-adds, so the elementwise warps never wait for dQ.  The 16 warps
+  // start with 128 registers each (65,536 in all); the warpgroups then set
+  // their own budgets: elementwise 184, control (loader, MMA x2, one idle) 64,
+  // dQ 80.  Per SM sub-partition (one warp of each warpgroup) that is 512
+  // registers per lane, exactly its 16,384.
+  static constexpr bool DQ_WARPS = TWO_ISSUERS;
+  static constexpr int DQ_WARP0 = 12;
+  static constexpr int REG_ELEM = 184, REG_CTRL = 64, REG_DQ = 80;
+  static_assert(!DQ_WARPS || 2 * REG_ELEM + REG_CTRL + REG_DQ <= 512, "register split");
+  static constexpr int THREADS = DQ_WARPS ? 512 : (TWO_ISSUERS ? 352 : 320);
   static constexpr int LOAD_WARP = 8, MMA_WARP = 9, GRAD_WARP = 10;
   // tensor memory columns
   static constexpr int COL_S = 0, COL_DP = 128, COL_DQ = 192, COL_DV = 256, COL_DK = 256 + DH;
@@ -668,14 +678,14 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     if (tid == 0 && i < 200) TRACE(i * 8 + 3);
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.ds_ready[b]);
-    if (i >= 1 && !dq_out(i - 1)) {
+    if (!C::DQ_WARPS && i >= 1 && !dq_out(i - 1)) {
       ok = false;
       break;
     }
     if (tid == 0 && i < 200) TRACE(i * 8 + 4);
   }
-  if (ok && t.n_iter > 0) ok = dq_out(t.n_iter - 1);
-  if constexpr (C::DQ_TMA) {
+  if (!C::DQ_WARPS && ok && t.n_iter > 0) ok = dq_out(t.n_iter - 1);
+  if constexpr (C::DQ_TMA && !C::DQ_WARPS) {
     if (lane == 0) bulk_wait0();  // this warp's reduces are complete
   }
   if (ok && t.n_iter > 0) ok = uniform_wait(s.dkv_full, 0, 5);
@@ -711,6 +721,53 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
   }
 }
 
+// ---------------------------------------------------------------------------
+// dQ warpgroup (head_dim 64/128): warp wq reads features [32 wq, 32 wq + 32) of
+// dQ^T (TMEM lane = feature) for all 64 query columns of a block and adds them
+// into the fp32 accumulator with TMA reduce-adds, 32 queries at a time.
+// Query rows past the segment carry exact zeros (their P is 0).
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void bwd_dq(const BwdParams& p, const BwdTile& t, const BwdSmem& s,
+                                       uint32_t tmem, const CUtensorMap* tmDQ) {
+  using C = BwdCfg<D>;
+  const int wq = (threadIdx.x >> 5) & 3;
+  const int lane = lane_id();
+  const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+  const int mcount = t.m_hi - t.m_lo;
+  const bool d_ok = wq * 32 < C::DH;  // head_dim 64: lanes 64-127 hold the zero panel
+  for (int j = 0; j < t.n_iter; ++j) {
+    if (!__all_sync(0xffffffffu, mbar_wait(s.dq_full, j & 1, s.abort, p.err, ERR_BWD_ELEM | 1,
+                                           p.timeout_ns)))
+      break;
+    tc_fence_after();
+    const int h = t.h0 + j / mcount;
+    const int m0 = (t.m_lo + j % mcount) * C::BM;
+    uint32_t r0[32], r1[32];
+    tmem_ld32x2(tmem + lane_base + C::COL_DQ, r0, tmem + lane_base + C::COL_DQ + 32, r1);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.dq_free);
+    if (!d_ok) continue;
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {
+      float* stg = reinterpret_cast<float*>(s.dqs + (hq * (C::DH / 32) + wq) * C::DQ_WARP_BYTES);
+      // this slot's previous reduce (one group before the other slot's) has read it
+      if (lane == 0) bulk_wait_read1();
+      __syncwarp();
+#pragma unroll
+      for (int x = 0; x < 32; ++x) stg[x * 32 + lane] = __uint_as_float(hq ? r1[x] : r0[x]);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_3d(tmDQ, stg, t.dh * C::DH + wq * 32, h, t.q0 + m0 + hq * 32);
+        bulk_commit();
+      }
+    }
+  }
+  if (lane == 0) bulk_wait0();  // every reduce of this warp is complete
+}
+
 template <int D, bool CAUSAL, bool SOFTCAP>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -741,7 +798,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     mbar_init(s.dp_full, 1);
     mbar_init(s.dp_free, C::ELEM_THREADS / 32);
     mbar_init(s.dq_full, 1);
-    mbar_init(s.dq_free, C::ELEM_THREADS / 32);
+    mbar_init(s.dq_free, C::DQ_WARPS ? 4 : C::ELEM_THREADS / 32);
     mbar_init(s.dkv_full, 1);
     mbar_init(s.oth_full, 1);
     mbar_init(s.oth_empty, 1);
@@ -769,13 +826,24 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s.tmem_base;
+  // each warpgroup sets its register budget in the branch it then runs (every
+  // warp of a warpgroup executes the same setmaxnreg)
   if (warp < 8) {
+    if constexpr (C::DQ_WARPS) setmaxnreg_inc<C::REG_ELEM>();
     bwd_elem<D, CAUSAL, SOFTCAP>(p, t, s, tmem, &tmDQ);
-  } else if (warp == C::LOAD_WARP) {
-    bwd_load<D>(p, t, s, &tmK, &tmV, &tmQ, &tmO);
+  } else if (!C::DQ_WARPS || warp < C::DQ_WARP0) {
+    if constexpr (C::DQ_WARPS) setmaxnreg_dec<C::REG_CTRL>();
+    if (warp == C::LOAD_WARP) {
+      bwd_load<D>(p, t, s, &tmK, &tmV, &tmQ, &tmO);
+    } else if (warp == C::MMA_WARP || warp == C::GRAD_WARP) {
+      if (lane_id() == 0) bwd_mma<D>(p, t, s, tmem, warp - C::MMA_WARP);
+      __syncwarp();
+    }
   } else {
-    if (lane_id() == 0) bwd_mma<D>(p, t, s, tmem, warp - C::MMA_WARP);
-    __syncwarp();
+    if constexpr (C::DQ_WARPS) {
+      setmaxnreg_dec<C::REG_DQ>();
+      bwd_dq<D>(p, t, s, tmem, &tmDQ);
+    }
   }
   tc_fence_before();
   __syncthreads();
