@@ -17,13 +17,13 @@
 //
 // Main-kernel layout for one CTA (128 keys; head_dim 256 is split into two
 // 128-wide halves handled by two CTAs, each recomputing S and dP in full):
-//   tensor memory: S^T x2 (64 cols each; P^T in bf16 is written back over
-//                  columns 0-15 and 32-47), dP^T (64), dQ^T (64), dV (DH),
+//   tensor memory: S^T x2 (64 cols each; per warpgroup P^T in bf16 is written
+//                  back over columns 0-15 / 32-47 and dS^T over 16-31 / 48-63,
+//                  the A operands of dV and dK), dP^T (64), dQ^T (64), dV (DH),
 //                  dK (DH)  = 512 cols
 //   shared memory: K and V tiles (resident), a ring of NST (Q, dO) stages of
 //                  64 query rows, two dS^T tiles (128 keys x 64 queries, bf16,
-//                  128-byte swizzled: the same bytes are the K-major A operand of
-//                  dK += dS^T Q and the MN-major B operand of dQ^T = K^T dS^T),
+//                  128-byte swizzled: the MN-major B operand of dQ^T = K^T dS^T),
 //                  and per-block LSE/D vectors.
 //   warps: 4 elementwise warps (thread = key row = TMEM lane), 1 TMA warp,
 //          1 MMA warp.
@@ -403,10 +403,12 @@ struct BwdMma {
       mma_ts(tmem + C::COL_DV, tmem + C::COL_S + bj * 64 + (ks >> 1) * 32 + (ks & 1) * 8,
              sdesc_sw128(do_half + ks * 2048, C::QD_PANEL, 1024), C::IDESC_KV,
              (!first || ks) ? 1u : 0u);
-    // dK += dS^T Q  (A = dS^T K-major in shared memory)
+    // dK += dS^T Q  (A = dS^T in tensor memory, 16 columns after each
+    // warpgroup's P^T; the shared-memory copy is for dQ)
+    (void)ds;
 #pragma unroll
     for (int ks = 0; ks < C::BM / 16; ++ks)
-      mma_ss(tmem + C::COL_DK, sdesc_sw128(ds + ks * 32, 16, 1024),
+      mma_ts(tmem + C::COL_DK, tmem + C::COL_S + bj * 64 + (ks >> 1) * 32 + 16 + (ks & 1) * 8,
              sdesc_sw128(q_half + ks * 2048, C::QD_PANEL, 1024), C::IDESC_KV,
              (!first || ks) ? 1u : 0u);
   }
@@ -662,6 +664,19 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     // columns, which this warpgroup has already read: the other warpgroup may
     // still be reading its own columns
     tmem_st16(tmem + lane_base + C::COL_S + b * 64 + wg * 32, pk);
+    {
+      // dS^T (bf16 pairs) over the other 16 of the warpgroup's own columns: the
+      // A operand of dK += dS^T Q, read from tensor memory
+      uint32_t dsw[16];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        dsw[4 * ch] = dsk[ch].x;
+        dsw[4 * ch + 1] = dsk[ch].y;
+        dsw[4 * ch + 2] = dsk[ch].z;
+        dsw[4 * ch + 3] = dsk[ch].w;
+      }
+      tmem_st16(tmem + lane_base + C::COL_S + b * 64 + wg * 32 + 16, dsw);
+    }
     if (tid == 0 && i < 200) TRACE(i * 8 + 2);
     // the dS buffer b is free once the dK and dQ MMAs of block i-2 are done
     if (i >= 2 && !uniform_wait(&s.ds_free[b], ((i - 2) >> 1) & 1, 4)) {
