@@ -125,16 +125,16 @@ struct FwdCfg {
   static constexpr int CHUNK = BN * 128;       // ring slot: one K panel of BN rows
   static constexpr int VROWS = CHUNK / (2 * D);  // V key rows per chunk (all D columns)
   static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int NSLOT = (D == 64) ? 14 : (D == 128 ? 20 : 10);
+  static constexpr int NSLOT = (D == 64) ? 14 : (D == 128 ? 20 : 9);
   // ring barriers guard stages of G chunks.  DBUF: stage j holds K_j and
   // V_{j-1} (exactly what one MMA iteration consumes), so each iteration waits
   // on and releases one barrier.  head_dim 256: one chunk per stage.
   static constexpr int G = DBUF ? 2 * PANELS : 1;
   static constexpr int NSTAGE = NSLOT / G;
-  // head_dim 64: two threads per query row, each with half of the row's key
-  // columns, so four softmax warps share each SM sub-partition and keep its
+  // head_dim 64 and 256: two threads per query row, each with half of the row's
+  // key columns, so more softmax warps share each SM sub-partition and keep its
   // exp unit busy (one warp alone cannot: its exps are latency-bound)
-  static constexpr int ROW_SPLIT = (D == 64) ? 2 : 1;
+  static constexpr int ROW_SPLIT = (D == 128) ? 1 : 2;
   static constexpr int SOFTMAX_WARPS = 4 * NQ * ROW_SPLIT;
   static constexpr int LOAD_WARP = SOFTMAX_WARPS;
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;  // one MMA warp per query tile
@@ -403,6 +403,45 @@ struct FwdMma {
       }
     }
   }
+  // head_dim 256 (one chunk per stage): the next tile's panels one at a time.
+  // Waiting for a panel's chunk right before its MMAs, and releasing it right
+  // after, lets each wait overlap the MMAs already queued.
+  __device__ bool wait_next_chunk() {
+    if (!mbar_wait(&s.kv_full[stage], phase, s.abort, p.err, ERR_FWD_MMA | 1, p.timeout_ns))
+      return false;
+    tc_fence_after();
+    return true;
+  }
+  __device__ bool issue_s_streamed(int qt, int slot) {
+    const uint32_t d_tmem = tmem + slot * C::BN;
+    const uint64_t qd = qdesc0 + (uint64_t)(qt * (C::Q_BYTES >> 4));
+    for (int c = 0; c < C::PANELS; ++c) {
+      if (!wait_next_chunk()) return false;
+      const uint64_t kd = kdesc0 + (uint64_t)(stage * C::G * (C::CHUNK >> 4));
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(d_tmem, qd + (c * (C::QPANEL >> 4) + kk * 2), kd + kk * 2, C::IDESC_S,
+               (c | kk) != 0);
+      release_stages(1);
+    }
+    return true;
+  }
+  __device__ bool issue_pv_streamed(int qt, int slot, bool accumulate) {
+    const uint32_t d_tmem = tmem + C::O_COL0 + qt * D;
+    const uint32_t p_tmem = tmem + slot * C::BN;
+    for (int c = 0; c < C::PANELS; ++c) {
+      if (!wait_next_chunk()) return false;
+      const uint64_t vd = vdesc0 + (uint64_t)(stage * C::G * (C::CHUNK >> 4));
+#pragma unroll
+      for (int kk = 0; kk < C::VROWS / 16; ++kk) {
+        const int kstep = c * (C::VROWS / 16) + kk;
+        mma_ts(d_tmem, p_tmem + kstep * 8, vd + kk * 128, C::IDESC_O,
+               (accumulate || kstep) ? 1u : 0u);
+      }
+      release_stages(1);
+    }
+    return true;
+  }
   __device__ static uint32_t wrap(uint32_t chunk) {
     if constexpr (C::G == 1) {
       if (chunk >= (uint32_t)C::NSLOT) chunk -= C::NSLOT;
@@ -487,34 +526,30 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
     }
     mma_commit(&s.o_final[qt]);
   } else {
-    // one query tile, two S slots alternating over key blocks; one chunk per stage
-    constexpr int P = C::PANELS;
-    uint32_t ch;
-    if (!m.wait_stages(P, ch)) return;
-    m.issue_s(0, 0, ch);
+    // one query tile, two S slots alternating over key blocks; one chunk per
+    // stage, each waited for right before its MMAs
+    if (!m.issue_s_streamed(0, 0)) return;
     mma_commit(&s.s_full[0]);
-    m.release_stages(P);
     if (n > 1) {
-      if (!m.wait_stages(P, ch)) return;
-      m.issue_s(0, 1, ch);
+      if (!m.issue_s_streamed(0, 1)) return;
       mma_commit(&s.s_full[1]);
-      m.release_stages(P);
     }
     for (int j = 0; j < n; ++j) {
       const int slot = j & 1;
+      [[maybe_unused]] const int tr = (j < 64) ? 2048 + 16 * j : -1;
+      TRACE(tr);
       if (!mbar_wait(&s.p_full[slot], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
                      p.timeout_ns))
         return;
       tc_fence_after();
-      if (!m.wait_stages(P, ch)) return;
-      m.issue_pv(0, slot, ch, j > 0);
+      TRACE(tr + 1);
+      if (!m.issue_pv_streamed(0, slot, j > 0)) return;
       mma_commit(&s.o_ready[0]);
-      m.release_stages(P);
+      TRACE(tr + 3);
       if (j + 2 < n) {
-        if (!m.wait_stages(P, ch)) return;
-        m.issue_s(0, slot, ch);
+        if (!m.issue_s_streamed(0, slot)) return;
         mma_commit(&s.s_full[slot]);
-        m.release_stages(P);
+        TRACE(tr + 5);
       }
     }
     mma_commit(&s.o_final[0]);
@@ -809,9 +844,16 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
                                                   const FwdSmem& s, uint32_t tmem, int qt,
                                                   int hf) {
   using C = FwdCfg<D>;
-  constexpr int NC = C::BN / 2;  // key columns per thread and block: 32 + 16
+  // key columns per thread and block: 96-key blocks (head_dim 64) 32 + 16,
+  // 128-key blocks (head_dim 256) 64
+  constexpr int NC = C::BN / 2;
   constexpr int OC = D / 2;      // O columns per thread
-  static_assert(C::BN == 96 && OC % 32 == 0, "row split layout");
+  static_assert((C::BN == 96 || C::BN == 128) && OC % 32 == 0, "row split layout");
+  // segment-local key (within the block) of this thread's score column i
+  auto key_of = [&](int i) {
+    if constexpr (C::BN == 96) return i < 32 ? hf * 32 + i : 64 + hf * 16 + (i - 32);
+    else return hf * 64 + i;
+  };
   const int quad = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant
   const int lane = lane_id();
   const int row_in_tile = quad * 32 + lane;
@@ -835,47 +877,53 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
   float l_run = 0.f;
   bool ok = true;
   for (int j = 0; j < n; ++j) {
-    const int slot = 2 * qt + (j & 1);
+    const int slot = C::DBUF ? 2 * qt + (j & 1) : (j & 1);
     [[maybe_unused]] const int tr = (tr_on && j < 64) ? 1024 * qt + j * 8 : -1;
     if (ok)
       ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], (j >> 1) & 1, s.abort, p.err,
                                              ERR_FWD_SOFTMAX | 1, p.timeout_ns));
     const uint32_t s_addr = tmem + lane_base + slot * C::BN;
-    uint32_t sa[32], sb[16];  // keys 32 hf + i, then 64 + 16 hf + i
+    uint32_t sr[NC];  // this thread's scores of the block (fp32 bits), see key_of
     float mx = -INFINITY;
     const int kb = (t.n_lo + j) * C::BN;  // segment-local key of column 0
     const bool masked = (kb + C::BN > mask_from) || (kb < lo_until);
     TRACE(tr);
     if (ok) {
       tc_fence_after();
-      tmem_ld32_16(s_addr + hf * 32, sa, s_addr + 64 + hf * 16, sb);
+      if constexpr (C::BN == 96) {
+        uint32_t sa[32], sb[16];
+        tmem_ld32_16(s_addr + hf * 32, sa, s_addr + 64 + hf * 16, sb);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sr[i] = sa[i];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sr[32 + i] = sb[i];
+      } else {
+        tmem_ld64(s_addr + hf * 64, sr);
+      }
       if (masked) {
         const int lim = key_lim - kb, lo = key_lo - kb;
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (hf * 32 + i >= lim || hf * 32 + i < lo) sa[i] = 0xff800000u;  // -inf
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (64 + hf * 16 + i >= lim || 64 + hf * 16 + i < lo) sb[i] = 0xff800000u;
+        for (int i = 0; i < NC; ++i)
+          if (key_of(i) >= lim || key_of(i) < lo) sr[i] = 0xff800000u;  // -inf
       }
       if constexpr (SOFTCAP) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sa[i] = fwd_cap(p, sa[i]);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sb[i] = fwd_cap(p, sb[i]);
+        for (int i = 0; i < NC; ++i) sr[i] = fwd_cap(p, sr[i]);
       }
       float ch[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        ch[k] = fmax3(__uint_as_float(sa[k]), __uint_as_float(sa[k + 8]),
-                      __uint_as_float(sa[k + 16]));
-        ch[k] = fmax3(ch[k], __uint_as_float(sa[k + 24]), __uint_as_float(sb[k]));
-        ch[k] = fmaxf(ch[k], __uint_as_float(sb[k + 8]));
-      }
+      for (int k = 0; k < 8; ++k) ch[k] = __uint_as_float(sr[k]);
+#pragma unroll
+      for (int i = 8; i < NC; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          ch[k] = (i + 8 < NC) ? fmax3(ch[k], __uint_as_float(sr[i + k]),
+                                       __uint_as_float(sr[i + 8 + k]))
+                               : fmaxf(ch[k], __uint_as_float(sr[i + k]));
       mx = fmaxf(fmax3(ch[0], ch[1], ch[2]), fmax3(ch[3], ch[4], fmax3(ch[5], ch[6], ch[7])));
     }
     // both threads of the row have read their scores once they pass the
-    // barrier, so P may then go over the slot's first 48 columns
+    // barrier, so P may then go over the slot's first BN/2 columns
     float* xb = xch + (j & 1) * (2 * C::BM);
     xb[hf * C::BM + row_in_tile] = mx;
     TRACE(tr + 1);
@@ -898,21 +946,29 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
     {
       const uint64_t cc2 = f2_pack(c, c), mm2 = f2_pack(-m_sub, -m_sub);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-      uint32_t pa[16], pb[8];  // P of keys 32 hf + 2i.. and 64 + 16 hf + 2i.. (bf16 pairs)
+      uint32_t pk[NC / 2];  // P of the score pairs (2i, 2i + 1), bf16
 #pragma unroll
-      for (int i = 0; i < 24; ++i) {
-        const uint32_t u0 = (i < 16) ? sa[2 * i] : sb[2 * (i - 16)];
-        const uint32_t u1 = (i < 16) ? sa[2 * i + 1] : sb[2 * (i - 16) + 1];
+      for (int i = 0; i < NC / 2; ++i) {
         float x0, x1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(u0), __uint_as_float(u1)), cc2, mm2), x0, x1);
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                         cc2, mm2),
+                  x0, x1);
         const float p0 = ex2(x0), p1 = ex2(x1);
         acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-        if (i < 16) pa[i] = pack_bf16(p0, p1);
-        else pb[i - 16] = pack_bf16(p0, p1);
+        pk[i] = pack_bf16(p0, p1);
       }
       // key k's P is at column k / 2 of the slot
-      tmem_st16(s_addr + hf * 16, pa);
-      tmem_st8(s_addr + 32 + hf * 8, pb);
+      if constexpr (C::BN == 96) {
+        uint32_t pa[16], pb[8];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pa[i] = pk[i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pb[i] = pk[16 + i];
+        tmem_st16(s_addr + hf * 16, pa);
+        tmem_st8(s_addr + 32 + hf * 8, pb);
+      } else {
+        tmem_st32(s_addr + hf * 32, pk);
+      }
       TRACE(tr + 3);
       float a0, a1, a2, a3;
       f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
