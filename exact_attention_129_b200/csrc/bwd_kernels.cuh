@@ -349,7 +349,7 @@ __device__ __forceinline__ void bwd_load(const BwdParams& p, const BwdTile& t, c
 }
 
 // ---------------------------------------------------------------------------
-// MMA warp (one thread issues)
+// MMA warps (all lanes run the role; one elected lane issues)
 // ---------------------------------------------------------------------------
 template <int D>
 struct BwdMma {
@@ -362,65 +362,68 @@ struct BwdMma {
       : p(p_), s(s_), t(t_), tmem(tm) {}
 
   __device__ bool wait(uint64_t* bar, uint32_t parity, uint32_t code) {
-    if (!mbar_wait(bar, parity, s.abort, p.err, ERR_BWD_MMA | code, p.timeout_ns)) return false;
+    if (!mbar_wait_warp(bar, parity, s.abort, p.err, ERR_BWD_MMA | code, p.timeout_ns))
+      return false;
     tc_fence_after();
     return true;
   }
+  // Shared-memory descriptors are built once per call; each MMA then adds its
+  // byte offset >> 4 to the start-address field (addresses stay below 256 KB,
+  // so the 14-bit field never carries), which keeps the issuing thread to a
+  // few instructions per MMA.
+  static __device__ __forceinline__ uint64_t at(uint64_t desc, uint32_t bytes) {
+    return desc + static_cast<uint64_t>(bytes >> 4);
+  }
   // X^T = A B^T with A = K or V (128 keys x D, K-major) and B = Q_i or dO_i (64 x D)
   __device__ void issue_kt(uint32_t d_col, const uint8_t* a, const uint8_t* b) {
-    const uint32_t aa = smem_u32(a), ba = smem_u32(b);
+    const uint64_t ad = sdesc_sw128(smem_u32(a), 16, 1024), bd = sdesc_sw128(smem_u32(b), 16, 1024);
 #pragma unroll
     for (int pn = 0; pn < C::PANELS; ++pn)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_ss(tmem + d_col, sdesc_sw128(aa + pn * C::KV_PANEL + kk * 32, 16, 1024),
-               sdesc_sw128(ba + pn * C::QD_PANEL + kk * 32, 16, 1024), C::IDESC_SDP,
-               (pn | kk) != 0);
+        mma_ss(tmem + d_col, at(ad, pn * C::KV_PANEL + kk * 32), at(bd, pn * C::QD_PANEL + kk * 32),
+               C::IDESC_SDP, (pn | kk) != 0);
   }
   // the K-steps of X^T = A B^T over panels [p0, p0 + 2) only (head_dim 256)
   __device__ void issue_kt_pair(uint32_t d_col, const uint8_t* a, const uint8_t* b, int p0,
                                 bool first) {
-    const uint32_t aa = smem_u32(a), ba = smem_u32(b);
+    const uint64_t ad = sdesc_sw128(smem_u32(a) + p0 * C::KV_PANEL, 16, 1024);
+    const uint64_t bd = sdesc_sw128(smem_u32(b) + p0 * C::QD_PANEL, 16, 1024);
 #pragma unroll
     for (int pp = 0; pp < 2; ++pp)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_ss(tmem + d_col, sdesc_sw128(aa + (p0 + pp) * C::KV_PANEL + kk * 32, 16, 1024),
-               sdesc_sw128(ba + (p0 + pp) * C::QD_PANEL + kk * 32, 16, 1024), C::IDESC_SDP,
-               (!first || pp || kk) ? 1u : 0u);
+        mma_ss(tmem + d_col, at(ad, pp * C::KV_PANEL + kk * 32), at(bd, pp * C::QD_PANEL + kk * 32),
+               C::IDESC_SDP, (!first || pp || kk) ? 1u : 0u);
   }
   __device__ void grads(int j, bool first) {
     const int bj = j & 1;
     const uint8_t* stg = s.st + (j % C::NST) * C::STAGE_BYTES;
-    const uint32_t q_half = smem_u32(stg) + t.dh * 2 * C::QD_PANEL;
-    const uint32_t do_half = smem_u32(stg) + (C::PANELS + t.dh * 2) * C::QD_PANEL;
-    const uint32_t ds = smem_u32(s.ds + bj * C::DS_BYTES);
+    const uint64_t qd = sdesc_sw128(smem_u32(stg) + t.dh * 2 * C::QD_PANEL, C::QD_PANEL, 1024);
+    const uint64_t dod =
+        sdesc_sw128(smem_u32(stg) + (C::PANELS + t.dh * 2) * C::QD_PANEL, C::QD_PANEL, 1024);
     // dV += P^T dO  (A = P^T in tensor memory, B = dO rows, MN-major).  The
     // P of query columns [32 w, 32 w + 32) sits at columns 32 w .. 32 w + 15 of
     // the S buffer, 8 columns per 16-query k-step.
 #pragma unroll
     for (int ks = 0; ks < C::BM / 16; ++ks)
       mma_ts(tmem + C::COL_DV, tmem + C::COL_S + bj * 64 + (ks >> 1) * 32 + (ks & 1) * 8,
-             sdesc_sw128(do_half + ks * 2048, C::QD_PANEL, 1024), C::IDESC_KV,
-             (!first || ks) ? 1u : 0u);
+             at(dod, ks * 2048), C::IDESC_KV, (!first || ks) ? 1u : 0u);
     // dK += dS^T Q  (A = dS^T in tensor memory, 16 columns after each
     // warpgroup's P^T; the shared-memory copy is for dQ)
-    (void)ds;
 #pragma unroll
     for (int ks = 0; ks < C::BM / 16; ++ks)
       mma_ts(tmem + C::COL_DK, tmem + C::COL_S + bj * 64 + (ks >> 1) * 32 + 16 + (ks & 1) * 8,
-             sdesc_sw128(q_half + ks * 2048, C::QD_PANEL, 1024), C::IDESC_KV,
-             (!first || ks) ? 1u : 0u);
+             at(qd, ks * 2048), C::IDESC_KV, (!first || ks) ? 1u : 0u);
   }
   __device__ void dq(int j) {
     const int bj = j & 1;
-    const uint32_t ka = smem_u32(s.k) + t.dh * 2 * C::KV_PANEL;
-    const uint32_t ds = smem_u32(s.ds + bj * C::DS_BYTES);
+    const uint64_t kd = sdesc_sw128(smem_u32(s.k) + t.dh * 2 * C::KV_PANEL, C::KV_PANEL, 1024);
+    const uint64_t dsd = sdesc_sw128(smem_u32(s.ds + bj * C::DS_BYTES), C::QD_PANEL, 1024);
     // dQ^T = K^T dS^T  (A = K tile read MN-major, B = dS^T MN-major)
 #pragma unroll
     for (int ks = 0; ks < C::BN / 16; ++ks)
-      mma_ss(tmem + C::COL_DQ, sdesc_sw128(ka + ks * 2048, C::KV_PANEL, 1024),
-             sdesc_sw128(ds + ks * 2048, C::QD_PANEL, 1024), C::IDESC_DQ, ks ? 1u : 0u);
+      mma_ss(tmem + C::COL_DQ, at(kd, ks * 2048), at(dsd, ks * 2048), C::IDESC_DQ, ks ? 1u : 0u);
   }
 };
 
@@ -851,8 +854,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     if (warp == C::LOAD_WARP) {
       bwd_load<D>(p, t, s, &tmK, &tmV, &tmQ, &tmO);
     } else if (warp == C::MMA_WARP || warp == C::GRAD_WARP) {
-      if (lane_id() == 0) bwd_mma<D>(p, t, s, tmem, warp - C::MMA_WARP);
-      __syncwarp();
+      bwd_mma<D>(p, t, s, tmem, warp - C::MMA_WARP);  // the whole warp; one lane issues
     }
   } else {
     if constexpr (C::DQ_WARPS) {

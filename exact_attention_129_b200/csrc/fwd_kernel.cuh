@@ -357,7 +357,7 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, c
 }
 
 // ---------------------------------------------------------------------------
-// MMA warp (one thread issues)
+// MMA warp (all lanes run it; one elected lane issues)
 // ---------------------------------------------------------------------------
 template <int D>
 struct FwdMma {
@@ -383,7 +383,7 @@ struct FwdMma {
     first_chunk = stage * C::G;
     uint32_t st = stage, ph = phase;
     for (int i = 0; i < count; ++i) {
-      if (!mbar_wait(&s.kv_full[st], ph, s.abort, p.err, ERR_FWD_MMA | 1, p.timeout_ns))
+      if (!mbar_wait_warp(&s.kv_full[st], ph, s.abort, p.err, ERR_FWD_MMA | 1, p.timeout_ns))
         return false;
       if (++st == (uint32_t)C::NSTAGE) {
         st = 0;
@@ -407,7 +407,7 @@ struct FwdMma {
   // Waiting for a panel's chunk right before its MMAs, and releasing it right
   // after, lets each wait overlap the MMAs already queued.
   __device__ bool wait_next_chunk() {
-    if (!mbar_wait(&s.kv_full[stage], phase, s.abort, p.err, ERR_FWD_MMA | 1, p.timeout_ns))
+    if (!mbar_wait_warp(&s.kv_full[stage], phase, s.abort, p.err, ERR_FWD_MMA | 1, p.timeout_ns))
       return false;
     tc_fence_after();
     return true;
@@ -486,7 +486,7 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
   FwdMma<D> m(p, s, tmem);
   const int n = t.n_blocks;
   if (n == 0) return;
-  if (!mbar_wait(&s.q_full[qt], 0, s.abort, p.err, ERR_FWD_MMA | 2, p.timeout_ns)) return;
+  if (!mbar_wait_warp(&s.q_full[qt], 0, s.abort, p.err, ERR_FWD_MMA | 2, p.timeout_ns)) return;
   tc_fence_after();
 
   if constexpr (C::DBUF) {
@@ -514,7 +514,7 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
         mma_commit(&s.s_full[2 * qt + (b ^ 1)]);
       }
       TRACE(tr + 2);
-      if (!mbar_wait(&s.p_full[2 * qt + b], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
+      if (!mbar_wait_warp(&s.p_full[2 * qt + b], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
                      p.timeout_ns))
         return;
       tc_fence_after();
@@ -538,7 +538,7 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, co
       const int slot = j & 1;
       [[maybe_unused]] const int tr = (j < 64) ? 2048 + 16 * j : -1;
       TRACE(tr);
-      if (!mbar_wait(&s.p_full[slot], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
+      if (!mbar_wait_warp(&s.p_full[slot], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
                      p.timeout_ns))
         return;
       tc_fence_after();
@@ -1135,7 +1135,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     if (lane_id() == 0) fwd_load<D>(p, t, s, &tmQ, &tmK, &tmV);
   } else {
     const int qt = warp - C::MMA_WARP;
-    if (lane_id() == 0 && t.m_base + qt * t.rows < t.sq) fwd_mma<D>(p, t, s, tmem, qt);
+    if (t.m_base + qt * t.rows < t.sq) fwd_mma<D>(p, t, s, tmem, qt);
     __syncwarp();
   }
   tc_fence_before();

@@ -275,12 +275,18 @@ __device__ __forceinline__ void tmem_st_wait() {
 // ---------------------------------------------------------------------------
 // tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in TMEM), one CTA
 // ---------------------------------------------------------------------------
+// The MMA and commit wrappers are executed by all 32 lanes of the issuing
+// warp, in warp-uniform control flow; elect.sync picks the one lane that
+// issues.  Keeping the issuing warp's code uniform lets its operands live in
+// uniform registers, so the warp needs few issue slots per MMA even while the
+// elementwise warps of its SM sub-partition keep the scheduler busy.
 // A and B from shared memory (descriptors)
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -288,17 +294,26 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// Arrive once on `bar` when every MMA this thread issued so far has completed.
+// Arrive once on `bar` when every MMA this warp issued so far has completed
+// (one elected lane commits).
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
           smem_u32(bar))
       : "memory");
+}
+// mbar_wait for every lane of a warp, with one outcome for all of them
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort, uint32_t* err,
+                                               uint32_t code, uint64_t timeout_ns) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err, code, timeout_ns));
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (SM100 layout, version 1).
