@@ -25,8 +25,13 @@
 //                  64 query rows, two dS^T tiles (128 keys x 64 queries, bf16,
 //                  128-byte swizzled: the MN-major B operand of dQ^T = K^T dS^T),
 //                  and per-block LSE/D vectors.
-//   warps: 4 elementwise warps (thread = key row = TMEM lane), 1 TMA warp,
-//          1 MMA warp.
+//   warps: 8 elementwise warps (two warpgroups, each taking 32 of a block's 64
+//          query columns; thread = key row = TMEM lane), 1 TMA warp and MMA
+//          warps that run their role warp-wide, one elected lane issuing.
+//          head_dim 64/128: two MMA warps (S and dP; dV, dK and dQ), one idle
+//          warp and a dQ warpgroup that reads dQ^T out and issues its TMA
+//          reduce-adds, 512 threads with setmaxnreg.  head_dim 256: one MMA
+//          warp; the elementwise warps add dQ with atomics (320 threads).
 #pragma once
 
 #include <cuda.h>

@@ -13,18 +13,22 @@
 //     for head_dim 64/128 (both tiles share every K/V tile brought on chip),
 //     NQ = 1 for head_dim 256 (its 128 x 256 fp32 accumulator fills half of
 //     tensor memory).
-//   * Warp roles: 4*NQ softmax warps (one warpgroup per query tile; thread i of
-//     a warpgroup owns row i of its tile), one TMA producer warp, one MMA warp.
-//   * Tensor memory (512 columns): two 128-column S slots and the O
-//     accumulators.  With NQ = 2 each tile has its own S slot; with NQ = 1 the
-//     two slots double-buffer S across consecutive K/V blocks.  P (bf16) is
-//     written back over the first 64 columns of its S slot and read from there
-//     by the P.V MMA (A operand in tensor memory).
-//   * Shared memory: the Q tiles, then a ring of 16 KB chunks holding K and V
-//     tiles in the order the MMA warp consumes them.  A K tile is D/64 chunks
-//     (one per 64-column panel, K-major); a V tile is D/64 chunks of
-//     8192/D key rows each (all D columns, MN-major operand).  Every chunk is
-//     written by TMA with the 128-byte swizzle.
+//   * Warp roles: softmax warps (head_dim 128: one warpgroup per query tile,
+//     thread i owning row i; head_dim 64 and 256: two warpgroups per tile, two
+//     threads per row, each with half of the row's key columns), one TMA
+//     producer warp, and one MMA warp per query tile.  An MMA warp runs its
+//     role in warp-uniform code and one elected lane issues each tcgen05.mma.
+//   * Tensor memory (512 columns): the S slots and the O accumulators.
+//     head_dim 64: four 96-column S slots (two per tile) and 2 x 64 O columns;
+//     head_dim 128: four 64-column slots and 2 x 128; head_dim 256: two
+//     128-column slots double-buffering S across K/V blocks and 256 O columns.
+//     P (bf16) is written back over the first BN/2 columns of its S slot and
+//     read from there by the P.V MMA (A operand in tensor memory).
+//   * Shared memory: the Q tiles, then a ring of chunks of BN rows x 128 bytes
+//     holding K and V tiles in the order the MMA warps consume them.  A K tile
+//     is D/64 chunks (one per 64-column panel, K-major); a V tile is D/64 chunks
+//     of BN*64/D key rows each (all D columns, MN-major operand).  Every chunk
+//     is written by TMA with the 128-byte swizzle.
 //   * Online softmax in the log2 domain: x = s * scale * log2(e), p = 2^(x - m).
 //     The running max m is only raised when a row's max grows by more than 8
 //     (a factor 256); until then p may exceed 1 by at most that factor, which
