@@ -273,6 +273,56 @@ def config_of(wl, l2, num_splits=1):
             "softmax_scale": wl.scale, "l2": l2, "parallelism": "replicas"}
 
 
+def fwd_lse_on_off(ea, wl, q, k, v, cu_q, cu_k, out, lse, dev, rounds=8, calls=8):
+    """The forward alone with return_lse on and off (the head_dim-64 config asks
+    that both reach the same throughput class).  After about a second of bf16
+    matmuls to bring the clocks up, each arm is a CUDA graph of `calls` forward
+    calls, replayed in rounds that alternate which arm goes first, so clock drift
+    under the power cap falls on both arms alike; medians over the rounds."""
+    a = torch.randn(8192, 8192, device=dev, dtype=torch.bfloat16)
+    t0 = time.time()
+    while time.time() - t0 < 1.0:
+        for _ in range(8):
+            torch.mm(a, a)
+        torch.cuda.synchronize()
+    del a
+    graphs = {}
+    for rl in (True, False):
+        def fwd(rl=rl):
+            ea.attn_fwd(q, k, v, cu_q, cu_k, wl.max_q, wl.max_k, scale=wl.scale,
+                        causal=wl.causal, window=wl.window, softcap=wl.softcap,
+                        return_lse=rl, out=out, lse=lse if rl else None)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(2):
+                fwd()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(calls):
+                fwd()
+        graphs[rl] = g
+    times = {True: [], False: []}
+    for r in range(rounds):
+        for rl in ((True, False) if r % 2 == 0 else (False, True)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graphs[rl].replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times[rl].append(e0.elapsed_time(e1) / calls)
+    rc, msg = ea.last_device_error()
+    if rc != 0:
+        raise RuntimeError(f"device error in the return_lse comparison: {msg}")
+    F = wl.fwd_flops()
+    on, off = statistics.median(times[True]), statistics.median(times[False])
+    return {"lse_on_tflops": F / (on * 1e-3) / 1e12, "lse_off_tflops": F / (off * 1e-3) / 1e12,
+            "off_over_on": on / off, "rounds": rounds, "calls_per_graph": calls,
+            "method": "CUDA-graph replay, alternating order, 1 s matmul warm-up, medians"}
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -415,6 +465,8 @@ def run_ours(args, wl, world, rank, local):
         "gpu_launches": 4 * args.steps,
         "library": ea.library().attn_version().decode(),
     }
+    if args.lse_ab or args.workload == "d64_mha":
+        line["fwd_lse_on_off"] = fwd_lse_on_off(ea, wl, q, k, v, cu_q, cu_k, out, lse, dev)
     return line
 
 
@@ -429,6 +481,9 @@ def main():
     ap.add_argument("--num-splits", type=int, default=1,
                     help="SplitKV parts of the forward (1: plain forward)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lse-ab", action="store_true",
+                    help="also time the forward alone with return_lse on and off "
+                         "(always done for the d64_mha workload)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
