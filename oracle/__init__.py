@@ -67,8 +67,10 @@ def _load(mutation: int = 0, out_dir: str | None = None):
                                           dp, dp, dp]
             lib.oracle_rows_ex.argtypes = [dp, dp, dp, dp, ip, ip, i, i, i, i, d, i, lg, lg, d,
                                            i, ip, lp, dp, dp, dp]
+            lib.oracle_cols_ex.argtypes = [dp, dp, dp, dp, ip, ip, i, i, i, i, d, i, lg, lg, d,
+                                           i, ip, lp, dp, dp]
             for fn in (lib.oracle_fwd, lib.oracle_bwd, lib.oracle_rows, lib.oracle_fwd_ex,
-                       lib.oracle_bwd_ex, lib.oracle_rows_ex):
+                       lib.oracle_bwd_ex, lib.oracle_rows_ex, lib.oracle_cols_ex):
                 fn.restype = ctypes.c_int
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_mutation.restype = ctypes.c_int
@@ -189,3 +191,33 @@ def rows(q, k, v, cu_q, cu_k, scale, causal, heads, row_index, dout=None, *,
     if rc != 0:
         raise ValueError(f"oracle_rows rejected its arguments (code {rc})")
     return out, lse, dq
+
+
+def cols(q, k, v, dout, cu_q, cu_k, scale, causal, kv_heads, key_index, *,
+         window=None, softcap=0.0, mutation: int = 0, lib_dir=None):
+    """dK and dV for chosen (kv head, global key row) pairs, summed over the
+    query heads of the group.
+
+    Exact at any length; a key row needs every query row's LSE and D_i, so the
+    forward statistics of the segments and heads involved are computed first
+    (their full forward).  Returns ``(dk [n,D], dv [n,D])``.
+    """
+    wl, wr, cap = _mask_args(window, softcap)
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    cu_q, cu_k = _i32(cu_q), _i32(cu_k)
+    Tq, Hq, Tk, Hkv, D, B = _dims(q, k, cu_q)
+    kv_heads = _i32(kv_heads)
+    key_index = np.ascontiguousarray(np.asarray(key_index, dtype=np.int64))
+    n = len(kv_heads)
+    assert len(key_index) == n
+    dk = np.zeros((n, D), np.float64)
+    dv = np.zeros((n, D), np.float64)
+    rc = _load(mutation, lib_dir).oracle_cols_ex(
+        _ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double),
+        _ptr(dout, ctypes.c_double), _ptr(cu_q, ctypes.c_int32), _ptr(cu_k, ctypes.c_int32),
+        B, Hq, Hkv, D, float(scale), int(bool(causal)), wl, wr, cap, n,
+        _ptr(kv_heads, ctypes.c_int32), _ptr(key_index, ctypes.c_int64),
+        _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_cols rejected its arguments (code {rc})")
+    return dk, dv

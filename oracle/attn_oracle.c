@@ -255,6 +255,52 @@ static void row_dq(const problem_t* pb, int h, long k0, long sk, const double* d
 #endif
 }
 
+/*
+ * dK_j and dV_j of one key row kr of kv head hk, summed over the query heads of
+ * its group, given every query row's LSE and D_i ([Hq][Tq]):
+ *   dV_j = sum_{h, i} P_ij dO_i,  dK_j = scale * sum_{h, i} dS_ij q_i,
+ *   dS_ij = P_ij (dO_i . v_j - D_i) (times the softcap derivative).
+ */
+static void key_grads(const problem_t* pb, const int32_t* cu_q, const int32_t* cu_k, int batch,
+                      long Tq, const double* lse_all, const double* delta_all, int hk, long kr,
+                      double* dkj, double* dvj) {
+  const int D = pb->D, Hq = pb->Hq, Hkv = pb->Hkv;
+  const double scale = pb->scale;
+  const int b = segment_of(cu_k, batch, kr);
+  const long sq = cu_q[b + 1] - cu_q[b], sk = cu_k[b + 1] - cu_k[b];
+  const long j = kr - cu_k[b];
+  for (int d = 0; d < D; ++d) { dkj[d] = 0.0; dvj[d] = 0.0; }
+  const double* kj = pb->k + ((size_t)kr * Hkv + hk) * D;
+  const double* vj = pb->v + ((size_t)kr * Hkv + hk) * D;
+  for (int h = 0; h < Hq; ++h) {
+    if (kv_head_of(h, Hq, Hkv) != hk) continue;
+    for (long i = 0; i < sq; ++i) {
+      if (!key_allowed(&pb->mk, i, j, sq, sk)) continue;
+      const long r = cu_q[b] + i;
+      const double l = lse_all[(size_t)h * Tq + r];
+      if (l == -INFINITY) continue;
+      const double* qi = pb->q + ((size_t)r * Hq + h) * D;
+      const double* doi = pb->dout + ((size_t)r * Hq + h) * D;
+      const double sij = score(&pb->mk, scale, dot(qi, kj, D));
+      const double pij = exp(sij - l);
+#if ORACLE_MUTATION == 2
+      double dsij = pij * (delta_all[(size_t)h * Tq + r] - dot(doi, vj, D));
+#else
+      double dsij = pij * (dot(doi, vj, D) - delta_all[(size_t)h * Tq + r]);
+#endif
+      dsij *= score_grad(&pb->mk, sij);
+      for (int d = 0; d < D; ++d) {
+#if ORACLE_MUTATION == 6
+        dkj[d] += scale * dsij * doi[d]; /* planted: wrong operand */
+#else
+        dkj[d] += scale * dsij * qi[d];
+#endif
+        dvj[d] += pij * doi[d];
+      }
+    }
+  }
+}
+
 static long max_seg_len(const int32_t* cu, int batch) {
   long m = 0;
   for (int b = 0; b < batch; ++b) {
@@ -373,41 +419,8 @@ int oracle_bwd_ex(const double* q, const double* k, const double* v, const doubl
   for (long u = 0; u < n_keys; ++u) {
     const int hk = (int)(u / (Tk ? Tk : 1));
     const long kr = u % Tk;
-    const int b = segment_of(cu_k, batch, kr);
-    const long sq = cu_q[b + 1] - cu_q[b], sk = cu_k[b + 1] - cu_k[b];
-    const long j = kr - cu_k[b];
-    double* dkj = dk + ((size_t)kr * Hkv + hk) * D;
-    double* dvj = dv + ((size_t)kr * Hkv + hk) * D;
-    for (int d = 0; d < D; ++d) { dkj[d] = 0.0; dvj[d] = 0.0; }
-    const double* kj = k + ((size_t)kr * Hkv + hk) * D;
-    const double* vj = v + ((size_t)kr * Hkv + hk) * D;
-    for (int h = 0; h < Hq; ++h) {
-      if (kv_head_of(h, Hq, Hkv) != hk) continue;
-      for (long i = 0; i < sq; ++i) {
-        if (!key_allowed(&pb.mk, i, j, sq, sk)) continue;
-        const long r = cu_q[b] + i;
-        const double l = lse_all[(size_t)h * Tq + r];
-        if (l == -INFINITY) continue;
-        const double* qi = q + ((size_t)r * Hq + h) * D;
-        const double* doi = dout + ((size_t)r * Hq + h) * D;
-        const double sij = score(&pb.mk, scale, dot(qi, kj, D));
-        const double pij = exp(sij - l);
-#if ORACLE_MUTATION == 2
-        double dsij = pij * (delta_all[(size_t)h * Tq + r] - dot(doi, vj, D));
-#else
-        double dsij = pij * (dot(doi, vj, D) - delta_all[(size_t)h * Tq + r]);
-#endif
-        dsij *= score_grad(&pb.mk, sij);
-        for (int d = 0; d < D; ++d) {
-#if ORACLE_MUTATION == 6
-          dkj[d] += scale * dsij * doi[d]; /* planted: wrong operand */
-#else
-          dkj[d] += scale * dsij * qi[d];
-#endif
-          dvj[d] += pij * doi[d];
-        }
-      }
-    }
+    key_grads(&pb, cu_q, cu_k, batch, Tq, lse_all, delta_all, hk, kr,
+              dk + ((size_t)kr * Hkv + hk) * D, dv + ((size_t)kr * Hkv + hk) * D);
   }
   (void)G;
   free(lse_all);
@@ -475,4 +488,71 @@ int oracle_rows(const double* q, const double* k, const double* v, const double*
                 double* dq_rows) {
   return oracle_rows_ex(q, k, v, dout, cu_q, cu_k, batch, Hq, Hkv, D, scale, causal, -1, -1,
                         0.0, n, row_head, row_index, out_rows, lse_rows, dq_rows);
+}
+
+/*
+ * Sampled key rows: for n (kv head, global key row) pairs, the row's dK and dV
+ * summed over the query heads of the group.  A key row needs the LSE and D_i
+ * of every query row that can see it, so the forward statistics of the
+ * segments and heads involved are computed first (all their rows); the result
+ * is exact at any length, at the cost of those segments' full forward.
+ * dk_rows/dv_rows are [n][D].
+ */
+int oracle_cols_ex(const double* q, const double* k, const double* v, const double* dout,
+                   const int32_t* cu_q, const int32_t* cu_k, int batch, int Hq, int Hkv,
+                   int D, double scale, int causal, long window_left, long window_right,
+                   double softcap, int n, const int32_t* key_head, const int64_t* key_index,
+                   double* dk_rows, double* dv_rows) {
+  int rc = check_args(cu_q, cu_k, batch, Hq, Hkv, D);
+  if (rc) return rc;
+  if (!q || !k || !v || !dout || !key_head || !key_index || !dk_rows || !dv_rows) return -1;
+  if (batch == 0 || n == 0) return 0;
+  const problem_t pb = {q, k, v, dout, Hq, Hkv, D, scale,
+                        {causal, window_left, window_right, softcap}};
+  const long Tq = cu_q[batch], Tk = cu_k[batch];
+  for (int t = 0; t < n; ++t)
+    if (key_head[t] < 0 || key_head[t] >= Hkv || key_index[t] < 0 || key_index[t] >= Tk)
+      return -6;
+  /* which (query head, segment) pairs the sampled keys need */
+  unsigned char* need = (unsigned char*)calloc((size_t)Hq * batch, 1);
+  double* lse_all = (double*)malloc(sizeof(double) * (size_t)Hq * (Tq ? Tq : 1));
+  double* delta_all = (double*)malloc(sizeof(double) * (size_t)Hq * (Tq ? Tq : 1));
+  if (!need || !lse_all || !delta_all) {
+    free(need); free(lse_all); free(delta_all);
+    return -5;
+  }
+  for (int t = 0; t < n; ++t) {
+    const int b = segment_of(cu_k, batch, (long)key_index[t]);
+    for (int h = 0; h < Hq; ++h)
+      if (kv_head_of(h, Hq, Hkv) == key_head[t]) need[(size_t)h * batch + b] = 1;
+  }
+  const long msk = max_seg_len(cu_k, batch);
+  const long n_rows = (long)Hq * Tq;
+#pragma omp parallel
+  {
+    double* s = (double*)malloc(sizeof(double) * (msk + 1));
+    double* p = (double*)malloc(sizeof(double) * (msk + 1));
+    double* o = (double*)malloc(sizeof(double) * D);
+#pragma omp for schedule(dynamic, 8)
+    for (long u = 0; u < n_rows; ++u) {
+      const int h = (int)(u / Tq);
+      const long r = u % Tq;
+      const int b = segment_of(cu_q, batch, r);
+      if (!need[(size_t)h * batch + b]) continue;
+      const long sq = cu_q[b + 1] - cu_q[b], sk = cu_k[b + 1] - cu_k[b];
+      double l;
+      row_forward(&pb, h, r, r - cu_q[b], cu_k[b], sq, sk, s, p, o, &l);
+      lse_all[(size_t)h * Tq + r] = l;
+      delta_all[(size_t)h * Tq + r] = row_delta(&pb, h, r, o);
+    }
+    free(s); free(p); free(o);
+  }
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int t = 0; t < n; ++t)
+    key_grads(&pb, cu_q, cu_k, batch, Tq, lse_all, delta_all, key_head[t], (long)key_index[t],
+              dk_rows + (size_t)t * D, dv_rows + (size_t)t * D);
+  free(need);
+  free(lse_all);
+  free(delta_all);
+  return 0;
 }

@@ -349,6 +349,28 @@ def check_rows_match_full(mutation=0):
     return True, "ok"
 
 
+def check_cols_match_full(mutation=0):
+    # sampled key rows (dK, dV summed over the group) equal the full backward's,
+    # with GQA, two segments, causal both ways, a window and a softcap
+    Hq, Hkv, D = 4, 2, 8
+    lq = [11, 16]
+    cu = _cu(lq)
+    T = sum(lq)
+    q, k, v, do = (_rand((T, h, D), s) for h, s in ((Hq, 40), (Hkv, 41), (Hkv, 42), (Hq, 43)))
+    keys = np.array([0, 10, 11, 26, 17, 3], np.int64)
+    khead = np.array([0, 1, 1, 0, 0, 1], np.int32)
+    for causal, window, cap in ((False, None, 0.0), (True, None, 0.0), (True, (4, 0), 0.0),
+                                (False, None, 2.5)):
+        _, dk, dv = oracle.bwd(q, k, v, do, cu, cu, 0.5, causal, window=window, softcap=cap,
+                               mutation=mutation)
+        cdk, cdv = oracle.cols(q, k, v, do, cu, cu, 0.5, causal, khead, keys, window=window,
+                               softcap=cap, mutation=mutation)
+        if not (np.array_equal(cdk, dk[keys, khead]) and np.array_equal(cdv, dv[keys, khead])):
+            return False, (f"sampled key rows differ from the full oracle "
+                           f"(causal={causal}, window={window}, softcap={cap})")
+    return True, "ok"
+
+
 def check_fully_masked_rows(mutation=0):
     # causal with s_q > s_k: the first s_q - s_k rows see no key at all
     q = _rand((6, 1, 4), 24)
@@ -501,6 +523,7 @@ ALL_CHECKS = [
     check_gradient_identities,
     check_structure,
     check_rows_match_full,
+    check_cols_match_full,
     check_fully_masked_rows,
     check_torch_reference,
     check_torch_reference_masks,

@@ -171,10 +171,46 @@ def sampled_dq_check(wl, n_rows, seed=0):
     sum_properties(wl, grads, host)
 
 
+def sampled_dkdv_check(wl, n_keys, kv_heads, segments, seed=0):
+    """dK and dV of sampled key rows against the oracle, which computes the
+    forward statistics of the chosen segments and kv groups itself."""
+    host, _, grads = run_fwd_bwd(wl, guard=False)
+    q, k, v, do = host
+    rng = np.random.default_rng(seed)
+    keys, heads = [], []
+    for b in segments:
+        k0, k1 = int(wl.cu_k[b]), int(wl.cu_k[b + 1])
+        picks = np.concatenate([rng.integers(k0, k1, size=n_keys), [k0, k1 - 1]])
+        keys.append(picks)
+        heads.append(rng.choice(np.asarray(kv_heads), size=picks.size))
+    keys, heads = np.concatenate(keys).astype(np.int64), np.concatenate(heads).astype(np.int32)
+    rdk, rdv = oracle.cols(q, k, v, do, wl.cu_q, wl.cu_k, wl.scale, wl.causal, heads, keys)
+    for got_full, ref, name in ((grads[1], rdk, "dK"), (grads[2], rdv, "dV")):
+        got = got_full[torch.from_numpy(keys), torch.from_numpy(heads)].float().cpu().numpy()
+        full_max = float(got_full.float().abs().max())
+        err = float(np.max(np.abs(got - ref)))
+        assert err <= GRAD_REL * full_max, f"{name}: {err:.3e} > {GRAD_REL} x {full_max:.3e}"
+
+
 def test_full_size_varlen_gqa_sampled():
     sampled_dq_check(si.varlen_gqa(), n_rows=256)
+
+
+def test_full_size_varlen_gqa_dkdv_sampled():
+    wl = si.varlen_gqa()
+    sampled_dkdv_check(wl, n_keys=16, kv_heads=[0, 5], segments=range(len(wl.lengths_k)))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_size_d256_mha_16k_dkdv_sampled(causal):
+    sampled_dkdv_check(si.d256_mha(16384, causal), n_keys=24, kv_heads=[3], segments=[1])
 
 
 @pytest.mark.parametrize("causal", [False, True])
 def test_full_size_gqa8_128k_sampled(causal):
     sampled_dq_check(si.d256_gqa8(131072, causal), n_rows=16)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_size_d256_mha_16k_sampled(causal):
+    sampled_dq_check(si.d256_mha(16384, causal), n_rows=32)

@@ -233,3 +233,10 @@ def test_full_size_d64_sampled():
 @pytest.mark.parametrize("causal", [False, True])
 def test_full_size_gqa8_128k_sampled(causal):
     sampled_check(si.d256_gqa8(131072, causal), n_rows=24)
+
+
+@pytest.mark.parametrize("seqlen", [16384, 131072])
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_size_d256_mha_sampled(seqlen, causal):
+    # head_dim 256 MHA, 8 heads: batch 2 at 16K and batch 1 at 128K
+    sampled_check(si.d256_mha(seqlen, causal), n_rows=48 if seqlen <= 16384 else 16)
