@@ -53,6 +53,14 @@ WORKLOADS = {
     "gqa_16k_softcap": lambda: si.gqa_softcap(16384, 50.0),
     "tiny": lambda: si.tiny(),
 }
+# the rest of the pages' shape lists: GQA head_dim 128 single segments
+# (1K/4K/32K; 16K and 64K above) and head_dim 256 MHA with 8 heads at batch
+# 8/4/2/1 x 4K/8K/16K/32K and batch 1 at 64K/128K, causal and not
+for _s in (1024, 4096, 32768):
+    WORKLOADS[f"gqa_{_s // 1024}k"] = (lambda s=_s: si.single_gqa(s))
+for _s in (4096, 8192, 32768, 65536, 131072):
+    WORKLOADS[f"d256_mha_{_s // 1024}k"] = (lambda s=_s: si.d256_mha(s, False))
+    WORKLOADS[f"d256_mha_{_s // 1024}k_causal"] = (lambda s=_s: si.d256_mha(s, True))
 
 
 def measured_peaks():
