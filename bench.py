@@ -52,6 +52,7 @@ WORKLOADS = {
     "decode_64x64k": lambda: si.decode_gqa(64, 65536),
     "gqa_16k_softcap": lambda: si.gqa_softcap(16384, 50.0),
     "tiny": lambda: si.tiny(),
+    "varlen_short": lambda: si.short_segments(128, 16384),
 }
 # the rest of the pages' shape lists: GQA head_dim 128 single segments
 # (1K/4K/32K; 16K and 64K above) and head_dim 256 MHA with 8 heads at batch
@@ -331,6 +332,40 @@ def fwd_lse_on_off(ea, wl, q, k, v, cu_q, cu_k, out, lse, dev, rounds=8, calls=8
             "method": "CUDA-graph replay, alternating order, 1 s matmul warm-up, medians"}
 
 
+def kernel_rooflines(wl, fwd_ms, bwd_main_ms, peaks, peak_kind):
+    """Per kernel: algorithmic FLOPs (the pages' convention: the backward is
+    2.5x the forward) and the bytes the method must move, over the live
+    CUDA-event time, with the roof that binds at that arithmetic intensity;
+    and the roofline object of the dominant kernel (the one that takes longer)
+    against the measured peak of its bound."""
+    F = wl.fwd_flops()
+    peak = peaks.get("bf16_tflops_sustained", 1400.0)
+    peak_bw = peaks.get("hbm_gbs", 6650.0)
+    kernels = {}
+    for kname, kflops, kbytes, kms in (("attn_fwd", F, wl.fwd_bytes(True), fwd_ms),
+                                      ("attn_bwd_main", 2.5 * F, wl.bwd_main_bytes(),
+                                       bwd_main_ms)):
+        kernels[kname] = {
+            "ms_per_launch": kms, "algorithmic_flops_per_launch": kflops,
+            "algorithmic_bytes_per_launch": kbytes,
+            "tflops": kflops / (kms * 1e-3) / 1e12, "gbs": kbytes / (kms * 1e-3) / 1e9,
+            "bound": "hbm" if kbytes / peak_bw > kflops / (peak * 1e3) else "tensor"}
+    kname = "attn_bwd_main" if bwd_main_ms >= fwd_ms else "attn_fwd"
+    kd = kernels[kname]
+    if kd["bound"] == "tensor":
+        roofline = {"bound": "tensor", "achieved": kd["tflops"], "peak": peak,
+                    "unit": "TFLOP/s", "frac": kd["tflops"] / peak,
+                    "peak_kind": f"{peak_kind} sustained bf16 matmul"}
+    else:
+        roofline = {"bound": "hbm", "achieved": kd["gbs"], "peak": peak_bw, "unit": "GB/s",
+                    "frac": kd["gbs"] / peak_bw, "peak_kind": f"{peak_kind} HBM copy"}
+    roofline.update({"kernel": kname, "traffic": None,
+                     "algorithmic_flops_per_launch": kd["algorithmic_flops_per_launch"],
+                     "algorithmic_bytes_per_launch": kd["algorithmic_bytes_per_launch"],
+                     "ms_per_launch": kd["ms_per_launch"]})
+    return kernels, roofline
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -440,19 +475,8 @@ def run_ours(args, wl, world, rank, local):
                "ms_per_step": e_ms / n_e2e}
 
     peaks, peak_kind = measured_peaks()
-    # dominant kernel: the backward main kernel (2.5x the forward FLOPs by the
-    # pages' convention) unless the forward kernel takes longer
-    if bwd_main_ms >= fwd_ms:
-        kname, kflops, kms = "attn_bwd_main", 2.5 * F, bwd_main_ms
-    else:
-        kname, kflops, kms = "attn_fwd", F, fwd_ms
-    achieved = kflops / (kms * 1e-3) / 1e12
-    peak = peaks.get("bf16_tflops_sustained", 1400.0)
-    roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_kind": f"{peak_kind} sustained bf16 matmul",
-                "traffic": recorded_traffic(kname, wl.name),
-                "algorithmic_flops_per_launch": kflops, "ms_per_launch": kms}
+    kernels, roofline = kernel_rooflines(wl, fwd_ms, bwd_main_ms, peaks, peak_kind)
+    roofline["traffic"] = recorded_traffic(roofline["kernel"], wl.name)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -468,6 +492,7 @@ def run_ours(args, wl, world, rank, local):
             "fwd": 100 * F / (fwd_ms * 1e-3) / 1e12 / peaks.get("bf16_tflops", 1590.0),
             "fwd_bwd": 100 * value / world / peaks.get("bf16_tflops", 1590.0)},
         "roofline": roofline,
+        "kernels": kernels,
         "clocks": sampler.summary(),
         "e2e": e2e,
         "gpu_launches": 4 * args.steps,

@@ -139,6 +139,20 @@ class Workload:
             pairs += int(np.maximum(0, hi - lo + 1).sum())
         return 4.0 * pairs * self.hq * self.d
 
+    def fwd_bytes(self, return_lse: bool = True) -> float:
+        """Bytes the forward must move through HBM at the least: read Q, K, V,
+        write O (bf16) and, if asked, the fp32 LSE."""
+        e = 2 * self.d  # bytes per row of one head
+        return (e * (2 * self.total_q * self.hq + 2 * self.total_k * self.hkv)
+                + (4 * self.hq * self.total_q if return_lse else 0))
+
+    def bwd_main_bytes(self) -> float:
+        """Bytes the backward's main kernel must move at the least: read Q, dO,
+        K, V, the LSE and D_i, write dK and dV.  The fp32 dQ accumulator is
+        traffic of this implementation, not of the method, and is not counted."""
+        e = 2 * self.d
+        return e * (2 * self.total_q * self.hq + 4 * self.total_k * self.hkv) + 8 * self.hq * self.total_q
+
 
 # The five problem families of the pages, by name.
 def tiny() -> Workload:
@@ -173,6 +187,16 @@ def gqa_softcap(seqlen: int = 16384, cap: float = 50.0) -> Workload:
     """The GQA head_dim-128 family, causal, with the scores soft-capped."""
     return Workload(f"gqa_s{seqlen}_hq32_hkv8_d128_causal_softcap{cap:g}", [seqlen], 32, 8, 128,
                     True, softcap=cap)
+
+
+def short_segments(seqlen: int = 128, total: int = 16384) -> Workload:
+    """The GQA head_dim-128 family as a packed batch of equal short segments
+    (total // seqlen segments of seqlen tokens, non-causal).  A 128-token
+    segment does about 100 FLOPs per byte it has to move, under the B200's
+    ridge of roughly 210, so such batches are bound by HBM, not by the
+    tensor cores."""
+    return Workload(f"varlen_short_s{seqlen}_t{total}_hq32_hkv8_d128",
+                    dense_lengths(total // seqlen, seqlen), 32, 8, 128, False)
 
 
 def d64_mha() -> Workload:

@@ -1,0 +1,34 @@
+"""Host logic of bench.py's roofline object: which roof binds a kernel at its
+arithmetic intensity, and the achieved figure against that roof."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth_inputs as si  # noqa: E402
+
+PEAKS = {"bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
+
+
+def test_long_segments_are_tensor_bound():
+    wl = si.varlen_gqa()
+    F = wl.fwd_flops()
+    fwd_ms, bwd_ms = F / 1e15 * 1e3, 2.5 * F / 0.9e15 * 1e3  # 1000 and 900 TF/s
+    k, r = bench.kernel_rooflines(wl, fwd_ms, bwd_ms, PEAKS, "measured")
+    assert k["attn_fwd"]["bound"] == "tensor" and k["attn_bwd_main"]["bound"] == "tensor"
+    assert r["kernel"] == "attn_bwd_main" and r["unit"] == "TFLOP/s"
+    assert abs(r["achieved"] - 900.0) < 1e-6 and abs(r["frac"] - 900.0 / 1400.0) < 1e-9
+
+
+def test_short_segments_forward_is_hbm_bound():
+    wl = si.short_segments(128, 16384)
+    # bytes: Q, O 32 heads and K, V 8 heads of 16384 rows x 256 bytes, LSE 4 bytes per row-head
+    assert wl.fwd_bytes(True) == 256 * (2 * 16384 * 32 + 2 * 16384 * 8) + 4 * 32 * 16384
+    assert wl.bwd_main_bytes() == 256 * (2 * 16384 * 32 + 4 * 16384 * 8) + 8 * 32 * 16384
+    fwd_ms = wl.fwd_bytes(True) / 5e12 * 1e3  # 5 TB/s
+    k, r = bench.kernel_rooflines(wl, fwd_ms, 0.5 * fwd_ms, PEAKS, "measured")
+    assert k["attn_fwd"]["bound"] == "hbm"
+    assert r["kernel"] == "attn_fwd" and r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - 5000.0) < 1e-6 and abs(r["frac"] - 5000.0 / 6500.0) < 1e-9
