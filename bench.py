@@ -495,7 +495,8 @@ def run_ours(args, wl, world, rank, local):
         "kernels": kernels,
         "clocks": sampler.summary(),
         "e2e": e2e,
-        "gpu_launches": 4 * args.steps,
+        # per step: forward (+ SplitKV combine), backward preprocess, main, dQ convert
+        "gpu_launches": (5 if args.num_splits > 1 else 4) * args.steps,
         "library": ea.library().attn_version().decode(),
     }
     if args.lse_ab or args.workload == "d64_mha":

@@ -90,13 +90,14 @@ uint64_t test_epilogue_delay_ns() {
 // Packed GQA for the forward: a CTA serves all G query heads of a key/value head
 // (tile row r = query row r / G of head r % G), so short query segments fill
 // its tiles and K/V is loaded once per group.  Used when G is a power of two in
-// [2, 16] and the longest query segment would leave a tile mostly empty
-// (max_seqlen_q < 128).  ATTN_PACK_GQA=0 / 1 forces it off / on (where G allows),
+// [2, 16] and no query segment is longer than one 128-row tile
+// (max_seqlen_q <= 128): unpacked, such a segment leaves the CTA's second query
+// tile empty.  ATTN_PACK_GQA=0 / 1 forces it off / on (where G allows),
 // read on every call so tests can exercise both.  Returns log2 G or 0.
 int pack_gqa_shift(int group, int max_seqlen_q) {
   if (group < 2 || group > 16 || (group & (group - 1)) != 0) return 0;
   const char* e = std::getenv("ATTN_PACK_GQA");
-  bool on = max_seqlen_q < 128;
+  bool on = max_seqlen_q <= 128;
   if (e && e[0] == '0') on = false;
   if (e && e[0] == '1') on = true;
   if (!on) return 0;

@@ -604,6 +604,10 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     if (tid == 0 && i < 200) TRACE(i * 8 + 0);
     const float* lse2 = s.lsd + (i % C::NST) * 128 + qc0;  // LSE in the log2 domain
     const float* dlt = s.lsd + (i % C::NST) * 128 + 64 + qc0;  // D_i
+    // lane x reads the LSE and D_i of query column x and the pair loop takes
+    // them from that lane by shuffles: a read of one value by all 32 lanes costs
+    // a shared-memory wavefront per value (measured ~2% slower at head_dim 128)
+    const float lse_lane = lse2[lane], d_lane = dlt[lane];
     uint32_t sr[32], dr[32];
     tmem_ld32x2(tmem + lane_base + C::COL_S + b * 64 + qc0, sr, tmem + lane_base + C::COL_DP + qc0,
                 dr);
@@ -618,15 +622,24 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
     uint32_t pk[16];
     uint4 dsk[4];
     const uint64_t c2 = f2_pack(c, c);
-    // most threads have all 32 of their query columns allowed: only the others
-    // run the per-element mask
-    const bool all_in = key_ok && xmin <= 0 && xmax >= 31;
+    // most warps have all 32 query columns of every lane allowed: only the
+    // others run the per-element mask.  The choice is warp-uniform, so the
+    // shuffles below are met by every lane (a lane-wise choice would split the
+    // warp across the two loop bodies and their separate shuffle sites)
+    const bool all_in = __all_sync(0xffffffffu, key_ok && xmin <= 0 && xmax >= 31);
     auto pairs = [&](auto masked_tag) {
     constexpr bool MASKED = decltype(masked_tag)::value;
 #pragma unroll
     for (int x4 = 0; x4 < 8; ++x4) {
-      const float4 l4 = reinterpret_cast<const float4*>(lse2)[x4];
-      const float4 d4 = reinterpret_cast<const float4*>(dlt)[x4];
+      float4 l4, d4;
+      l4.x = __shfl_sync(0xffffffffu, lse_lane, x4 * 4 + 0);
+      l4.y = __shfl_sync(0xffffffffu, lse_lane, x4 * 4 + 1);
+      l4.z = __shfl_sync(0xffffffffu, lse_lane, x4 * 4 + 2);
+      l4.w = __shfl_sync(0xffffffffu, lse_lane, x4 * 4 + 3);
+      d4.x = __shfl_sync(0xffffffffu, d_lane, x4 * 4 + 0);
+      d4.y = __shfl_sync(0xffffffffu, d_lane, x4 * 4 + 1);
+      d4.z = __shfl_sync(0xffffffffu, d_lane, x4 * 4 + 2);
+      d4.w = __shfl_sync(0xffffffffu, d_lane, x4 * 4 + 3);
 #pragma unroll
       for (int hp = 0; hp < 2; ++hp) {
         const int x = x4 * 4 + hp * 2;
