@@ -495,8 +495,12 @@ def run_ours(args, wl, world, rank, local):
         "kernels": kernels,
         "clocks": sampler.summary(),
         "e2e": e2e,
-        # per step: forward (+ SplitKV combine), backward preprocess, main, dQ convert
-        "gpu_launches": (5 if args.num_splits > 1 else 4) * args.steps,
+        # per step: forward (+ SplitKV combine), backward preprocess, main and,
+        # unless every key segment fits one 128-key block (dQ stored directly),
+        # the dQ convert
+        "gpu_launches": ((2 if args.num_splits > 1 else 1) + 2
+                         + (0 if wl.max_k <= 128 and os.environ.get("ATTN_BWD_DQ_DIRECT") != "0"
+                            else 1)) * args.steps,
         "library": ea.library().attn_version().decode(),
     }
     if args.lse_ab or args.workload == "d64_mha":

@@ -273,8 +273,21 @@ attn_status_t launch_bwd_main(const BwdArgs& a, const BwdParams& bp, cudaStream_
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Direct dQ stores: when every key segment fits one key block of the backward
+// (max_seqlen_k <= 128), the single CTA of each (segment, key/value head) holds
+// the complete dQ of its rows and stores it as bf16, with no fp32 accumulator
+// round trip and no postprocess launch.  ATTN_BWD_DQ_DIRECT=0 forces the
+// accumulator path (read on every call so tests can compare the two).
+bool bwd_dq_direct(int max_k) {
+  const char* e = std::getenv("ATTN_BWD_DQ_DIRECT");
+  if (e && e[0] == '0') return false;
+  return max_k <= 128;
+}
+
 template <int D>
 attn_status_t bwd_launch_d(const BwdArgs& a, cudaStream_t stream) {
+  static_assert(BwdCfg<D>::BN == 128, "direct dQ assumes 128-key blocks");
+  const bool direct = bwd_dq_direct(a.max_k);
   float* dq_acc = static_cast<float*>(a.workspace);
   float* delta = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) +
                                           bwd_align256(static_cast<size_t>(a.total_q) * a.hq * D * 4));
@@ -284,7 +297,7 @@ attn_status_t bwd_launch_d(const BwdArgs& a, cudaStream_t stream) {
     const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
     attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
         static_cast<const uint16_t*>(a.out), static_cast<const uint16_t*>(a.dout), delta, dq_acc,
-        a.total_q, a.hq);
+        direct ? static_cast<uint16_t*>(a.dq) : nullptr, a.total_q, a.hq);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   BwdParams bp;
@@ -293,6 +306,7 @@ attn_status_t bwd_launch_d(const BwdArgs& a, cudaStream_t stream) {
   bp.lse = a.lse;
   bp.delta = delta;
   bp.dq_acc = dq_acc;
+  bp.dq_out = direct ? static_cast<uint16_t*>(a.dq) : nullptr;
   bp.dk = a.dk;
   bp.dv = a.dv;
   bp.err = a.err;
@@ -316,7 +330,7 @@ attn_status_t bwd_launch_d(const BwdArgs& a, cudaStream_t stream) {
                    : launch_bwd_main<D, false, false>(a, bp, stream);
     if (st != ATTN_OK) return st;
   }
-  if (n_rh > 0) {
+  if (n_rh > 0 && !direct) {
     const long long n8 = n_rh * D / 8;
     long long blocks = (n8 + 255) / 256;
     if (blocks > 148 * 32) blocks = 148 * 32;

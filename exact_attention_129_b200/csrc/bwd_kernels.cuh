@@ -15,6 +15,13 @@
 //      is added into the fp32 accumulator with coalesced reductions;
 //   3. postprocess: dQ = scale * accumulator, rounded to bf16.
 //
+// When every key segment fits one 128-key block (max_seqlen_k <= 128), the one
+// CTA of a (segment, key/value head) sees all keys of its query rows, so its dQ
+// is already complete: it stores scale * dQ as bf16 straight into dq, the
+// preprocess zeroes dq instead of the accumulator (rows that see no key are
+// never stored), and the postprocess is not launched.  Short segments are
+// bound by HBM, and this drops the fp32 accumulator's round trip.
+//
 // Main-kernel layout for one CTA (128 keys; head_dim 256 is split into two
 // 128-wide halves handled by two CTAs, each recomputing S and dP in full):
 //   tensor memory: S^T x2 (64 cols each; per warpgroup P^T in bf16 is written
@@ -79,6 +86,10 @@ struct BwdParams {
   const float* lse;    // [Hq][Tq]
   const float* delta;  // [Hq][Tq]
   float* dq_acc;       // [Tq][Hq][D]
+  // non-null when every key segment fits one 128-key block: each CTA then holds
+  // the complete dQ of its rows and stores scale * dQ as bf16 here ([Tq][Hq][D])
+  // instead of adding into dq_acc
+  uint16_t* dq_out;
   void* dk;            // bf16 [Tk][Hkv][D]
   void* dv;
   uint32_t* err;
@@ -581,10 +592,16 @@ __device__ __forceinline__ void bwd_elem(const BwdParams& p, const BwdTile& t, c
       }
     } else {
       const int rows = min(C::BM, t.sq - m0) - qc0;
-      float* acc = p.dq_acc + (static_cast<size_t>(t.q0 + m0 + qc0) * p.nheads_q + h) * D +
-                   t.dh * C::DH + row;
+      const size_t off = (static_cast<size_t>(t.q0 + m0 + qc0) * p.nheads_q + h) * D +
+                         t.dh * C::DH + row;
       const size_t row_stride = static_cast<size_t>(p.nheads_q) * D;
-      if (d_ok) {
+      if (d_ok && p.dq_out != nullptr) {
+        // the CTA's key block is the whole key segment: store the finished rows
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          if (x < rows) p.dq_out[off + x * row_stride] = bf16_bits(__uint_as_float(r0[x]) * p.scale);
+      } else if (d_ok) {
+        float* acc = p.dq_acc + off;
 #pragma unroll
         for (int x = 0; x < 32; ++x)
           if (x < rows) atomicAdd(acc + x * row_stride, __uint_as_float(r0[x]));
@@ -785,6 +802,24 @@ __device__ __forceinline__ void bwd_dq(const BwdParams& p, const BwdTile& t, con
     __syncwarp();
     if (lane == 0) mbar_arrive(s.dq_free);
     if (!d_ok) continue;
+    if (p.dq_out != nullptr) {
+      // the CTA's key block is the whole key segment: these rows' dQ is
+      // complete, so store scale * dQ (bf16) for the rows inside the segment;
+      // lane = feature, so each store covers 64 contiguous bytes of a row
+      const int rows = min(C::BM, t.sq - m0);
+      const size_t row_stride = static_cast<size_t>(p.nheads_q) * D;
+      uint16_t* dst = p.dq_out + (static_cast<size_t>(t.q0 + m0) * p.nheads_q + h) * D +
+                      t.dh * C::DH + wq * 32 + lane;
+      // one running pointer, and r0 dead before r1 is stored: within this
+      // warpgroup's register budget
+#pragma unroll
+      for (int x = 0; x < 32; ++x, dst += row_stride)
+        if (x < rows) *dst = bf16_bits(__uint_as_float(r0[x]) * p.scale);
+#pragma unroll
+      for (int x = 0; x < 32; ++x, dst += row_stride)
+        if (x + 32 < rows) *dst = bf16_bits(__uint_as_float(r1[x]) * p.scale);
+      continue;
+    }
 #pragma unroll
     for (int hq = 0; hq < 2; ++hq) {
       float* stg = reinterpret_cast<float*>(s.dqs + (hq * (C::DH / 32) + wq) * C::DQ_WARP_BYTES);
@@ -889,13 +924,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// preprocess: D_i = dO_i . O_i, zero the dQ accumulator
+// preprocess: D_i = dO_i . O_i, zero the dQ accumulator (or, with direct dQ
+// stores, the bf16 dQ itself)
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const uint16_t* __restrict__ out,
                                                            const uint16_t* __restrict__ dout,
                                                            float* __restrict__ delta,
                                                            float* __restrict__ dq_acc,
+                                                           uint16_t* __restrict__ dq_zero,
                                                            int total_q, int hq) {
   constexpr int TPR = D / 8;  // threads per (row, head), 8 elements each
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -912,9 +949,14 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const uint16_t* __res
       acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
       acc = fmaf(__uint_as_float(av[i] & 0xffff0000u), __uint_as_float(bv[i] & 0xffff0000u), acc);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + rh * D + part * 8);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (dq_zero != nullptr) {
+      // direct dQ: rows that see no key are never stored by the main kernel
+      *reinterpret_cast<uint4*>(dq_zero + rh * D + part * 8) = make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      float4* z = reinterpret_cast<float4*>(dq_acc + rh * D + part * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, TPR);

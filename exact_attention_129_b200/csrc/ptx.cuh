@@ -394,6 +394,12 @@ __device__ __forceinline__ float rcp_approx(float x) {
 __device__ __forceinline__ float tanh_from_ex2(float x_times_k2) {
   return 1.f - 2.f * rcp_approx(ex2(x_times_k2) + 1.f);
 }
+// one float -> bf16 bits (round to nearest even)
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+  return r;
+}
 // two floats -> packed bf16x2, `lo` in the low half (round to nearest even)
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;

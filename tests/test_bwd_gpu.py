@@ -105,6 +105,38 @@ def test_causal_sq_ne_sk(d):
     check_full(wl)
 
 
+SHORT = [1, 127, 128, 0, 64, 100, 128, 33]
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_direct_dq_short_segments(d, causal):
+    # every key segment fits one 128-key block, so each CTA stores its rows'
+    # finished dQ as bf16 (no fp32 accumulator); ragged and empty segments
+    check_full(si.Workload(f"short_d{d}", SHORT, 4, 2, d, causal, seed=61))
+    # s_q > s_k under bottom-right causal: rows that see no key keep dQ = 0; GQA 8/1
+    check_full(si.Workload(f"short_sqsk_d{d}", [120, 128, 7], 8, 1, d, causal,
+                           lengths_k=[40, 128, 100], seed=62))
+    # local windows (rows whose window holds no key) and a softcap
+    check_full(si.Workload(f"short_win_d{d}", [128, 90], 4, 4, d, causal,
+                           lengths_k=[128, 20], seed=63), window=(5, 3))
+    check_full(si.Workload(f"short_cap_d{d}", [77, 128], 4, 1, d, causal, seed=64),
+               softcap=2.0)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_direct_dq_equals_accumulator_path(d, monkeypatch):
+    # with one key block per segment each dQ element has exactly one partial
+    # sum, so the direct bf16 store and the fp32 accumulator + convert agree bit
+    # for bit; dK and dV do not depend on the choice
+    wl = si.Workload(f"direct_vs_acc_d{d}", SHORT, 4, 2, d, True, seed=65)
+    _, _, direct = run_fwd_bwd(wl)
+    monkeypatch.setenv("ATTN_BWD_DQ_DIRECT", "0")
+    _, _, acc = run_fwd_bwd(wl)
+    for name, a, b in zip(("dQ", "dK", "dV"), direct, acc):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"{name} differs"
+
+
 def test_keys_without_queries_get_zero_grads():
     # a segment with keys but no query rows: its dK/dV must be written as zeros
     wl = si.Workload("no_queries", [64, 0, 32], 2, 2, 128, False, lengths_k=[64, 80, 32], seed=17)
