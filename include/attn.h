@@ -193,7 +193,10 @@ size_t attn_bwd_workspace_size(int32_t batch, int32_t total_q, int32_t nheads_q,
  *                  bytes, 256-byte aligned; its contents on entry do not
  *                  matter and are clobbered.
  * Other arguments as for attn_fwd.  Calls that share a workspace must not
- * overlap on the GPU.
+ * overlap on the GPU.  When max_seqlen_k <= 128 every key segment fits one key
+ * block, dQ is stored directly (no accumulator, two kernel launches instead of
+ * three) and the accumulator part of the workspace is left untouched; the
+ * results are the same bit for bit.
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
                        const float* lse, const void* dout,

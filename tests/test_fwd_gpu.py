@@ -174,8 +174,19 @@ def test_pack_gqa_masks_and_splits(d, monkeypatch):
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_unpacked_forced(d, causal, monkeypatch):
+    # GQA packs by default; one query head per tile stays correct when forced
+    monkeypatch.setenv("ATTN_PACK_GQA", "0")
+    check_full(si.Workload(f"unpacked_ragged_d{d}", RAGGED, 4, 2, d, causal, seed=82))
+    wl = si.Workload(f"unpacked_window_d{d}", [300, 1, 515, 129], 8, 1, d, causal,
+                     lengths_k=[400, 1, 515, 64], seed=83)
+    check_full(wl, window=(100, 37), o_tol=few_key_o_tol(wl.tensors(False)[2].float()))
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_decode_shapes_default_path(d):
-    # max_seqlen_q < 128 with G = 4: packed by default, with and without SplitKV
+    # short query segments with G = 4 (packed by default), with and without SplitKV
     wl = si.Workload(f"decode_small_d{d}", [1, 16, 100], 8, 2, d, True,
                      lengths_k=[3000, 700, 4100], seed=81)
     for splits in (1, 6):
