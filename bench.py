@@ -73,13 +73,43 @@ def measured_peaks():
     return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}, "fallback"
 
 
+def strip_c_comments(text: str) -> str:
+    """C/C++ source without its comments and with runs of blank space collapsed,
+    so that edits to comments alone do not change the source hash.  String and
+    character literals are kept as they are."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def library_source_hash():
+    """Hash of the kernel and ABI sources with comments removed: a recorded ncu
+    traffic figure stays valid across comment edits, not across code edits."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_129_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+        if not name.endswith((".cu", ".cuh", ".h")):
+            continue
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(strip_c_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

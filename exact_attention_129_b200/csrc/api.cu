@@ -624,7 +624,9 @@ extern "C" attn_status_t attn_bwd_static_scratch(
   });
   if (sc.status != cudaSuccess || sc.ptr == nullptr) return ATTN_ERR_CUDA;
   // attn_bwd's own checks and launches, with the array as its workspace; its
-  // preprocess kernel zeroes the dQ accumulator and rewrites D_i on every call
+  // preprocess kernel rewrites D_i and zeroes what must start at zero (the dQ
+  // accumulator, or dq itself when every key segment fits one key block) on
+  // every call
   return attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
                   max_seqlen_q, max_seqlen_k, nheads_q, nheads_kv, head_dim, scale, causal, dq,
                   dk, dv, sc.ptr, ATTN_STATIC_SCRATCH_BYTES, stream);

@@ -32,3 +32,11 @@ def test_short_segments_forward_is_hbm_bound():
     assert k["attn_fwd"]["bound"] == "hbm"
     assert r["kernel"] == "attn_fwd" and r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert abs(r["achieved"] - 5000.0) < 1e-6 and abs(r["frac"] - 5000.0 / 6500.0) < 1e-9
+
+
+def test_source_hash_ignores_comments_only():
+    src = 'int a = 1; // note\n/* block\n comment */ const char* s = "x//y /* z */";\n'
+    assert bench.strip_c_comments(src) == 'int a = 1; const char* s = "x//y /* z */";'
+    assert bench.strip_c_comments(src) == bench.strip_c_comments(
+        src.replace("// note", "// another note"))
+    assert bench.strip_c_comments(src) != bench.strip_c_comments(src.replace("a = 1", "a = 2"))
