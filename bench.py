@@ -268,13 +268,32 @@ def time_oracle(sample: si.Workload):
     return time.perf_counter() - t0
 
 
+def host_cpu():
+    """The host's CPU model and its logical and physical core counts."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        import psutil
+        physical = psutil.cpu_count(logical=False)
+    except Exception:
+        physical = None
+    return {"cpu_model": model, "logical_cores": os.cpu_count(), "physical_cores": physical}
+
+
 def cpu_baseline(wl, seconds=15.0):
     import oracle
     sample, desc = oracle_sample(wl, seconds)
     dt = time_oracle(sample)
     return {"value": 3.5 * sample.fwd_flops() / dt / 1e12, "unit": "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle", "sample": desc,
-            "seconds": round(dt, 2)}
+            "seconds": round(dt, 2), **host_cpu()}
 
 
 def run_reference(args, wl, world, rank):
@@ -297,7 +316,7 @@ def run_reference(args, wl, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(wl, "none (CPU)"),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
-                         "kind": "oracle", "sample": desc},
+                         "kind": "oracle", "sample": desc, **host_cpu()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
