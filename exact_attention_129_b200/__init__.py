@@ -111,6 +111,42 @@ def _check_layout(name, t, dtype):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _check_like(name, t, shape, dtype, dev):
+    """A caller-supplied buffer must match what the kernels will read or write:
+    the C ABI takes raw pointers, so a smaller tensor would be overrun."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    _check_layout(name, t, dtype)
+    if t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, expected {dev}")
+
+
+def _check_problem(q, k, v, cu_seqlens_q, cu_seqlens_k):
+    """Shapes, dtypes and devices of one attention problem (before any launch)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        if t.dim() != 3:
+            raise ValueError(f"{n} must be [tokens, heads, head_dim], got shape {tuple(t.shape)}")
+        _check_layout(n, t, torch.bfloat16)
+    if tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"v must have the shape of k {tuple(k.shape)}, got {tuple(v.shape)}")
+    if k.shape[2] != q.shape[2]:
+        raise ValueError(f"q and k head_dim differ: {q.shape[2]} and {k.shape[2]}")
+    if k.shape[1] < 1 or q.shape[1] % k.shape[1] != 0:
+        raise ValueError(f"nheads_q {q.shape[1]} is not a multiple of nheads_kv {k.shape[1]}")
+    for n, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if t.dim() != 1 or t.numel() < 2:
+            raise ValueError(f"{n} must be a 1-D int32 tensor of batch + 1 offsets")
+        _check_layout(n, t, torch.int32)
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel():
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+    for n, t in (("k", k), ("v", v), ("cu_seqlens_q", cu_seqlens_q),
+                 ("cu_seqlens_k", cu_seqlens_k)):
+        if t.device != q.device:
+            raise ValueError(f"{n} is on {t.device}, q on {q.device}")
+
+
 def _window(window):
     if window is None:
         return -1, -1
@@ -132,13 +168,12 @@ def attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
     ``softcap`` > 0 caps each scaled score at softcap * tanh(s / softcap).
     ``num_splits`` > 1 runs the SplitKV forward (key range of every query tile
     cut into that many parts, merged by LSE) in ``workspace`` (allocated if None)."""
-    _check_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k, out, lse)
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _check_layout(n, t, torch.bfloat16)
-    _check_layout("cu_seqlens_q", cu_seqlens_q, torch.int32)
-    _check_layout("cu_seqlens_k", cu_seqlens_k, torch.int32)
+    _check_problem(q, k, v, cu_seqlens_q, cu_seqlens_k)
     tq, hq, d = q.shape
     tk, hkv, _ = k.shape
+    _check_like("out", out, q.shape, torch.bfloat16, q.device)
+    _check_like("lse", lse, (hq, tq), torch.float32, q.device)
+    _check_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k, out, lse)
     if scale is None:
         scale = d ** -0.5
     if out is None:
@@ -151,6 +186,8 @@ def attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
         if workspace is None:
             workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
         _check_cuda(workspace)
+        if not workspace.is_contiguous() or workspace.device != q.device:
+            raise ValueError("workspace must be a contiguous tensor on q's device")
         rc = library().attn_fwd_split(
             _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
             cu_seqlens_q.numel() - 1, tq, tk, int(max_seqlen_q), int(max_seqlen_k), hq, hkv, d,
@@ -179,12 +216,20 @@ def attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, 
              workspace=None):
     """Backward pass; returns (dq, dk, dv) in the layouts of q, k, v.  ``causal``,
     ``window`` and ``softcap`` must match the forward call."""
-    _check_cuda(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, dq, dk, dv, workspace)
-    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
-        _check_layout(n, t, torch.bfloat16)
-    _check_layout("lse", lse, torch.float32)
+    _check_problem(q, k, v, cu_seqlens_q, cu_seqlens_k)
     tq, hq, d = q.shape
     tk, hkv, _ = k.shape
+    if out is None or lse is None or dout is None:
+        raise ValueError("out, lse and dout are required")
+    _check_like("out", out, q.shape, torch.bfloat16, q.device)
+    _check_like("dout", dout, q.shape, torch.bfloat16, q.device)
+    _check_like("lse", lse, (hq, tq), torch.float32, q.device)
+    _check_like("dq", dq, q.shape, torch.bfloat16, q.device)
+    _check_like("dk", dk, k.shape, torch.bfloat16, q.device)
+    _check_like("dv", dv, v.shape, torch.bfloat16, q.device)
+    if workspace is not None and (not workspace.is_contiguous() or workspace.device != q.device):
+        raise ValueError("workspace must be a contiguous tensor on q's device")
+    _check_cuda(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, dq, dk, dv, workspace)
     batch = cu_seqlens_q.numel() - 1
     if scale is None:
         scale = d ** -0.5

@@ -136,3 +136,68 @@ def test_watchdog_selftest_rejects_bad_timeouts(lib):
     # validated on the host, before any device call
     assert lib.attn_watchdog_selftest(0, None) == 1
     assert lib.attn_watchdog_selftest(2_000_000, None) == 1
+
+
+def _problem(tq=8, hq=4, tk=8, hkv=2, d=64):
+    import torch
+    bf = torch.bfloat16
+    q = torch.zeros(tq, hq, d, dtype=bf)
+    k = torch.zeros(tk, hkv, d, dtype=bf)
+    v = torch.zeros(tk, hkv, d, dtype=bf)
+    cq = torch.tensor([0, tq], dtype=torch.int32)
+    ck = torch.tensor([0, tk], dtype=torch.int32)
+    return q, k, v, cq, ck
+
+
+@pytest.mark.parametrize("case", ["v_shape", "head_dim", "groups", "cu_dtype", "cu_len",
+                                  "out_shape", "lse_shape", "q_rank"])
+def test_python_binding_checks_shapes_before_any_launch(case):
+    # the C ABI takes raw pointers: a buffer smaller than the problem would be
+    # overrun on the device, so the binding rejects mismatches up front (these
+    # checks run before the CUDA-device check, so they are testable on CPU)
+    import torch
+    q, k, v, cq, ck = _problem()
+    kw = {}
+    if case == "v_shape":
+        v = v[:4]
+    elif case == "head_dim":
+        k = torch.zeros(8, 2, 128, dtype=torch.bfloat16)
+        v = k.clone()
+    elif case == "groups":
+        k = torch.zeros(8, 3, 64, dtype=torch.bfloat16)
+        v = k.clone()
+    elif case == "cu_dtype":
+        cq = cq.long()
+    elif case == "cu_len":
+        ck = torch.tensor([0, 4, 8], dtype=torch.int32)
+    elif case == "out_shape":
+        kw["out"] = torch.zeros(4, 4, 64, dtype=torch.bfloat16)
+    elif case == "lse_shape":
+        kw["lse"] = torch.zeros(8, 4, dtype=torch.float32)
+    elif case == "q_rank":
+        q = q.reshape(8, 256)
+    with pytest.raises(ValueError) as e:
+        ea.attn_fwd(q, k, v, cq, ck, 8, 8, **kw)
+    assert "CUDA tensors only" not in str(e.value)
+
+
+@pytest.mark.parametrize("case", ["dout_shape", "dq_shape", "dk_dtype", "lse_dtype", "missing"])
+def test_python_binding_checks_backward_buffers(case):
+    import torch
+    q, k, v, cq, ck = _problem()
+    out, dout = torch.zeros_like(q), torch.zeros_like(q)
+    lse = torch.zeros(4, 8, dtype=torch.float32)
+    kw = {}
+    if case == "dout_shape":
+        dout = dout[:2]
+    elif case == "dq_shape":
+        kw["dq"] = torch.zeros(8, 4, 32, dtype=torch.bfloat16)
+    elif case == "dk_dtype":
+        kw["dk"] = torch.zeros(8, 2, 64, dtype=torch.float32)
+    elif case == "lse_dtype":
+        lse = lse.double()
+    elif case == "missing":
+        lse = None
+    with pytest.raises(ValueError) as e:
+        ea.attn_bwd(q, k, v, out, lse, dout, cq, ck, 8, 8, **kw)
+    assert "CUDA tensors only" not in str(e.value)
