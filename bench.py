@@ -291,9 +291,13 @@ def cpu_baseline(wl, seconds=15.0):
     import oracle
     sample, desc = oracle_sample(wl, seconds)
     dt = time_oracle(sample)
-    return {"value": 3.5 * sample.fwd_flops() / dt / 1e12, "unit": "TFLOP/s",
+    rate = 3.5 * sample.fwd_flops() / dt  # FLOP/s of the oracle on this sample
+    return {"value": rate / 1e12, "unit": "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle", "sample": desc,
-            "seconds": round(dt, 2), **host_cpu()}
+            "seconds": round(dt, 2),
+            # the whole workload at the sample's rate (extrapolated, not run)
+            "full_workload_seconds_extrapolated": round(3.5 * wl.fwd_flops() / rate, 1),
+            **host_cpu()}
 
 
 def run_reference(args, wl, world, rank):
