@@ -493,10 +493,11 @@ int oracle_rows(const double* q, const double* k, const double* v, const double*
 /*
  * Sampled key rows: for n (kv head, global key row) pairs, the row's dK and dV
  * summed over the query heads of the group.  A key row needs the LSE and D_i
- * of every query row that can see it, so the forward statistics of the
- * segments and heads involved are computed first (all their rows); the result
- * is exact at any length, at the cost of those segments' full forward.
- * dk_rows/dv_rows are [n][D].
+ * of every query row that can see it, so the forward statistics of exactly
+ * those (query head, row) pairs are computed first; the result is exact at
+ * any length.  Under a causal mask a key near the end of a long segment is
+ * seen by few rows, which keeps this cheap there; without a mask it costs the
+ * segment's full forward for the group.  dk_rows/dv_rows are [n][D].
  */
 int oracle_cols_ex(const double* q, const double* k, const double* v, const double* dout,
                    const int32_t* cu_q, const int32_t* cu_k, int batch, int Hq, int Hkv,
@@ -513,18 +514,34 @@ int oracle_cols_ex(const double* q, const double* k, const double* v, const doub
   for (int t = 0; t < n; ++t)
     if (key_head[t] < 0 || key_head[t] >= Hkv || key_index[t] < 0 || key_index[t] >= Tk)
       return -6;
-  /* which (query head, segment) pairs the sampled keys need */
-  unsigned char* need = (unsigned char*)calloc((size_t)Hq * batch, 1);
+  /* which (query head, query row) pairs the sampled keys need: a row's LSE and
+   * D_i enter key j's gradient only if key j is allowed for that row, so only
+   * those rows get their forward statistics (the others stay at LSE = -inf,
+   * which key_grads skips, as it skips rows with no allowed key) */
+  unsigned char* need = (unsigned char*)calloc((size_t)Hq * (Tq ? Tq : 1), 1);
   double* lse_all = (double*)malloc(sizeof(double) * (size_t)Hq * (Tq ? Tq : 1));
   double* delta_all = (double*)malloc(sizeof(double) * (size_t)Hq * (Tq ? Tq : 1));
   if (!need || !lse_all || !delta_all) {
     free(need); free(lse_all); free(delta_all);
     return -5;
   }
+  for (size_t u = 0; u < (size_t)Hq * Tq; ++u) { lse_all[u] = -INFINITY; delta_all[u] = 0.0; }
   for (int t = 0; t < n; ++t) {
     const int b = segment_of(cu_k, batch, (long)key_index[t]);
-    for (int h = 0; h < Hq; ++h)
-      if (kv_head_of(h, Hq, Hkv) == key_head[t]) need[(size_t)h * batch + b] = 1;
+    const long sq = cu_q[b + 1] - cu_q[b], sk = cu_k[b + 1] - cu_k[b];
+    const long j = (long)key_index[t] - cu_k[b];
+    for (int h = 0; h < Hq; ++h) {
+      if (kv_head_of(h, Hq, Hkv) != key_head[t]) continue;
+      for (long i = 0; i < sq; ++i) {
+#if ORACLE_MUTATION == 11
+        /* planted: the row on the key's diagonal is left out of the selection */
+        if (key_allowed(&pb.mk, i, j, sq, sk) && j != i + (sk - sq))
+#else
+        if (key_allowed(&pb.mk, i, j, sq, sk))
+#endif
+          need[(size_t)h * Tq + cu_q[b] + i] = 1;
+      }
+    }
   }
   const long msk = max_seg_len(cu_k, batch);
   const long n_rows = (long)Hq * Tq;
@@ -535,10 +552,10 @@ int oracle_cols_ex(const double* q, const double* k, const double* v, const doub
     double* o = (double*)malloc(sizeof(double) * D);
 #pragma omp for schedule(dynamic, 8)
     for (long u = 0; u < n_rows; ++u) {
+      if (!need[u]) continue;
       const int h = (int)(u / Tq);
       const long r = u % Tq;
       const int b = segment_of(cu_q, batch, r);
-      if (!need[(size_t)h * batch + b]) continue;
       const long sq = cu_q[b + 1] - cu_q[b], sk = cu_k[b + 1] - cu_k[b];
       double l;
       row_forward(&pb, h, r, r - cu_q[b], cu_k[b], sq, sk, s, p, o, &l);

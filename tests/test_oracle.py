@@ -87,6 +87,7 @@ MUTATIONS = {
     8: "the window's far edge is excluded",
     9: "the softcap's derivative is dropped from dS",
     10: "the softcap is applied to the unscaled score",
+    11: "the sampled-key oracle leaves the diagonal row out of its selection",
 }
 
 
@@ -107,11 +108,12 @@ def test_pins_catch_planted_mistake(mutation, tmp_path_factory):
 
 def check_in(check, mutation, lib_dir):
     # route every oracle call of the check to the mutant library in lib_dir
-    orig = (oracle.fwd, oracle.bwd, oracle.rows)
+    orig = (oracle.fwd, oracle.bwd, oracle.rows, oracle.cols)
     oracle.fwd = lambda *a, **kw: orig[0](*a, **{**kw, "lib_dir": lib_dir})
     oracle.bwd = lambda *a, **kw: orig[1](*a, **{**kw, "lib_dir": lib_dir})
     oracle.rows = lambda *a, **kw: orig[2](*a, **{**kw, "lib_dir": lib_dir})
+    oracle.cols = lambda *a, **kw: orig[3](*a, **{**kw, "lib_dir": lib_dir})
     try:
         return check(mutation=mutation)
     finally:
-        oracle.fwd, oracle.bwd, oracle.rows = orig
+        oracle.fwd, oracle.bwd, oracle.rows, oracle.cols = orig
