@@ -222,15 +222,18 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_
       !make_map(&mk, k, total_k, hkv, D, C::BN) ||
       !make_map(&mv, v, total_k, hkv, D, C::VROWS))
     return ATTN_ERR_CUDA;
+  // the limit is raised once per device; its outcome is kept, so a failure is
+  // reported on every call, not only the first
   static std::once_flag attr_once[kMaxDevices];
+  static cudaError_t attr_status[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once[dev], [&] {
-    attr_err = cudaFuncSetAttribute(attn_fwd_kernel<D, CAUSAL, SOFTCAP>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    attr_status[dev] = cudaFuncSetAttribute(attn_fwd_kernel<D, CAUSAL, SOFTCAP>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            C::SMEM_BYTES);
   });
-  if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+  if (attr_status[dev] != cudaSuccess) return ATTN_ERR_CUDA;
   const int rows_per_cta = (C::BM * C::NQ) >> p.pack_shift;
   const int m_tiles = (max_q + rows_per_cta - 1) / rows_per_cta;
   if (m_tiles == 0) return ATTN_OK;
@@ -246,15 +249,18 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_
 template <int D, bool CAUSAL, bool SOFTCAP>
 attn_status_t launch_bwd_main(const BwdArgs& a, const BwdParams& bp, cudaStream_t stream) {
   using C = BwdCfg<D>;
+  // the limit is raised once per device; its outcome is kept, so a failure is
+  // reported on every call, not only the first
   static std::once_flag attr_once[kMaxDevices];
+  static cudaError_t attr_status[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once[dev], [&] {
-    attr_err = cudaFuncSetAttribute(attn_bwd_main_kernel<D, CAUSAL, SOFTCAP>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    attr_status[dev] = cudaFuncSetAttribute(attn_bwd_main_kernel<D, CAUSAL, SOFTCAP>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            C::SMEM_BYTES);
   });
-  if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+  if (attr_status[dev] != cudaSuccess) return ATTN_ERR_CUDA;
   CUtensorMap mk, mv, mq, mo, mdq;
   if (!make_map(&mk, a.k, a.total_k, a.hkv, D, 128) ||
       !make_map(&mv, a.v, a.total_k, a.hkv, D, 128) ||

@@ -9,17 +9,30 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 import synth_inputs as si  # noqa: E402
 
-PEAKS = {"bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
+PEAKS = {"bf16_tflops": 1650.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
 
 
 def test_long_segments_are_tensor_bound():
     wl = si.varlen_gqa()
     F = wl.fwd_flops()
     fwd_ms, bwd_ms = F / 1e15 * 1e3, 2.5 * F / 0.9e15 * 1e3  # 1000 and 900 TF/s
-    k, r = bench.kernel_rooflines(wl, fwd_ms, bwd_ms, PEAKS, "measured")
+    # a short timed region: the burst peak is the roof
+    k, r = bench.kernel_rooflines(wl, fwd_ms, bwd_ms, PEAKS, "measured", 0.05)
     assert k["attn_fwd"]["bound"] == "tensor" and k["attn_bwd_main"]["bound"] == "tensor"
     assert r["kernel"] == "attn_bwd_main" and r["unit"] == "TFLOP/s"
-    assert abs(r["achieved"] - 900.0) < 1e-6 and abs(r["frac"] - 900.0 / 1400.0) < 1e-9
+    assert abs(r["achieved"] - 900.0) < 1e-6 and abs(r["frac"] - 900.0 / 1650.0) < 1e-9
+    assert r["peak"] == 1650.0 and "burst" in r["peak_kind"]
+    assert abs(r["frac_of_sustained"] - 900.0 / 1400.0) < 1e-9
+
+
+def test_long_timed_region_uses_sustained_peak():
+    wl = si.d256_gqa8(131072, False)
+    F = wl.fwd_flops()
+    k, r = bench.kernel_rooflines(wl, F / 1.3e15 * 1e3, 2.5 * F / 0.7e15 * 1e3, PEAKS,
+                                  "measured", 16.0)
+    assert r["kernel"] == "attn_bwd_main" and r["peak"] == 1400.0
+    assert "sustained" in r["peak_kind"]
+    assert abs(r["frac"] - 700.0 / 1400.0) < 1e-9 and abs(r["frac_of_burst"] - 700 / 1650) < 1e-9
 
 
 def test_short_segments_forward_is_hbm_bound():
@@ -28,7 +41,7 @@ def test_short_segments_forward_is_hbm_bound():
     assert wl.fwd_bytes(True) == 256 * (2 * 16384 * 32 + 2 * 16384 * 8) + 4 * 32 * 16384
     assert wl.bwd_main_bytes() == 256 * (2 * 16384 * 32 + 4 * 16384 * 8) + 8 * 32 * 16384
     fwd_ms = wl.fwd_bytes(True) / 5e12 * 1e3  # 5 TB/s
-    k, r = bench.kernel_rooflines(wl, fwd_ms, 0.5 * fwd_ms, PEAKS, "measured")
+    k, r = bench.kernel_rooflines(wl, fwd_ms, 0.5 * fwd_ms, PEAKS, "measured", 0.05)
     assert k["attn_fwd"]["bound"] == "hbm"
     assert r["kernel"] == "attn_fwd" and r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert abs(r["achieved"] - 5000.0) < 1e-6 and abs(r["frac"] - 5000.0 / 6500.0) < 1e-9

@@ -1,11 +1,10 @@
 """GPU parity of the backward kernels (dQ, dK, dV) against the fp64 oracle."""
-import numpy as np
 import pytest
 import torch
 
 import oracle
 import synth_inputs as si
-from tests.gpu_helpers import GRAD_REL, guarded_empty, guards_intact, to_dev
+from tests.gpu_helpers import grad_check, guarded_empty, guards_intact, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -36,25 +35,13 @@ def run_fwd_bwd(wl, guard=True, window=None, softcap=0.0):
     return host, (out, lse), (dq, dk, dv)
 
 
-def rel_err(got, ref):
-    got = np.asarray(got, np.float64)
-    ref = np.asarray(ref, np.float64)
-    scale = float(np.max(np.abs(ref))) if ref.size else 0.0
-    if scale == 0.0:
-        return float(np.max(np.abs(got))) if got.size else 0.0
-    return float(np.max(np.abs(got - ref))) / scale
-
-
 def check_full(wl, window=None, softcap=0.0):
     host, _, grads = run_fwd_bwd(wl, window=window, softcap=softcap)
     q, k, v, do = host
     ref = oracle.bwd(q, k, v, do, wl.cu_q, wl.cu_k, wl.scale, wl.causal, window=window,
                      softcap=softcap)
     for name, g, r in zip(("dQ", "dK", "dV"), grads, ref):
-        gn = g.float().cpu().numpy()
-        assert np.isfinite(gn).all(), f"{wl.name}: {name} not finite"
-        e = rel_err(gn, r)
-        assert e <= GRAD_REL, f"{wl.name}: {name} max err {e:.3e} x max|ref|"
+        grad_check(g.float().cpu().numpy(), r, f"{wl.name}: {name}")
 
 
 def test_tiny_config():
@@ -150,99 +137,5 @@ def test_autograd_function():
     out = ea.attention(qg, kg, vg, cu_q, cu_k, wl.max_q, wl.max_k, causal=True)
     out.backward(do)
     ref = oracle.bwd(*host, wl.cu_q, wl.cu_k, wl.scale, True)
-    for g, r in zip((qg.grad, kg.grad, vg.grad), ref):
-        assert rel_err(g.float().cpu().numpy(), r) <= GRAD_REL
-
-
-def sum_properties(wl, grads, host):
-    """dK summed over a segment's keys is zero (rows of dS sum to zero); dV summed
-    over the keys equals dO summed over the group's query rows (rows of P sum to
-    one).  Both hold at any size.
-
-    Error bound, from the arithmetic: each dK/dV element is an fp32 tensor-core
-    accumulation over n = G * ceil(s_q / 64) * 4 MMA k-steps, and those adds may
-    truncate, so an element can carry a relative bias of up to n * 2^-23 (one ulp
-    per add); the bias has one sign, so it adds up over the summed keys.  On top
-    of it every row is rounded to bf16 once (2^-9, independent per row)."""
-    _, _, _, do = host
-    dq, dk, dv = (g.float().cpu() for g in grads)
-    do = do.float()
-    G = wl.hq // wl.hkv
-    for b, (sq, sk) in enumerate(zip(wl.lengths_q, wl.lengths_k)):
-        if sq == 0 or sk == 0:
-            continue
-        k0, q0 = int(wl.cu_k[b]), int(wl.cu_q[b])
-        n_acc = G * ((sq + 63) // 64) * 4
-        rel = n_acc * 2.0 ** -23
-        for name, g, ref in (
-            ("dK", dk[k0:k0 + sk].double(), torch.zeros(wl.hkv, wl.d, dtype=torch.float64)),
-            ("dV", dv[k0:k0 + sk].double(),
-             do[q0:q0 + sq].double().sum(0).view(wl.hkv, G, wl.d).sum(1)),
-        ):
-            tol = rel * g.abs().sum(0) + 2.0 ** -9 * np.sqrt(sk) * float(g.abs().max()) * 4
-            err = (g.sum(0) - ref).abs()
-            assert bool((err <= tol).all()), (
-                f"segment {b}: sum {name} off by {float(err.max()):.3e} "
-                f"(bound {float(tol[err.argmax() // wl.d, err.argmax() % wl.d]):.3e})")
-
-
-def sampled_dq_check(wl, n_rows, seed=0):
-    host, _, grads = run_fwd_bwd(wl, guard=False)
-    q, k, v, do = host
-    rng = np.random.default_rng(seed)
-    T = wl.total_q
-    rows = np.concatenate([rng.integers(0, T, size=n_rows), np.array([0, 127, 128, T - 1])])
-    heads = rng.integers(0, wl.hq, size=rows.size)
-    _, _, rdq = oracle.rows(q, k, v, wl.cu_q, wl.cu_k, wl.scale, wl.causal, heads, rows, dout=do)
-    got = grads[0][torch.from_numpy(rows), torch.from_numpy(heads)].float().cpu().numpy()
-    # the bound is relative to the largest dQ of the sampled rows' heads
-    full_max = float(grads[0].float().abs().max())
-    assert np.max(np.abs(got - rdq)) <= GRAD_REL * full_max
-    for g in grads:
-        assert torch.isfinite(g.float()).all()
-    sum_properties(wl, grads, host)
-
-
-def sampled_dkdv_check(wl, n_keys, kv_heads, segments, seed=0):
-    """dK and dV of sampled key rows against the oracle, which computes the
-    forward statistics of the chosen segments and kv groups itself."""
-    host, _, grads = run_fwd_bwd(wl, guard=False)
-    q, k, v, do = host
-    rng = np.random.default_rng(seed)
-    keys, heads = [], []
-    for b in segments:
-        k0, k1 = int(wl.cu_k[b]), int(wl.cu_k[b + 1])
-        picks = np.concatenate([rng.integers(k0, k1, size=n_keys), [k0, k1 - 1]])
-        keys.append(picks)
-        heads.append(rng.choice(np.asarray(kv_heads), size=picks.size))
-    keys, heads = np.concatenate(keys).astype(np.int64), np.concatenate(heads).astype(np.int32)
-    rdk, rdv = oracle.cols(q, k, v, do, wl.cu_q, wl.cu_k, wl.scale, wl.causal, heads, keys)
-    for got_full, ref, name in ((grads[1], rdk, "dK"), (grads[2], rdv, "dV")):
-        got = got_full[torch.from_numpy(keys), torch.from_numpy(heads)].float().cpu().numpy()
-        full_max = float(got_full.float().abs().max())
-        err = float(np.max(np.abs(got - ref)))
-        assert err <= GRAD_REL * full_max, f"{name}: {err:.3e} > {GRAD_REL} x {full_max:.3e}"
-
-
-def test_full_size_varlen_gqa_sampled():
-    sampled_dq_check(si.varlen_gqa(), n_rows=256)
-
-
-def test_full_size_varlen_gqa_dkdv_sampled():
-    wl = si.varlen_gqa()
-    sampled_dkdv_check(wl, n_keys=16, kv_heads=[0, 5], segments=range(len(wl.lengths_k)))
-
-
-@pytest.mark.parametrize("causal", [False, True])
-def test_full_size_d256_mha_16k_dkdv_sampled(causal):
-    sampled_dkdv_check(si.d256_mha(16384, causal), n_keys=24, kv_heads=[3], segments=[1])
-
-
-@pytest.mark.parametrize("causal", [False, True])
-def test_full_size_gqa8_128k_sampled(causal):
-    sampled_dq_check(si.d256_gqa8(131072, causal), n_rows=16)
-
-
-@pytest.mark.parametrize("causal", [False, True])
-def test_full_size_d256_mha_16k_sampled(causal):
-    sampled_dq_check(si.d256_mha(16384, causal), n_rows=32)
+    for name, g, r in zip(("dQ", "dK", "dV"), (qg.grad, kg.grad, vg.grad), ref):
+        grad_check(g.float().cpu().numpy(), r, f"autograd: {name}")

@@ -5,8 +5,8 @@ plug-in whose host owns the allocator, a service that reserved the whole device
 for its own pool, a loop that may not call cudaMalloc/cudaFree because they can
 synchronise the device).  It keeps its scratch in one device array inside the
 library instead of a caller-provided workspace.  This test calls it through the
-C ABI twice in a row -- the second call finds the first call's leftovers in
-that shared array -- and compares both results with attn_bwd on the same
+C ABI several times in a row -- each call finds the previous call's leftovers
+in that shared array -- and compares each result with attn_bwd on the same
 inputs, within the tolerance the other backward tests use.  The file name makes
 pytest collect it last.
 """
@@ -39,9 +39,12 @@ def _call_static(lib, wl, q, k, v, out, lse, do, cu_q, cu_k, dq, dk, dv):
 def test_static_scratch_matches_attn_bwd_twice(causal):
     lib = ea.library()
     dev = torch.device("cuda", 0)
-    # two different problems, so the second call starts from the first one's leftovers
+    # different problems in a row, so each call starts from the previous one's
+    # leftovers; the third has no key segment longer than 128, so the backward
+    # stores dQ directly and only the D_i part of the array is used
     wls = [si.Workload("nsa_a", [700, 129, 64], 8, 2, 128, causal, seed=21),
-           si.Workload("nsa_b", [300, 1000], 4, 1, 64, causal, seed=22)]
+           si.Workload("nsa_b", [300, 1000], 4, 1, 64, causal, seed=22),
+           si.Workload("nsa_c", [100, 128, 37], 4, 2, 256, causal, seed=24)]
     for wl in wls:
         need = ea.bwd_workspace_size(len(wl.lengths_q), wl.total_q, wl.hq, wl.d)
         assert need <= (64 << 20)
