@@ -13,6 +13,7 @@
 
 #include "attn.h"
 #include "bwd_kernels.cuh"
+#include "bwd_pair_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace attn {
@@ -279,6 +280,45 @@ attn_status_t launch_bwd_main(const BwdArgs& a, const BwdParams& bp, cudaStream_
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// head_dim 256 without a softcap: the two-CTA kernel of bwd_pair_kernel.cuh
+// (one cluster per 128-key block, work split by role, nothing recomputed).
+// ATTN_BWD_PAIR=0 selects the head_dim-split kernel instead (read on every call,
+// so tests can compare the two).
+bool bwd_use_pair() {
+  const char* e = std::getenv("ATTN_BWD_PAIR");
+  return !(e && e[0] == '0');
+}
+
+template <bool CAUSAL>
+attn_status_t launch_bwd_pair(const BwdArgs& a, const BwdParams& bp, cudaStream_t stream) {
+  using C = PairCfg;
+  static std::once_flag attr_once[kMaxDevices];
+  static cudaError_t attr_status[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(attr_once[dev], [&] {
+    attr_status[dev] = cudaFuncSetAttribute(attn_bwd_pair_kernel<CAUSAL>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            C::SMEM_BYTES);
+  });
+  if (attr_status[dev] != cudaSuccess) return ATTN_ERR_CUDA;
+  CUtensorMap mk, mq, mo, mdq;
+  if (!make_map(&mk, a.k, a.total_k, a.hkv, C::D, C::BN) ||
+      !make_map(&mq, a.q, a.total_q, a.hq, C::D, C::BM) ||
+      !make_map(&mo, a.dout, a.total_q, a.hq, C::D, C::BM) ||
+      !make_map_f32(&mdq, bp.dq_acc, a.total_q, a.hq, C::D, 32, C::BM / 2))
+    return ATTN_ERR_CUDA;
+  const int n_blocks = (a.max_k + C::BN - 1) / C::BN;
+  if (n_blocks == 0) return ATTN_OK;
+  dim3 grid(2 * n_blocks, a.hkv, a.batch);
+  record_start(ATTN_KERNEL_BWD_MAIN, stream);
+  attn_bwd_pair_kernel<CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
+      mk, mq, mo, mdq, bp, static_cast<const uint16_t*>(a.k), static_cast<const uint16_t*>(a.v));
+  const cudaError_t e = cudaGetLastError();
+  record_stop(ATTN_KERNEL_BWD_MAIN, stream);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 // Direct dQ stores: when every key segment fits one key block of the backward
 // (max_seqlen_k <= 128), the single CTA of each (segment, key/value head) holds
 // the complete dQ of its rows and stores it as bf16, with no fp32 accumulator
@@ -331,6 +371,8 @@ attn_status_t bwd_launch_d(const BwdArgs& a, cudaStream_t stream) {
     if (a.softcap)
       st = a.upper ? launch_bwd_main<D, true, true>(a, bp, stream)
                    : launch_bwd_main<D, false, true>(a, bp, stream);
+    else if (D == 256 && bwd_use_pair())
+      st = a.upper ? launch_bwd_pair<true>(a, bp, stream) : launch_bwd_pair<false>(a, bp, stream);
     else
       st = a.upper ? launch_bwd_main<D, true, false>(a, bp, stream)
                    : launch_bwd_main<D, false, false>(a, bp, stream);
@@ -670,7 +712,8 @@ extern "C" attn_status_t attn_last_device_error(attn_stream_t stream, char* msg,
   }
   static const char* kernels[] = {"?", "fwd load", "fwd mma", "fwd softmax", "bwd preprocess",
                                   "bwd load", "bwd mma", "bwd softmax", "bwd dq convert",
-                                  "watchdog self-test"};
+                                  "watchdog self-test", "bwd pair load", "bwd pair mma",
+                                  "bwd pair elementwise", "bwd pair exchange", "bwd pair dq"};
   const uint32_t kid = (word >> 8) & 0xff;
   char buf[128];
   std::snprintf(buf, sizeof(buf), "timed-out wait in %s (wait %u)",
