@@ -322,7 +322,6 @@ __device__ __forceinline__ void bwd_load(const BwdParams& p, const BwdTile& t, c
     lsd[lane + 32] = nl2[1];
     lsd[64 + lane] = ndl[0];
     lsd[64 + lane + 32] = ndl[1];
-    if (i + 1 < t.n_iter) fetch(i + 1, nl2, ndl);
     if constexpr (C::NSPLIT == 2) {
       // own head_dim half of Q_i and dO_i (with the LSE/D vectors above); the
       // other half was issued earlier, as soon as S and dP of block i-1 ended
@@ -354,6 +353,9 @@ __device__ __forceinline__ void bwd_load(const BwdParams& p, const BwdTile& t, c
       }
     }
     ++issued;
+    // the next block's LSE and D_i, after this block's copies are issued: the
+    // warp stalls on these loads where their values are first used
+    if (i + 1 < t.n_iter) fetch(i + 1, nl2, ndl);
   }
   if (*s.abort && lane == 0) {
     // let this CTA's own copies land before its shared memory is released

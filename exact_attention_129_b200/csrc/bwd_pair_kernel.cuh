@@ -16,12 +16,14 @@
 //
 // and exchange the two bf16 tiles the other side needs: P^T goes from rank 0 to
 // rank 1 and dS^T from rank 1 to rank 0, 16 KB each per block, as shared-to-
-// shared bulk copies whose completion lands on the receiver's mbarrier.  Each
+// shared bulk copies whose completion lands on the receiver's mbarrier (the
+// copy engine moves them; stores from the elementwise warps into the peer's
+// shared memory measured 1600-2000 cycles per tile of those warps' time).  Each
 // rank issues about the same MMA work (one 256-deep N = 64 product, one
 // N = 256 gradient product and half of dQ), the minimal total.  Buffer-free
 // signals travel back as tcgen05.commit arrives on the peer's mbarrier.  The
 // K or V tile is the A operand of S or dP straight from tensor memory, so
-// shared memory holds only this rank's 128 columns of K (for dQ), three Q or dO
+// shared memory holds only this rank's 128 columns of K (for dQ), the Q or dO
 // stages and the exchange tiles.
 //
 // Per CTA: tensor memory  K or V (128 cols, bf16 pairs) | S^T or dP^T (64) |
@@ -46,6 +48,13 @@
 
 namespace attn {
 
+// Trace slots (ATTN_TRACE builds only) of block i < 200, per role:
+// elementwise 4i + {0 tile in registers, 1 P or dS computed, 2 exchange buffer
+// free, 3 tile written}; MMA A 800 + 2i + {0 issue, 1 committed}; MMA B
+// 1200 + 4i + {0 peer tile landed, 1 gradient issued, 2 dQ inputs ready,
+// 3 dQ committed}; exchange 2000 + 2i + {0 tile written, 1 copy issued};
+// dQ 2400 + 2i + {0 dQ^T ready, 1 added}; loader 2800 + 2i + {0 stage free,
+// 1 loads issued}.
 enum : uint32_t {
   ERR_BWDP_LOAD = 0x0A00,
   ERR_BWDP_MMA = 0x0B00,
@@ -59,7 +68,13 @@ struct PairCfg {
   static constexpr int KV_PANEL = BN * 128;               // 16 KB: 128 rows x 64 cols
   static constexpr int QD_PANEL = BM * 128;               // 8 KB: 64 rows x 64 cols
   static constexpr int STAGE_BYTES = PANELS * QD_PANEL;   // 32 KB: Q or dO, 64 rows x 256
-  static constexpr int NST = 3;
+  // Q stages (rank 0) and dO stages (rank 1).  Rank 0 holds a Q stage from S
+  // until dK, after the round trip of P^T and dS^T through rank 1, the longest
+  // hold in the pair; rank 1 holds a dO stage only until P^T arrives.  A
+  // fourth Q stage fits only with a single P^T send buffer, and waiting for
+  // that buffer measured slower than the third stage (676 against 752 TF/s).
+  static constexpr int NST0 = 3, NST1 = 3;
+  static constexpr int NST = NST0;
   static constexpr int X_BYTES = BN * BM * 2;             // 16 KB: 128 keys x 64 queries bf16
   static constexpr int DQ_SLOT = 32 * 32 * 4;             // 4 KB: 32 features x 32 queries
   static constexpr int OFF_KH = 0;
@@ -69,6 +84,8 @@ struct PairCfg {
   static constexpr int OFF_DQS = OFF_XB + 2 * X_BYTES;    // 2 slots per dQ warp
   static constexpr int OFF_LSD = OFF_DQS + 8 * DQ_SLOT;   // NST x 64 floats
   static constexpr int OFF_BAR = OFF_LSD + NST * BM * 4;
+  // st_empty counts the S or dP MMA, the gradient MMA and the 8 elementwise
+  // warps (which read the block's LSE' or D_i from this stage's slot).
   // kv_full, a_ready, st_full[NST], st_empty[NST], s_full, s_free, xa_full[2],
   // xa_written[2], xa_free[2], xb_full[2], xb_written[2], xb_free[2], xb_done[2],
   // dq_full, dq_free, dkv_full, drain[2]
@@ -96,6 +113,24 @@ struct PairSmem {
       *xa_free, *xb_full, *xb_written, *xb_free, *xb_done, *dq_full, *dq_free, *dkv_full, *drain;
   uint32_t* tmem_base;
   volatile int* abort;
+};
+
+__device__ __forceinline__ uint8_t* pair_stage(const PairSmem& s, int st) {
+  return s.st + st * PairCfg::STAGE_BYTES;
+}
+
+// (slot, phase parity) of a ring, advanced one block at a time
+struct Ring {
+  int slot = 0;
+  uint32_t phase = 0;
+  int n;
+  __device__ explicit Ring(int n_) : n(n_) {}
+  __device__ void next() {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
 };
 
 __device__ __forceinline__ PairSmem pair_smem(uint8_t* base) {
@@ -165,7 +200,7 @@ struct PairWait {
   uint64_t timeout_ns;
   uint32_t peer_abort;  // shared::cluster address of the peer's abort flag
   __device__ bool lane(uint64_t* bar, uint32_t parity, uint32_t code) const {
-    if (mbar_wait(bar, parity, abort, err, code, timeout_ns)) return true;
+    if (mbar_wait_cluster(bar, parity, abort, err, code, timeout_ns)) return true;
     st_cluster_u32(peer_abort, 1u);
     return false;
   }
@@ -213,33 +248,40 @@ __device__ __forceinline__ void pair_load(const BwdParams& p, const BwdTile& t, 
       }
     }
   };
+  const int nst = rank == 0 ? C::NST0 : C::NST1;
   float nv[2];
   fetch(0, nv);
   int issued = 0;
-  for (int i = 0; i < t.n_iter; ++i) {
-    const int st = i % C::NST;
-    if (i >= C::NST && !w.warp(&s.st_empty[st], ((i / C::NST) - 1) & 1, ERR_BWDP_LOAD | 1)) break;
-    float* lsd = s.lsd + st * C::BM;
+  Ring r(nst);
+  TRACE_INIT();
+  for (int i = 0; i < t.n_iter; ++i, r.next()) {
+    // the slot's previous block released it (phase parity of that use)
+    if (i >= nst && !w.warp(&s.st_empty[r.slot], r.phase ^ 1u, ERR_BWDP_LOAD | 1)) break;
+    if (lane == 0 && i < 200) TRACE(2800 + 2 * i);
+    float* lsd = s.lsd + r.slot * C::BM;
     lsd[lane] = nv[0];
     lsd[lane + 32] = nv[1];
-    if (i + 1 < t.n_iter) fetch(i + 1, nv);
     const int h = t.h0 + i / mcount;
     const int row = t.q0 + (t.m_lo + i % mcount) * C::BM;
-    uint8_t* dst = s.st + st * C::STAGE_BYTES;
+    uint8_t* dst = pair_stage(s, r.slot);
     if (lane == 0) {
-      mbar_expect_tx(&s.st_full[st], C::STAGE_BYTES);
+      mbar_expect_tx(&s.st_full[r.slot], C::STAGE_BYTES);
       for (int pn = 0; pn < C::PANELS; ++pn)
-        tma_load_3d(dst + pn * C::QD_PANEL, tmQO, &s.st_full[st], pn * 64, h, row);
+        tma_load_3d(dst + pn * C::QD_PANEL, tmQO, &s.st_full[r.slot], pn * 64, h, row);
     } else {
-      mbar_arrive(&s.st_full[st]);
+      mbar_arrive(&s.st_full[r.slot]);
     }
+    if (lane == 0 && i < 200) TRACE(2800 + 2 * i + 1);
     ++issued;
+    // the next block's LSE' or D_i, after this block's copies are issued: the
+    // warp stalls on these loads where their values are first used
+    if (i + 1 < t.n_iter) fetch(i + 1, nv);
   }
   if (*s.abort && lane == 0) {
     // let this CTA's own copies land before its shared memory is released
     mbar_wait_drain(s.kv_full, 0, 100000000ull);
-    for (int i = issued > C::NST ? issued - C::NST : 0; i < issued; ++i)
-      mbar_wait_drain(&s.st_full[i % C::NST], (i / C::NST) & 1, 100000000ull);
+    for (int i = issued > nst ? issued - nst : 0; i < issued; ++i)
+      mbar_wait_drain(&s.st_full[i % nst], (i / nst) & 1, 100000000ull);
   }
 }
 
@@ -252,24 +294,27 @@ __device__ __forceinline__ uint64_t pair_at(uint64_t desc, uint32_t bytes) {
 
 // warp 9: S^T = K Q^T (rank 0) or dP^T = V dO^T (rank 1), A from tensor memory
 __device__ __forceinline__ void pair_mma_a(const BwdTile& t, const PairSmem& s, const PairWait& w,
-                                           uint32_t tmem) {
+                                           uint32_t tmem, uint32_t rank) {
   using C = PairCfg;
   if (t.n_iter == 0) return;
+  TRACE_INIT();
   bool ok = w.warp(s.a_ready, 0, ERR_BWDP_MMA | 1);
-  for (int i = 0; ok && i < t.n_iter; ++i) {
-    const int st = i % C::NST;
-    if (!w.warp(&s.st_full[st], (i / C::NST) & 1, ERR_BWDP_MMA | 2) ||
+  Ring r(rank == 0 ? C::NST0 : C::NST1);
+  for (int i = 0; ok && i < t.n_iter; ++i, r.next()) {
+    if (!w.warp(&s.st_full[r.slot], r.phase, ERR_BWDP_MMA | 2) ||
         (i >= 1 && !w.warp(s.s_free, (i - 1) & 1, ERR_BWDP_MMA | 3))) {
       ok = false;
       break;
     }
-    const uint64_t bd = sdesc_sw128(smem_u32(s.st + st * C::STAGE_BYTES), 16, 1024);
+    if (lane_id() == 0 && i < 200) TRACE(800 + 2 * i);
+    const uint64_t bd = sdesc_sw128(smem_u32(pair_stage(s, r.slot)), 16, 1024);
 #pragma unroll
     for (int ks = 0; ks < 16; ++ks)
       mma_ts(tmem + C::COL_S, tmem + C::COL_A + ks * 8,
              pair_at(bd, (ks >> 2) * C::QD_PANEL + (ks & 3) * 32), C::IDESC_S, ks ? 1u : 0u);
     mma_commit(s.s_full);
-    mma_commit(&s.st_empty[st]);  // this warp's read of the stage
+    mma_commit(&s.st_empty[r.slot]);  // this warp's read of the stage
+    if (lane_id() == 0 && i < 200) TRACE(800 + 2 * i + 1);
   }
   if (!ok) {
     // let the MMAs already issued finish before tensor memory is released
@@ -287,15 +332,17 @@ __device__ __forceinline__ void pair_mma_b(const BwdTile& t, const PairSmem& s, 
   const int lane = lane_id();
   bool ok = w.warp(s.kv_full, 0, ERR_BWDP_MMA | 4);
   const uint64_t kd = sdesc_sw128(smem_u32(s.kh), C::KV_PANEL, 1024);
-  for (int j = 0; ok && j < t.n_iter; ++j) {
-    const int st = j % C::NST;
+  Ring r(rank == 0 ? C::NST0 : C::NST1);
+  TRACE_INIT();
+  for (int j = 0; ok && j < t.n_iter; ++j, r.next()) {
     const int b = j & 1;
-    // the tile from the peer: dS^T (rank 0) or P^T (rank 1)
+    // the tile from the peer: dS^T (rank 0) or P^T (rank 1), by bulk copy
     uint64_t* rx_full = rank == 0 ? &s.xb_full[b] : &s.xa_full[b];
     if (!w.warp(rx_full, (j >> 1) & 1, ERR_BWDP_MMA | 5)) {
       ok = false;
       break;
     }
+    if (lane == 0 && j < 200) TRACE(1200 + 4 * j);
     if (lane == 0) {
       *rx_done = j + 1;
       // arm the buffer for block j + 2 before the peer can learn it is free
@@ -306,12 +353,13 @@ __device__ __forceinline__ void pair_mma_b(const BwdTile& t, const PairSmem& s, 
     // dK += dS^T Q (rank 0) or dV += P^T dO (rank 1): A = the 128 x 64 tile
     // (K-major), B = the stage's 64 x 256 rows (MN-major), N = 256
     const uint64_t ad = sdesc_sw128(smem_u32(rx), 16, 1024);
-    const uint64_t gd = sdesc_sw128(smem_u32(s.st + st * C::STAGE_BYTES), C::QD_PANEL, 1024);
+    const uint64_t gd = sdesc_sw128(smem_u32(pair_stage(s, r.slot)), C::QD_PANEL, 1024);
 #pragma unroll
     for (int ks = 0; ks < C::BM / 16; ++ks)
       mma_ss(tmem + C::COL_G, pair_at(ad, ks * 32), pair_at(gd, ks * 2048), C::IDESC_G,
              (j > 0 || ks > 0) ? 1u : 0u);
-    if (rank == 0) mma_commit(&s.st_empty[st]);
+    mma_commit(&s.st_empty[r.slot]);  // this warp's read of the stage
+    if (lane == 0 && j < 200) TRACE(1200 + 4 * j + 1);
     // dS^T of this block: received (rank 0) or written here by the elementwise
     // warps (rank 1)
     if (rank == 1 && !w.warp(&s.xb_written[b], (j >> 1) & 1, ERR_BWDP_MMA | 6)) {
@@ -322,6 +370,7 @@ __device__ __forceinline__ void pair_mma_b(const BwdTile& t, const PairSmem& s, 
       ok = false;
       break;
     }
+    if (lane == 0 && j < 200) TRACE(1200 + 4 * j + 2);
     // dQ^T of this rank's 128 features = K^T dS^T (A = K columns MN-major,
     // B = dS^T MN-major), N = 64 queries, 128 keys deep
     const uint64_t dsd = sdesc_sw128(smem_u32(s.xb + b * C::X_BYTES), C::QD_PANEL, 1024);
@@ -334,13 +383,12 @@ __device__ __forceinline__ void pair_mma_b(const BwdTile& t, const PairSmem& s, 
       // rank 1 may send dS^T of block j + 2 into XB[b]
       mma_commit_to(&s.xb_free[b], peer_mask);
     } else {
-      // the elementwise warps read D_i of this block before dS^T was written:
-      // now the stage (dO rows and D_i) is free; XB[b] is read by dQ
-      mma_commit(&s.st_empty[st]);
-      mma_commit(&s.xb_done[b]);
-      // rank 0 may send P^T of block j + 2 into XA[b]
+      mma_commit(&s.xb_done[b]);  // XB[b] read by dQ
+      // rank 0 may store P^T of block j + 2 into XA[b]: dV has read it, and
+      // the elementwise warps read it before they wrote dS^T
       mma_commit_to(&s.xa_free[b], peer_mask);
     }
+    if (lane == 0 && j < 200) TRACE(1200 + 4 * j + 3);
   }
   if (ok) {
     mma_commit(s.dkv_full);
@@ -351,38 +399,41 @@ __device__ __forceinline__ void pair_mma_b(const BwdTile& t, const PairSmem& s, 
 }
 
 // ---------------------------------------------------------------------------
-// exchange warp: sends this rank's tile of each block to the peer; at the end
-// it waits for the peer's last free signals, so no arrive is still on its way
-// into this CTA when the cluster exits
+// exchange warp: sends this rank's tile of each block to the peer.  At the end
+// it waits for the peer's last release signals, so no arrive is still on its
+// way into this CTA when the cluster exits
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void pair_xchg(const BwdTile& t, const PairSmem& s, const PairWait& w,
                                           uint32_t rank, const volatile int* rx_done) {
   using C = PairCfg;
   if (t.n_iter == 0) return;
-  const uint32_t peer = rank ^ 1u;
   const int lane = lane_id();
+  int sent = 0;
+  TRACE_INIT();
   uint8_t* tx = rank == 0 ? s.xa : s.xb;
   uint64_t* tx_written = rank == 0 ? s.xa_written : s.xb_written;
-  uint64_t* tx_full = rank == 0 ? s.xa_full : s.xb_full;  // the peer's receive barriers
-  uint64_t* tx_free = rank == 0 ? s.xa_free : s.xb_free;  // the peer's release signals
-  int sent = 0;
+  const uint32_t peer = rank ^ 1u;
+  const uint32_t peer_tx = mapa_shared(smem_u32(tx), peer);
+  const uint32_t peer_bar = mapa_shared(smem_u32(rank == 0 ? s.xa_full : s.xb_full), peer);
   for (int i = 0; i < t.n_iter; ++i) {
     const int b = i & 1;
     if (!w.warp(&tx_written[b], (i >> 1) & 1, ERR_BWDP_XCHG | 1)) break;
+    if (lane == 0 && i < 200) TRACE(2000 + 2 * i);
     if (lane == 0)
-      bulk_copy_to_peer(mapa_shared(smem_u32(tx + b * C::X_BYTES), peer), tx + b * C::X_BYTES,
-                        C::X_BYTES, mapa_shared(smem_u32(&tx_full[b]), peer));
+      bulk_copy_to_peer(peer_tx + b * C::X_BYTES, tx + b * C::X_BYTES, C::X_BYTES, peer_bar + b * 8);
     __syncwarp();
+    if (lane == 0 && i < 200) TRACE(2000 + 2 * i + 1);
     ++sent;
   }
   if (lane == 0) {
     // the peer releases each block it received; the elementwise warps consumed
-    // the releases up to block sent - 3, these are the rest
+    // the releases up to block n_iter - 3, these are the rest
+    uint64_t* tx_free = rank == 0 ? s.xa_free : s.xb_free;
+    const uint64_t bound = *s.abort ? 1000000ull : 2000000000ull;
     for (int j = sent > 2 ? sent - 2 : 0; j < sent; ++j)
-      if (!mbar_wait_drain(&tx_free[j & 1], (j >> 1) & 1, *s.abort ? 1000000ull : 2000000000ull))
-        break;
+      if (!mbar_wait_drain(&tx_free[j & 1], (j >> 1) & 1, bound)) break;
     if (*s.abort) {
-      // copies from the peer that may still be landing here
+      // tiles from the peer that may still be landing here
       uint64_t* rx_full = rank == 0 ? s.xb_full : s.xa_full;
       for (int j = *rx_done; j < t.n_iter; ++j)
         if (!mbar_wait_drain(&rx_full[j & 1], (j >> 1) & 1, 1000000ull)) break;
@@ -438,24 +489,29 @@ __device__ __forceinline__ void pair_elem(const BwdParams& p, const BwdTile& t, 
   }
   const float c = p.scale_log2;
   const int causal_off = t.sk - t.sq;
+  TRACE_INIT();
   uint8_t* xrow_a = s.xa + row * 128;
   uint8_t* xrow_b = s.xb + row * 128;
-  for (int i = 0; i < t.n_iter && ok; ++i) {
-    const int st = i % C::NST;
+  Ring r(rank == 0 ? C::NST0 : C::NST1);
+  for (int i = 0; i < t.n_iter && ok; ++i, r.next()) {
     const int b = i & 1;
     const int m0 = (t.m_lo + i % mcount) * C::BM;
-    if (!w.warp(&s.st_full[st], (i / C::NST) & 1, ERR_BWDP_ELEM | 1) ||
+    if (!w.warp(&s.st_full[r.slot], r.phase, ERR_BWDP_ELEM | 1) ||
         !w.warp(s.s_full, i & 1, ERR_BWDP_ELEM | 2)) {
       ok = false;
       break;
     }
-    // lane x holds the LSE' (rank 0) or D_i (rank 1) of query column qc0 + x
-    const float v_lane = s.lsd[st * C::BM + qc0 + lane];
+    // lane x holds the LSE' (rank 0) or D_i (rank 1) of query column qc0 + x;
+    // the warp's last read of the stage slot
+    const float v_lane = s.lsd[r.slot * C::BM + qc0 + lane];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.st_empty[r.slot]);
     uint32_t sr[32];
     tmem_ld32(tmem + lane_base + C::COL_S + qc0, sr);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(s.s_free);
+    if (tid == 0 && i < 200) TRACE(4 * i);
     uint4 out[4];
     if (rank == 0) {
       // P^T = 2^(S^T c - LSE') with the masks
@@ -489,6 +545,7 @@ __device__ __forceinline__ void pair_elem(const BwdParams& p, const BwdTile& t, 
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch)
         out[ch] = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+      if (tid == 0 && i < 200) TRACE(4 * i + 1);
       // XA[b] held P^T of block i - 2 until rank 1 released it
       if (i >= 2 && !w.warp(&s.xa_free[b], ((i - 2) >> 1) & 1, ERR_BWDP_ELEM | 3)) {
         ok = false;
@@ -524,6 +581,7 @@ __device__ __forceinline__ void pair_elem(const BwdParams& p, const BwdTile& t, 
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch)
         out[ch] = make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+      if (tid == 0 && i < 200) TRACE(4 * i + 1);
       // XB[b] held dS^T of block i - 2: read by this CTA's dQ and by the copy
       // to rank 0, which released it after its own MMAs
       if (i >= 2 && (!w.warp(&s.xb_done[b], ((i - 2) >> 1) & 1, ERR_BWDP_ELEM | 5) ||
@@ -533,8 +591,8 @@ __device__ __forceinline__ void pair_elem(const BwdParams& p, const BwdTile& t, 
       }
     }
     // the 128 B row of this key (64 queries, 128-byte swizzle): the K-major A
-    // operand of the peer's or this CTA's gradient product and the MN-major B
-    // operand of dQ^T
+    // operand of the gradient product and the MN-major B operand of dQ^T
+    if (tid == 0 && i < 200) TRACE(4 * i + 2);
     uint8_t* xrow = (rank == 0 ? xrow_a : xrow_b) + b * C::X_BYTES;
 #pragma unroll
     for (int ch = 0; ch < 4; ++ch)
@@ -542,6 +600,7 @@ __device__ __forceinline__ void pair_elem(const BwdParams& p, const BwdTile& t, 
     fence_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(rank == 0 ? &s.xa_written[b] : &s.xb_written[b]);
+    if (tid == 0 && i < 200) TRACE(4 * i + 3);
   }
   if (ok && t.n_iter > 0) ok = w.warp(s.dkv_full, 0, ERR_BWDP_ELEM | 7);
   if (!ok) return;
@@ -590,8 +649,10 @@ __device__ __forceinline__ void pair_dq(const BwdParams& p, const BwdTile& t, co
   const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
   const int mcount = t.m_hi - t.m_lo;
   const int feat0 = static_cast<int>(rank) * 128 + wq * 32;
+  TRACE_INIT();
   for (int j = 0; j < t.n_iter; ++j) {
     if (!w.warp(s.dq_full, j & 1, ERR_BWDP_DQ | 1)) break;
+    if (wq == 0 && lane == 0 && j < 200) TRACE(2400 + 2 * j);
     const int h = t.h0 + j / mcount;
     const int m0 = (t.m_lo + j % mcount) * C::BM;
     uint32_t r0[32], r1[32];
@@ -626,6 +687,7 @@ __device__ __forceinline__ void pair_dq(const BwdParams& p, const BwdTile& t, co
         bulk_commit();
       }
     }
+    if (wq == 0 && lane == 0 && j < 200) TRACE(2400 + 2 * j + 1);
   }
   if (lane == 0) bulk_wait0();
 }
@@ -653,7 +715,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     mbar_init(s.a_ready, 8);
     for (int i = 0; i < C::NST; ++i) {
       mbar_init(&s.st_full[i], 32);
-      mbar_init(&s.st_empty[i], 2);
+      mbar_init(&s.st_empty[i], 2 + 8);
     }
     mbar_init(s.s_full, 1);
     mbar_init(s.s_free, 8);
@@ -704,7 +766,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     if (warp == C::LOAD_WARP)
       pair_load(p, t, s, w, rank, &tmK, rank == 0 ? &tmQ : &tmO);
     else if (warp == C::MMA_A_WARP)
-      pair_mma_a(t, s, w, tmem);
+      pair_mma_a(t, s, w, tmem, rank);
     else if (warp == C::MMA_B_WARP)
       pair_mma_b(t, s, w, tmem, rank, rx_done);
     else

@@ -75,6 +75,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// try_wait with acquire at cluster scope: for barriers that another CTA of the
+// cluster completes (its stores or copies into this CTA, its releases)
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort, uint32_t* err,
+                                                  uint32_t code, uint64_t timeout_ns) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      *abort = 1;
+      if (err) atomicCAS(err, 0u, code);
+      return false;
+    }
+  }
+}
+
 // Bounded wait that ignores the abort flag: used on the way out of a CTA that
 // gave up, to let its own TMA copies land before the shared memory is released.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
