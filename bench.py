@@ -66,6 +66,11 @@ for _s in (1024, 4096, 32768):
 for _s in (4096, 8192, 32768, 65536, 131072):
     WORKLOADS[f"d256_mha_{_s // 1024}k"] = (lambda s=_s: si.d256_mha(s, False))
     WORKLOADS[f"d256_mha_{_s // 1024}k_causal"] = (lambda s=_s: si.d256_mha(s, True))
+# head_dim 256 GQA ratio 8 at the shorter lengths of the same shape list (one
+# sequence each; the stated problem is the 128K one above)
+for _s in (4096, 8192, 16384, 32768, 65536):
+    WORKLOADS[f"d256_gqa8_{_s // 1024}k"] = (lambda s=_s: si.d256_gqa8(s, False))
+    WORKLOADS[f"d256_gqa8_{_s // 1024}k_causal"] = (lambda s=_s: si.d256_gqa8(s, True))
 
 
 def measured_peaks():

@@ -26,7 +26,10 @@ __all__ = ["attn_fwd", "attn_bwd", "attention", "bwd_workspace_size", "fwd_split
            "set_timing_events", "KERNEL_FWD", "KERNEL_BWD_MAIN",
            "library", "LIB_PATH", "AttnError", "STATUS"]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
+# ATTN_LIBRARY names another build of the same library (a variant built with
+# exact_attention_129_b200.build.build(out=..., extra=...)); default: the in-tree build
+LIB_PATH = os.environ.get("ATTN_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED",
           3: "ATTN_ERR_CUDA", 4: "ATTN_ERR_TIMEOUT", 5: "ATTN_ERR_SCRATCH_TOO_SMALL"}
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_fwd_ex", "attn_bwd_ex", "attn_fwd_split",

@@ -33,10 +33,13 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs() if os.path.exists(f))
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra=(), out: str | None = None) -> str:
+    """Compile libattn.so (or, with ``out``, a variant with the extra nvcc
+    arguments ``extra``, e.g. ``-DATTN_FWD_POLY_PAIRS=2``, at that path)."""
+    target = out or LIB
+    if out is None and not force and up_to_date():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = target + f".tmp{os.getpid()}"
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
            "-std=c++17", "-shared", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
            "--expt-relaxed-constexpr", "-Xptxas", "-v" if verbose else "-O3",
@@ -47,8 +50,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         raise RuntimeError("nvcc failed building libattn.so")
     if verbose:
         sys.stderr.write(r.stdout + r.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

@@ -762,4 +762,10 @@ extern "C" attn_status_t attn_watchdog_selftest(int32_t timeout_us, attn_stream_
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-extern "C" const char* attn_version(void) { return "exact_attention_b200 0.1 sm_100a"; }
+#define ATTN_STR2(x) #x
+#define ATTN_STR(x) ATTN_STR2(x)
+// the build's forward exp2 setting is part of the string, so a caller can see
+// which variant it loaded
+extern "C" const char* attn_version(void) {
+  return "exact_attention_b200 0.2 sm_100a fwd_poly_pairs=" ATTN_STR(ATTN_FWD_POLY_PAIRS);
+}
