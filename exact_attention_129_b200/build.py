@@ -15,7 +15,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libattn.so")
 SOURCES = ["api.cu"]
-HEADERS = ["ptx.cuh", "fwd_kernel.cuh", "bwd_kernels.cuh", "bwd_pair_kernel.cuh"]
+HEADERS = ["ptx.cuh", "fwd_kernel.cuh", "fwd_pair_kernel.cuh", "bwd_kernels.cuh",
+           "bwd_pair_kernel.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 

@@ -15,6 +15,7 @@
 #include "bwd_kernels.cuh"
 #include "bwd_pair_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "fwd_pair_kernel.cuh"
 
 namespace attn {
 
@@ -209,10 +210,57 @@ attn_status_t mask_args(int32_t causal, int32_t window_left, int32_t window_righ
   return ATTN_OK;
 }
 
+// head_dim 128 without softcap or SplitKV can run on the two-CTA kernel of
+// fwd_pair_kernel.cuh (M = 256 MMAs over a CTA pair, 128-key blocks) when
+// ATTN_FWD_PAIR=1 (read on every call, so tests can compare the two).  The
+// one-CTA kernel is the default: both are bound by the softmax warps' exps,
+// which cost the same per score in either, and the one-CTA kernel measured
+// faster.
+bool fwd_use_pair() {
+  const char* e = std::getenv("ATTN_FWD_PAIR");
+  return e && e[0] == '1';
+}
+
+template <bool CAUSAL>
+attn_status_t launch_fwd_pair(const void* q, const void* k, const void* v, int total_q,
+                              int total_k, int hkv, const FwdParams& p, int batch, int hq,
+                              int max_q, cudaStream_t stream) {
+  using C = FwdPairCfg;
+  CUtensorMap mq, mk, mv;
+  const int g = 1 << p.pack_shift;
+  if (!make_map(&mq, q, total_q, hq, C::D, C::BM / g, g) ||
+      !make_map(&mk, k, total_k, hkv, C::D, C::BN / 2) ||
+      !make_map(&mv, v, total_k, hkv, C::D, C::BN))
+    return ATTN_ERR_CUDA;
+  static std::once_flag attr_once[kMaxDevices];
+  static cudaError_t attr_status[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(attr_once[dev], [&] {
+    attr_status[dev] = cudaFuncSetAttribute(attn_fwd_pair_kernel<CAUSAL>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            C::SMEM_BYTES);
+  });
+  if (attr_status[dev] != cudaSuccess) return ATTN_ERR_CUDA;
+  const int rows_per_pair = (2 * C::BM) >> p.pack_shift;
+  const int pairs = (max_q + rows_per_pair - 1) / rows_per_pair;
+  if (pairs == 0) return ATTN_OK;
+  dim3 grid(2 * pairs, p.pack_shift > 0 ? hkv : hq, batch);
+  record_start(ATTN_KERNEL_FWD, stream);
+  attn_fwd_pair_kernel<CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  const cudaError_t e = cudaGetLastError();
+  record_stop(ATTN_KERNEL_FWD, stream);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 template <int D, bool CAUSAL, bool SOFTCAP>
 attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_q, int total_k,
                          int hkv, const FwdParams& p, int batch, int hq, int max_q,
                          cudaStream_t stream) {
+  if constexpr (D == 128 && !SOFTCAP) {
+    if (p.num_splits == 1 && fwd_use_pair())
+      return launch_fwd_pair<CAUSAL>(q, k, v, total_q, total_k, hkv, p, batch, hq, max_q, stream);
+  }
   using C = FwdCfg<D>;
   // Q: one 128-row box per 64-column panel; K: one BN-row box per panel;
   // V: VROWS rows per box, all panels of a chunk together
@@ -713,7 +761,8 @@ extern "C" attn_status_t attn_last_device_error(attn_stream_t stream, char* msg,
   static const char* kernels[] = {"?", "fwd load", "fwd mma", "fwd softmax", "bwd preprocess",
                                   "bwd load", "bwd mma", "bwd softmax", "bwd dq convert",
                                   "watchdog self-test", "bwd pair load", "bwd pair mma",
-                                  "bwd pair elementwise", "bwd pair exchange", "bwd pair dq"};
+                                  "bwd pair elementwise", "bwd pair exchange", "bwd pair dq",
+                                  "fwd pair load", "fwd pair mma", "fwd pair softmax"};
   const uint32_t kid = (word >> 8) & 0xff;
   char buf[128];
   std::snprintf(buf, sizeof(buf), "timed-out wait in %s (wait %u)",

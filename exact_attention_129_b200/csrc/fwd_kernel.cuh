@@ -14,8 +14,8 @@
 //     NQ = 1 for head_dim 256 (its 128 x 256 fp32 accumulator fills half of
 //     tensor memory).
 //   * Warp roles: softmax warps (head_dim 128: one warpgroup per query tile,
-//     thread i owning row i; head_dim 64 and 256: two warpgroups per tile, two
-//     threads per row, each with half of the row's key columns), one TMA
+//     thread i owning row i; head_dim 64 and 256: two warpgroups per tile,
+//     each warp over 16 whole rows with four threads per row), one TMA
 //     producer warp, and one MMA warp per query tile.  An MMA warp runs its
 //     role in warp-uniform code and one elected lane issues each tcgen05.mma.
 //   * Tensor memory (512 columns): the S slots and the O accumulators.
@@ -135,9 +135,10 @@ struct FwdCfg {
   // on and releases one barrier.  head_dim 256: one chunk per stage.
   static constexpr int G = DBUF ? 2 * PANELS : 1;
   static constexpr int NSTAGE = NSLOT / G;
-  // head_dim 64 and 256: two threads per query row, each with half of the row's
-  // key columns, so more softmax warps share each SM sub-partition and keep its
-  // exp unit busy (one warp alone cannot: its exps are latency-bound)
+  // head_dim 64 and 256: eight softmax warps per tile, each over 16 whole rows
+  // (16-lane tensor-memory accesses), so more softmax warps share each SM
+  // sub-partition and keep its exp unit busy (one warp alone cannot: its exps
+  // are latency-bound)
   static constexpr int ROW_SPLIT = (D == 128) ? 1 : 2;
   static constexpr int SOFTMAX_WARPS = 4 * NQ * ROW_SPLIT;
   static constexpr int LOAD_WARP = SOFTMAX_WARPS;
@@ -153,10 +154,7 @@ struct FwdCfg {
   // o_ready[NQ] o_final[NQ]
   static constexpr int NBAR = NQ + 2 * NSTAGE + 2 * NSS + 2 * NQ;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // row-split exchange: [tile][block parity][half][row] fp32
-  static constexpr int OFF_XCH = OFF_MISC + 64;
-  static constexpr int XCH_BYTES = (ROW_SPLIT == 2) ? NQ * 2 * 2 * BM * 4 : 0;
-  static constexpr int SMEM_BYTES = OFF_XCH + XCH_BYTES + 1024;  // + alignment slack
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -177,7 +175,6 @@ struct FwdSmem {
   uint64_t* o_final;  // one phase per CTA: the tile's last P.V is done
   uint32_t* tmem_base;
   volatile int* abort;
-  float* xch;
 };
 
 template <int D>
@@ -196,7 +193,6 @@ __device__ __forceinline__ FwdSmem fwd_smem(uint8_t* base) {
   s.o_final = s.o_ready + C::NQ;
   s.tmem_base = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
   s.abort = reinterpret_cast<volatile int*>(base + C::OFF_MISC + 4);
-  s.xch = reinterpret_cast<float*>(base + C::OFF_XCH);
   return s;
 }
 
@@ -834,151 +830,158 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
 }
 
 // ---------------------------------------------------------------------------
-// softmax with two threads per query row (head_dim 64, 96-key blocks): thread
-// (row, hf) owns keys [32 hf, 32 hf + 32) and [64 + 16 hf, 80 + 16 hf) of
-// every block (so every tensor-memory access is aligned to its width) and the
-// O columns [hf D/2, (hf + 1) D/2).  Both threads of a row sit in warps of the same TMEM
-// lane quadrant; per block they exchange their partial row max through shared
-// memory and a named barrier of those two warps, and at the end their partial
-// row sums.  Every thread meets every barrier, also after a timed-out wait
-// (then it only plays the barriers), so its partner never blocks for good.
+// softmax with 16 rows per warp (head_dim 64, 96-key blocks; head_dim 256,
+// 128-key blocks): eight warps per query tile, warp (quadrant, lane half lh)
+// serving the 16 tile rows [32 quad + 16 lh, +16) over all keys of every
+// block, through 16-lane tensor-memory accesses.  Thread t holds rows
+// rt0 = first + t/4 and rt0 + 8 and, of every 8 keys of the block, keys
+// 2(t%4) and 2(t%4) + 1: score register 4x + 2r + e is row rt0 + 8r, key
+// 8x + 2(t%4) + e.  The four threads of a row combine its max and sum with two
+// shuffles, so no warp waits for another warp's scores and the warps that
+// share an SM sub-partition drift apart, keeping its exp unit busy.
 // ---------------------------------------------------------------------------
 template <int D, bool CAUSAL, bool SOFTCAP>
-__device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdTile& t,
-                                                  const FwdSmem& s, uint32_t tmem, int qt,
-                                                  int hf) {
+__device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const FwdTile& t,
+                                                   const FwdSmem& s, uint32_t tmem, int qt,
+                                                   int lh) {
   using C = FwdCfg<D>;
-  // key columns per thread and block: 96-key blocks (head_dim 64) 32 + 16,
-  // 128-key blocks (head_dim 256) 64
-  constexpr int NC = C::BN / 2;
-  constexpr int OC = D / 2;      // O columns per thread
-  static_assert((C::BN == 96 || C::BN == 128) && OC % 32 == 0, "row split layout");
-  // segment-local key (within the block) of this thread's score column i
-  auto key_of = [&](int i) {
-    if constexpr (C::BN == 96) return i < 32 ? hf * 32 + i : 64 + hf * 16 + (i - 32);
-    else return hf * 64 + i;
-  };
-  const int quad = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant
+  constexpr int NX = C::BN / 8;  // 8-key groups per block: 12 or 16
+  static_assert((C::BN == 96 || C::BN == 128) && D % 64 == 0, "16-row layout");
+  const int quad = (threadIdx.x >> 5) & 3;
   const int lane = lane_id();
-  const int row_in_tile = quad * 32 + lane;
-  const int row = t.m_base + qt * t.rows + (row_in_tile >> p.pack_shift);
-  const int head = t.h + (row_in_tile & ((1 << p.pack_shift) - 1));
-  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+  const int cq = lane & 3;
+  const int rt0 = quad * 32 + lh * 16 + (lane >> 2);
+  const int tile_row0 = t.m_base + qt * t.rows;
+  const int delta = t.sk - t.sq;
+  int row[2], head[2], key_lim[2], key_lo[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int rt = rt0 + 8 * r;
+    row[r] = tile_row0 + (rt >> p.pack_shift);
+    head[r] = t.h + (rt & ((1 << p.pack_shift) - 1));
+    key_lim[r] = CAUSAL ? min(t.sk, row[r] + delta + p.hi_off + 1) : t.sk;
+    key_lo[r] = row[r] + delta - p.lo_off;
+  }
+  const uint32_t lane_base = static_cast<uint32_t>(quad * 32 + lh * 16) << 16;
   const int n = t.n_blocks;
   const float c = SOFTCAP ? 1.f : p.scale_log2;
-  const int delta = t.sk - t.sq;
-  const int key_lim = CAUSAL ? min(t.sk, row + delta + p.hi_off + 1) : t.sk;
-  const int key_lo = row + delta - p.lo_off;
-  const int tile_row0 = t.m_base + qt * t.rows;
   const int mask_from = CAUSAL ? min(t.sk, tile_row0 + delta + p.hi_off + 1) : t.sk;
   const int lo_until = tile_row0 + (t.rows - 1) + delta - p.lo_off;
-  const int pair_bar = 3 + qt * 4 + quad;
-  float* xch = s.xch + qt * (2 * 2 * C::BM);  // [block parity][half][row]
 
   TRACE_INIT();
-  [[maybe_unused]] const bool tr_on = (hf == 0) && (row_in_tile == 0);
-  float m_run = -INFINITY;
-  float l_run = 0.f;
+  [[maybe_unused]] const bool tr_on = (lh == 0) && (quad == 0) && (lane == 0);
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_run[2] = {0.f, 0.f};
   bool ok = true;
   for (int j = 0; j < n; ++j) {
     const int slot = C::DBUF ? 2 * qt + (j & 1) : (j & 1);
     [[maybe_unused]] const int tr = (tr_on && j < 64) ? 1024 * qt + j * 8 : -1;
-    if (ok)
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], (j >> 1) & 1, s.abort, p.err,
-                                             ERR_FWD_SOFTMAX | 1, p.timeout_ns));
+    if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], (j >> 1) & 1, s.abort, p.err,
+                                           ERR_FWD_SOFTMAX | 1, p.timeout_ns))) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    TRACE(tr);
     const uint32_t s_addr = tmem + lane_base + slot * C::BN;
-    uint32_t sr[NC];  // this thread's scores of the block (fp32 bits), see key_of
-    float mx = -INFINITY;
+    uint32_t sr[4 * NX];
+    if constexpr (NX == 16) {
+      tmem_ld16r_x16(s_addr, sr);
+    } else {
+      uint32_t sa[32], sb[16];
+      tmem_ld16r_x8_x4(s_addr, sa, s_addr + 64, sb);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) sr[i] = sa[i];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sr[32 + i] = sb[i];
+    }
     const int kb = (t.n_lo + j) * C::BN;  // segment-local key of column 0
     const bool masked = (kb + C::BN > mask_from) || (kb < lo_until);
-    TRACE(tr);
-    if (ok) {
-      tc_fence_after();
-      if constexpr (C::BN == 96) {
-        uint32_t sa[32], sb[16];
-        tmem_ld32_16(s_addr + hf * 32, sa, s_addr + 64 + hf * 16, sb);
+    if (masked) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sr[i] = sa[i];
+      for (int r = 0; r < 2; ++r) {
+        const int lim = key_lim[r] - kb - 2 * cq, lo = key_lo[r] - kb - 2 * cq;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) sr[32 + i] = sb[i];
-      } else {
-        tmem_ld64(s_addr + hf * 64, sr);
+        for (int x = 0; x < NX; ++x)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if (8 * x + e >= lim || 8 * x + e < lo) sr[4 * x + 2 * r + e] = 0xff800000u;  // -inf
       }
-      if (masked) {
-        const int lim = key_lim - kb, lo = key_lo - kb;
-#pragma unroll
-        for (int i = 0; i < NC; ++i)
-          if (key_of(i) >= lim || key_of(i) < lo) sr[i] = 0xff800000u;  // -inf
-      }
-      if constexpr (SOFTCAP) {
-#pragma unroll
-        for (int i = 0; i < NC; ++i) sr[i] = fwd_cap(p, sr[i]);
-      }
-      float ch[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) ch[k] = __uint_as_float(sr[k]);
-#pragma unroll
-      for (int i = 8; i < NC; i += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          ch[k] = (i + 8 < NC) ? fmax3(ch[k], __uint_as_float(sr[i + k]),
-                                       __uint_as_float(sr[i + 8 + k]))
-                               : fmaxf(ch[k], __uint_as_float(sr[i + k]));
-      mx = fmaxf(fmax3(ch[0], ch[1], ch[2]), fmax3(ch[3], ch[4], fmax3(ch[5], ch[6], ch[7])));
     }
-    // both threads of the row have read their scores once they pass the
-    // barrier, so P may then go over the slot's first BN/2 columns
-    float* xb = xch + (j & 1) * (2 * C::BM);
-    xb[hf * C::BM + row_in_tile] = mx;
+    if constexpr (SOFTCAP) {
+#pragma unroll
+      for (int i = 0; i < 4 * NX; ++i) sr[i] = fwd_cap(p, sr[i]);
+    }
+    // row maxima: four chains per row over this thread's keys, then the row's
+    // other three threads
+    float mx[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float ch[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int x = 0; x < NX; ++x)
+        ch[x & 3] = fmax3(ch[x & 3], __uint_as_float(sr[4 * x + 2 * r]),
+                          __uint_as_float(sr[4 * x + 2 * r + 1]));
+      float m = fmaxf(fmaxf(ch[0], ch[1]), fmaxf(ch[2], ch[3]));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      mx[r] = m;
+    }
     TRACE(tr + 1);
-    named_bar_sync(pair_bar, 64);
-    TRACE(tr + 2);
-    if (!ok) continue;
-    mx = fmaxf(mx, xb[(1 - hf) * C::BM + row_in_tile]);
-    const float m_new = fmaxf(m_run, mx * c);
     bool rescale = false;
-    float alpha = 1.f;
-    if (j == 0) {
-      m_run = m_new;
-    } else if (m_new - m_run > 8.f) {
-      alpha = ex2(m_run - m_new);
-      rescale = true;
-      m_run = m_new;
-      l_run *= alpha;
-    }
-    const float m_sub = (m_run == -INFINITY) ? 0.f : m_run;
-    {
-      const uint64_t cc2 = f2_pack(c, c), mm2 = f2_pack(-m_sub, -m_sub);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-      uint32_t pk[NC / 2];  // P of the score pairs (2i, 2i + 1), bf16
+    float alpha[2] = {1.f, 1.f};
+    uint64_t mm2[2];
 #pragma unroll
-      for (int i = 0; i < NC / 2; ++i) {
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
-                         cc2, mm2),
-                  x0, x1);
-        const float p0 = ex2(x0), p1 = ex2(x1);
-        acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-        pk[i] = pack_bf16(p0, p1);
+    for (int r = 0; r < 2; ++r) {
+      const float m_new = fmaxf(m_run[r], mx[r] * c);
+      if (j == 0) {
+        m_run[r] = m_new;
+      } else if (m_new - m_run[r] > 8.f) {
+        alpha[r] = ex2(m_run[r] - m_new);
+        rescale = true;
+        m_run[r] = m_new;
+        l_run[r] *= alpha[r];
       }
-      // key k's P is at column k / 2 of the slot
-      if constexpr (C::BN == 96) {
+      const float m_sub = (m_run[r] == -INFINITY) ? 0.f : m_run[r];
+      mm2[r] = f2_pack(-m_sub, -m_sub);
+    }
+    {
+      const uint64_t cc2 = f2_pack(c, c);
+      uint64_t acc[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
+      uint32_t pk[2 * NX];  // register 2x + r: P of keys 8x + 2(t%4) + {0, 1} of row rt0 + 8r
+#pragma unroll
+      for (int x = 0; x < NX; ++x)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * x + 2 * r]),
+                                   __uint_as_float(sr[4 * x + 2 * r + 1])),
+                           cc2, mm2[r]),
+                    x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          acc[r][x & 1] = f2_add(acc[r][x & 1], f2_pack(p0, p1));
+          pk[2 * x + r] = pack_bf16(p0, p1);
+        }
+      // keys 2i, 2i + 1 of the block have their P at column i of the slot
+      if constexpr (NX == 16) {
+        tmem_st16h_x16(s_addr, pk);
+      } else {
         uint32_t pa[16], pb[8];
 #pragma unroll
         for (int i = 0; i < 16; ++i) pa[i] = pk[i];
 #pragma unroll
         for (int i = 0; i < 8; ++i) pb[i] = pk[16 + i];
-        tmem_st16(s_addr + hf * 16, pa);
-        tmem_st8(s_addr + 32 + hf * 8, pb);
-      } else {
-        tmem_st32(s_addr + hf * 32, pk);
+        tmem_st16h_x8(s_addr, pa);
+        tmem_st16h_x4(s_addr + 32, pb);
       }
-      TRACE(tr + 3);
-      float a0, a1, a2, a3;
-      f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
-      f2_unpack(f2_add(acc[2], acc[3]), a2, a3);
-      l_run += (a0 + a1) + (a2 + a3);
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        float a0, a1;
+        f2_unpack(f2_add(acc[r][0], acc[r][1]), a0, a1);
+        l_run[r] += a0 + a1;  // this thread's share; the row's four are summed at the end
+      }
     }
+    TRACE(tr + 2);
     if (__any_sync(0xffffffffu, rescale)) {
       // O must not be rescaled while the previous P.V MMA may still write it.
       // o_ready has completed j-1 or j phases here (S(j), just read, was issued
@@ -987,33 +990,37 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
       if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (j - 1) & 1, s.abort, p.err,
                                              ERR_FWD_SOFTMAX | 2, p.timeout_ns))) {
         ok = false;
-        continue;
+        break;
       }
       tc_fence_after();
-      const uint32_t o_addr = tmem + lane_base + C::O_COL0 + qt * D + hf * OC;
+      const uint32_t o_addr = tmem + lane_base + C::O_COL0 + qt * D;
 #pragma unroll 1
-      for (int cc = 0; cc < OC / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(o_addr + cc * 32, r);
+      for (int hc = 0; hc < D / 64; ++hc) {
+        uint32_t o[32];
+        tmem_ld16r_x8(o_addr + hc * 64, o);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-        tmem_st32(o_addr + cc * 32, r);
+        for (int i = 0; i < 32; ++i)
+          o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha[(i >> 1) & 1]);
+        tmem_st16r_x8(o_addr + hc * 64, o);
       }
     }
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.p_full[slot]);
-    TRACE(tr + 4);
+    TRACE(tr + 3);
   }
 
-  // ---- epilogue: the row sum is the sum of both halves' sums ----
-  float* xe = xch + (n & 1) * (2 * C::BM);  // not read since block n-2
-  xe[hf * C::BM + row_in_tile] = l_run;
-  named_bar_sync(pair_bar, 64);
-  const float l_tot = l_run + xe[(1 - hf) * C::BM + row_in_tile];
-  const bool row_valid = row < t.sq;
-  const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+  // ---- epilogue: the row sums are the sums of the row's four threads ----
+  float inv_l[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    float l = l_run[r];
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    l_run[r] = l;
+    inv_l[r] = (l > 0.f) ? 1.f / l : 0.f;
+  }
   uint8_t* stage = s.q + qt * C::Q_BYTES;
   constexpr int CPR = D / 8;  // 16-byte chunks per row
   // the tile's last P.V, on its single-phase barrier (see fwd_softmax)
@@ -1023,43 +1030,51 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
                                            ERR_FWD_SOFTMAX | 3, p.timeout_ns));
   if (ok) {
     tc_fence_after();
-    const uint32_t o_addr = tmem + lane_base + C::O_COL0 + qt * D + hf * OC;
+    const uint32_t o_addr = tmem + lane_base + C::O_COL0 + qt * D;
 #pragma unroll 1
-    for (int cc = 0; cc < OC / 32; ++cc) {
-      uint32_t r[32];
+    for (int hc = 0; hc < D / 64; ++hc) {  // columns [64 hc, 64 hc + 64)
+      uint32_t o[32];
       if (n > 0) {
-        tmem_ld32(o_addr + cc * 32, r);
+        tmem_ld16r_x8(o_addr + hc * 64, o);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = 0u;
-      }
-      if (p.num_splits > 1) {  // SplitKV: fp32 partial, straight from registers
-        fwd_store_part<D>(p, t, row, head, hf * OC + cc * 32, r, inv_l);
-        continue;
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
       }
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint4 v;
-        v.x = pack_bf16(__uint_as_float(r[g * 8 + 0]) * inv_l, __uint_as_float(r[g * 8 + 1]) * inv_l);
-        v.y = pack_bf16(__uint_as_float(r[g * 8 + 2]) * inv_l, __uint_as_float(r[g * 8 + 3]) * inv_l);
-        v.z = pack_bf16(__uint_as_float(r[g * 8 + 4]) * inv_l, __uint_as_float(r[g * 8 + 5]) * inv_l);
-        v.w = pack_bf16(__uint_as_float(r[g * 8 + 6]) * inv_l, __uint_as_float(r[g * 8 + 7]) * inv_l);
-        const int chunk = (hf * OC + cc * 32) / 8 + g;
-        *reinterpret_cast<uint4*>(stage + row_in_tile * (D * 2) +
-                                  ((chunk ^ (row_in_tile & 7)) * 16)) = v;
-      }
+      for (int x = 0; x < 8; ++x)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float v0 = __uint_as_float(o[4 * x + 2 * r]) * inv_l[r];
+          const float v1 = __uint_as_float(o[4 * x + 2 * r + 1]) * inv_l[r];
+          const int col = hc * 64 + 8 * x + 2 * cq;
+          if (p.num_splits > 1) {  // SplitKV: fp32 partial, straight from registers
+            if (row[r] < t.sq)
+              *reinterpret_cast<float2*>(
+                  p.o_part +
+                  ((static_cast<size_t>(t.split) * p.total_q + t.q0 + row[r]) * p.nheads_q +
+                   head[r]) * D + col) = make_float2(v0, v1);
+          } else {
+            // 16-byte chunk 8 hc + x of the row, 4 bytes at 4(t%4), swizzled
+            const int rt = rt0 + 8 * r;
+            *reinterpret_cast<uint32_t*>(stage + rt * (D * 2) +
+                                         (((8 * hc + x) ^ (rt & 7)) * 16) + 4 * cq) =
+                pack_bf16(v0, v1);
+          }
+        }
     }
   }
-  named_bar_sync(1 + qt, 256);  // both halves of the tile
+  named_bar_sync(1 + qt, 256);  // the whole tile is staged
   if (ok && p.num_splits > 1) {
-    if (hf == 0)
-      fwd_store_part_lse(p, t, row, head,
-                         (l_tot > 0.f) ? (m_run + __log2f(l_tot)) * 0.69314718055994530942f
-                                       : -INFINITY);
+    if (cq == 0)
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        fwd_store_part_lse(p, t, row[r], head[r],
+                           (l_run[r] > 0.f) ? (m_run[r] + __log2f(l_run[r])) * 0.69314718055994530942f
+                                            : -INFINITY);
   } else if (ok) {
     const int rows_left = t.sq - tile_row0;
     uint8_t* out = static_cast<uint8_t*>(p.out);
-    const int tid = hf * 128 + row_in_tile;
+    const int tid = lh * 128 + quad * 32 + lane;
 #pragma unroll 4
     for (int q = tid; q < C::BM * CPR; q += 256) {
       const int r = q / CPR, ch = q % CPR;
@@ -1071,10 +1086,13 @@ __device__ __forceinline__ void fwd_softmax_split(const FwdParams& p, const FwdT
         *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + gh) * D) * 2 + ch * 16) = v;
       }
     }
-    if (p.return_lse && row_valid && hf == 0) {
-      const float lse =
-          (l_tot > 0.f) ? (m_run + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
-      p.lse[static_cast<size_t>(head) * p.total_q + t.q0 + row] = lse;
+    if (p.return_lse && cq == 0) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        if (row[r] < t.sq)
+          p.lse[static_cast<size_t>(head[r]) * p.total_q + t.q0 + row[r]] =
+              (l_run[r] > 0.f) ? (m_run[r] + __log2f(l_run[r])) * 0.69314718055994530942f
+                               : -INFINITY;
     }
   }
 }
@@ -1131,7 +1149,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int qt = grp / C::ROW_SPLIT;
     if (t.m_base + qt * t.rows < t.sq) {
       if constexpr (C::ROW_SPLIT == 2)
-        fwd_softmax_split<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt, grp % 2);
+        fwd_softmax_rows16<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt, grp % 2);
       else
         fwd_softmax<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt);
     }
