@@ -192,6 +192,7 @@ struct MaskArgs {
   bool softcap;
   float cap_k2;    // 2 log2(e) scale / c
   float cap_log2;  // c * log2(e)
+  float cap_k1;    // scale / c
 };
 
 attn_status_t mask_args(int32_t causal, int32_t window_left, int32_t window_right,
@@ -207,6 +208,7 @@ attn_status_t mask_args(int32_t causal, int32_t window_left, int32_t window_righ
   m->softcap = softcap > 0.f;
   m->cap_k2 = m->softcap ? 2.f * 1.4426950408889634f * scale / softcap : 0.f;
   m->cap_log2 = m->softcap ? softcap * 1.4426950408889634f : 0.f;
+  m->cap_k1 = m->softcap ? scale / softcap : 0.f;
   return ATTN_OK;
 }
 
@@ -504,6 +506,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
   p.lo_off = mk.lo_off;
   p.cap_k2 = mk.cap_k2;
   p.cap_log2 = mk.cap_log2;
+  p.cap_k1 = mk.cap_k1;
   p.num_splits = num_splits;
   p.o_part = nullptr;
   p.lse_part = nullptr;

@@ -78,9 +78,10 @@ struct FwdParams {
   int hi_off;
   int lo_off;
   // softcap c: scores become c tanh(s scale / c); cap_k2 = 2 log2(e) scale / c,
-  // cap_log2 = c log2(e)
+  // cap_log2 = c log2(e), cap_k1 = scale / c
   float cap_k2;
   float cap_log2;
+  float cap_k1;
   // SplitKV: num_splits > 1 splits every CTA's key-block range into that many
   // contiguous parts (grid.z = batch * num_splits); each part writes its own
   // normalised O and LSE to o_part / lse_part for the combine kernel
@@ -102,6 +103,46 @@ struct FwdParams {
 __device__ __forceinline__ uint32_t fwd_cap(const FwdParams& p, uint32_t bits) {
   const float x = __uint_as_float(bits);
   return x == -INFINITY ? bits : __float_as_uint(p.cap_log2 * tanh_from_ex2(x * p.cap_k2));
+}
+
+// softcap of a thread's scores in place, in the log2 domain.  When no score of
+// the block is masked and every score of the warp has |s scale / c| <= 1/2,
+// tanh runs as an odd polynomial on the FMA pipe (softcap_poly_pair);
+// otherwise every score takes the identity through ex2 and rcp (fwd_cap;
+// masked -inf stays -inf).  `masked` is the same for the whole warp.
+template <int N>
+__device__ __forceinline__ void fwd_cap_scores(const FwdParams& p, uint32_t (&sr)[N],
+                                               bool masked) {
+  static_assert(N % 2 == 0, "score pairs");
+  bool poly = false;
+  if (!masked) {
+    float ma = 0.f;
+#pragma unroll
+    for (int i = 0; i < N; i += 2)
+      ma = fmax3(ma, fabsf(__uint_as_float(sr[i])), fabsf(__uint_as_float(sr[i + 1])));
+    poly = __all_sync(0xffffffffu, ma * p.cap_k1 <= tanhpoly::kY0);
+  }
+  if (poly) {
+    const float K = p.cap_log2;
+    const uint64_t k1 = f2_pack(p.cap_k1, p.cap_k1);
+    const uint64_t ka[5] = {f2_pack(K * tanhpoly::kA0, K * tanhpoly::kA0),
+                            f2_pack(K * tanhpoly::kA1, K * tanhpoly::kA1),
+                            f2_pack(K * tanhpoly::kA2, K * tanhpoly::kA2),
+                            f2_pack(K * tanhpoly::kA3, K * tanhpoly::kA3),
+                            f2_pack(K * tanhpoly::kA4, K * tanhpoly::kA4)};
+#pragma unroll
+    for (int i = 0; i < N; i += 2) {
+      float c0, c1;
+      f2_unpack(softcap_poly_pair(f2_pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
+                                  k1, ka),
+                c0, c1);
+      sr[i] = __float_as_uint(c0);
+      sr[i + 1] = __float_as_uint(c1);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) sr[i] = fwd_cap(p, sr[i]);
+  }
 }
 
 __device__ __forceinline__ void fwd_test_delay(const FwdParams& p) {
@@ -634,10 +675,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       for (int i = 0; i < NCOL; ++i)
         if (i >= lim || i < lo) sr[i] = 0xff800000u;  // -inf
     }
-    if constexpr (SOFTCAP) {
-#pragma unroll
-      for (int i = 0; i < NCOL; ++i) sr[i] = fwd_cap(p, sr[i]);
-    }
+    if constexpr (SOFTCAP) fwd_cap_scores(p, sr, masked);
     // row max: 8 independent chains of three-input max, then a short tree
     float mx;
     {
@@ -908,10 +946,7 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
             if (8 * x + e >= lim || 8 * x + e < lo) sr[4 * x + 2 * r + e] = 0xff800000u;  // -inf
       }
     }
-    if constexpr (SOFTCAP) {
-#pragma unroll
-      for (int i = 0; i < 4 * NX; ++i) sr[i] = fwd_cap(p, sr[i]);
-    }
+    if constexpr (SOFTCAP) fwd_cap_scores(p, sr, masked);
     // row maxima: four chains per row over this thread's keys, then the row's
     // other three threads
     float mx[2];
@@ -953,12 +988,18 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
       for (int x = 0; x < NX; ++x)
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * x + 2 * r]),
-                                   __uint_as_float(sr[4 * x + 2 * r + 1])),
-                           cc2, mm2[r]),
-                    x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[4 * x + 2 * r]),
+                                             __uint_as_float(sr[4 * x + 2 * r + 1])),
+                                     cc2, mm2[r]);
+          float p0, p1;
+          if (!masked && (x & 7) < ATTN_FWD_POLY_PAIRS) {
+            exp2_fma_pair(x2, p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
           acc[r][x & 1] = f2_add(acc[r][x & 1], f2_pack(p0, p1));
           pk[2 * x + r] = pack_bf16(p0, p1);
         }
