@@ -45,6 +45,7 @@ struct DeviceState {
   uint32_t* err = nullptr;
   int sm_major = 0, sm_minor = 0;
   int smem_optin = 0;
+  int num_sms = 0;
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -120,10 +121,18 @@ DeviceState* device_state(int* dev_out) {
     cudaDeviceGetAttribute(&st.sm_major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&st.sm_minor, cudaDevAttrComputeCapabilityMinor, dev);
     cudaDeviceGetAttribute(&st.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
   });
   if (st.init_status != cudaSuccess) return nullptr;
   *dev_out = dev;
   return &st;
+}
+
+// SMs of the current device (set up by device_state before any launch)
+int device_sm_count() {
+  int dev = 0;
+  DeviceState* st = device_state(&dev);
+  return (st && st->num_sms > 0) ? st->num_sms : 1;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -212,34 +221,39 @@ attn_status_t mask_args(int32_t causal, int32_t window_left, int32_t window_righ
   return ATTN_OK;
 }
 
-// head_dim 128 without softcap or SplitKV can run on the two-CTA kernel of
-// fwd_pair_kernel.cuh (M = 256 MMAs over a CTA pair, 128-key blocks) when
-// ATTN_FWD_PAIR=1 (read on every call, so tests can compare the two).  The
-// one-CTA kernel is the default: both are bound by the softmax warps' exps,
-// which cost the same per score in either, and the one-CTA kernel measured
-// faster.
-bool fwd_use_pair() {
+// head_dim 128 and 256 without softcap or SplitKV can run on the two-CTA
+// kernels of fwd_pair_kernel.cuh (M = 256 MMAs over a CTA pair, 128-key
+// blocks, each CTA loading half of every K and V block).  ATTN_FWD_PAIR=1 / 0
+// forces them on / off (read on every call, so tests can compare); by default
+// head_dim 256 uses them (the one-CTA kernel is bound by shared-memory reads
+// there, which the pair halves) and head_dim 128 does not (both kernels are
+// bound by the softmax warps' exps, and the one-CTA kernel measured faster).
+bool fwd_use_pair(int d) {
   const char* e = std::getenv("ATTN_FWD_PAIR");
-  return e && e[0] == '1';
+  if (e && e[0] == '1') return true;
+  if (e && e[0] == '0') return false;
+  return false;
 }
 
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 attn_status_t launch_fwd_pair(const void* q, const void* k, const void* v, int total_q,
                               int total_k, int hkv, const FwdParams& p, int batch, int hq,
                               int max_q, cudaStream_t stream) {
-  using C = FwdPairCfg;
+  using C = FwdPairCfg<D>;
   CUtensorMap mq, mk, mv;
   const int g = 1 << p.pack_shift;
-  if (!make_map(&mq, q, total_q, hq, C::D, C::BM / g, g) ||
-      !make_map(&mk, k, total_k, hkv, C::D, C::BN / 2) ||
-      !make_map(&mv, v, total_k, hkv, C::D, C::BN))
+  // head_dim 128: K boxes of this CTA's 64 keys, V boxes of 128 keys x 64
+  // columns; head_dim 256: 64-row boxes for both
+  const int k_rows = C::BN / 2, v_rows = (D == 128) ? C::BN : 64;
+  if (!make_map(&mq, q, total_q, hq, D, C::BM / g, g) ||
+      !make_map(&mk, k, total_k, hkv, D, k_rows) || !make_map(&mv, v, total_k, hkv, D, v_rows))
     return ATTN_ERR_CUDA;
   static std::once_flag attr_once[kMaxDevices];
   static cudaError_t attr_status[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
   std::call_once(attr_once[dev], [&] {
-    attr_status[dev] = cudaFuncSetAttribute(attn_fwd_pair_kernel<CAUSAL>,
+    attr_status[dev] = cudaFuncSetAttribute(attn_fwd_pair_kernel<D, CAUSAL>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             C::SMEM_BYTES);
   });
@@ -249,19 +263,33 @@ attn_status_t launch_fwd_pair(const void* q, const void* k, const void* v, int t
   if (pairs == 0) return ATTN_OK;
   dim3 grid(2 * pairs, p.pack_shift > 0 ? hkv : hq, batch);
   record_start(ATTN_KERNEL_FWD, stream);
-  attn_fwd_pair_kernel<CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  attn_fwd_pair_kernel<D, CAUSAL><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   const cudaError_t e = cudaGetLastError();
   record_stop(ATTN_KERNEL_FWD, stream);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// The forward's grid.  Persistent (one CTA per SM, each walking a static
+// share of the tiles, so a tile's loads and first MMAs overlap the previous
+// tile's epilogue) when every tile has the same work; otherwise one CTA per
+// tile, so the hardware hands tiles of unequal work to whichever SM is free
+// (a static share measured 17% slower on a varlen batch).  ATTN_FWD_GRID=
+// tiles / persistent forces either (read on every call, for tests).
+bool fwd_grid_persistent(const FwdParams& p) {
+  const char* e = std::getenv("ATTN_FWD_GRID");
+  if (e && std::strcmp(e, "tiles") == 0) return false;
+  if (e && std::strcmp(e, "persistent") == 0) return true;
+  return p.uniform_tiles != 0;
 }
 
 template <int D, bool CAUSAL, bool SOFTCAP>
 attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_q, int total_k,
                          int hkv, const FwdParams& p, int batch, int hq, int max_q,
                          cudaStream_t stream) {
-  if constexpr (D == 128 && !SOFTCAP) {
-    if (p.num_splits == 1 && fwd_use_pair())
-      return launch_fwd_pair<CAUSAL>(q, k, v, total_q, total_k, hkv, p, batch, hq, max_q, stream);
+  if constexpr (D != 64 && !SOFTCAP) {
+    if (p.num_splits == 1 && fwd_use_pair(D))
+      return launch_fwd_pair<D, CAUSAL>(q, k, v, total_q, total_k, hkv, p, batch, hq, max_q,
+                                        stream);
   }
   using C = FwdCfg<D>;
   // Q: one 128-row box per 64-column panel; K: one BN-row box per panel;
@@ -288,10 +316,18 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, int total_
   const int rows_per_cta = (C::BM * C::NQ) >> p.pack_shift;
   const int m_tiles = (max_q + rows_per_cta - 1) / rows_per_cta;
   if (m_tiles == 0) return ATTN_OK;
-  dim3 grid(m_tiles, p.pack_shift > 0 ? hkv : hq, batch);
+  // tiles: (query tile, head, segment x split); see fwd_grid_persistent
+  FwdParams pt = p;
+  pt.tiles_x = m_tiles;
+  pt.tiles_y = p.pack_shift > 0 ? hkv : hq;
+  pt.tiles_total = static_cast<long long>(m_tiles) * pt.tiles_y * batch;
+  const long long ctas = fwd_grid_persistent(p)
+                             ? std::min<long long>(pt.tiles_total, device_sm_count())
+                             : pt.tiles_total;
+  if (ctas > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   record_start(ATTN_KERNEL_FWD, stream);
-  attn_fwd_kernel<D, CAUSAL, SOFTCAP><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv,
-                                                                                  p);
+  attn_fwd_kernel<D, CAUSAL, SOFTCAP><<<static_cast<unsigned>(ctas), C::THREADS, C::SMEM_BYTES,
+                                        stream>>>(mq, mk, mv, pt);
   const cudaError_t e = cudaGetLastError();
   record_stop(ATTN_KERNEL_FWD, stream);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -517,6 +553,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
         bwd_align256(static_cast<size_t>(num_splits) * total_q * nheads_q * head_dim * 4));
   }
   p.pack_shift = pack_gqa_shift(nheads_q / nheads_kv);
+  // equal segments have total = batch x max (no segment is longer than max)
+  p.uniform_tiles = !mk.upper && mk.lo_off >= kNoBound && num_splits == 1 &&
+                    static_cast<int64_t>(batch) * max_seqlen_q == total_q &&
+                    static_cast<int64_t>(batch) * max_seqlen_k == total_k;
   p.timeout_ns = wait_timeout_ns();
   p.epilogue_delay_ns = test_epilogue_delay_ns();
 

@@ -92,6 +92,16 @@ struct FwdParams {
   // G = 1 << pack_shift query heads of its group; tile row r is query row
   // r >> pack_shift of head (r & (G - 1)), and grid.y runs over key/value heads
   int pack_shift;
+  // persistent tile schedule: the work is tiles_total tiles, the cells of a
+  // (tiles_x = query tiles per segment) x (tiles_y = heads) x (segments x
+  // splits) grid; the grid's gridDim.x CTAs each take every gridDim.x-th tile
+  // (see fwd_tile_index)
+  int tiles_x;
+  int tiles_y;
+  long long tiles_total;
+  // host-side only: every tile has the same work (equal segments, no upper or
+  // lower key bound, no split), so a static share per CTA is balanced
+  int uniform_tiles;
   uint64_t timeout_ns;
   // test hook (0 in normal use): the softmax warps idle this long before their
   // final wait, so the tile's last P.V is sure to have completed by then
@@ -192,8 +202,8 @@ struct FwdCfg {
   static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
   static constexpr int OFF_BAR = OFF_RING + NSLOT * CHUNK;
   // barriers: q_full[NQ] kv_full[NSTAGE] kv_empty[NSTAGE] s_full[NSS] p_full[NSS]
-  // o_ready[NQ] o_final[NQ]
-  static constexpr int NBAR = NQ + 2 * NSTAGE + 2 * NSS + 2 * NQ;
+  // o_ready[NQ] o_final[NQ] q_empty[NQ] o_empty[NQ]
+  static constexpr int NBAR = NQ + 2 * NSTAGE + 2 * NSS + 4 * NQ;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, false, false);
@@ -213,7 +223,9 @@ struct FwdSmem {
   uint64_t* s_full;
   uint64_t* p_full;
   uint64_t* o_ready;  // one phase per P.V (rescales wait on the previous one)
-  uint64_t* o_final;  // one phase per CTA: the tile's last P.V is done
+  uint64_t* o_final;  // one phase per tile: the tile's last P.V is done
+  uint64_t* q_empty;  // one phase per tile: its last S has read Q
+  uint64_t* o_empty;  // one phase per tile: the epilogue has read O
   uint32_t* tmem_base;
   volatile int* abort;
 };
@@ -232,6 +244,8 @@ __device__ __forceinline__ FwdSmem fwd_smem(uint8_t* base) {
   s.p_full = s.s_full + C::NSS;
   s.o_ready = s.p_full + C::NSS;
   s.o_final = s.o_ready + C::NQ;
+  s.q_empty = s.o_final + C::NQ;
+  s.o_empty = s.q_empty + C::NQ;
   s.tmem_base = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
   s.abort = reinterpret_cast<volatile int*>(base + C::OFF_MISC + 4);
   return s;
@@ -270,16 +284,32 @@ __device__ __forceinline__ void fwd_store_part_lse(const FwdParams& p, const Fwd
     p.lse_part[(static_cast<size_t>(t.split) * p.nheads_q + head) * p.total_q + t.q0 + row] = lse;
 }
 
+// The tiles of this CTA, in order: the k-th is tile k * P + b for even k and
+// k * P + (P - 1 - b) for odd k (P CTAs, this one b), so each CTA's share
+// alternates between the front and the back of every run of P tiles; -1 once
+// past the last tile.
+__device__ __forceinline__ long long fwd_tile_index(const FwdParams& p, int k) {
+  const long long P = gridDim.x, b = blockIdx.x;
+  const long long L = static_cast<long long>(k) * P + ((k & 1) ? (P - 1 - b) : b);
+  return L < p.tiles_total ? L : -1;
+}
+
+// Tile L of the schedule: query tile x of segment (and split) z for head (or,
+// packing GQA, key/value head) y; false if it holds no query row.
 template <int D, bool CAUSAL>
-__device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t) {
+__device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t, long long L) {
   using C = FwdCfg<D>;
-  const int b = blockIdx.z / p.num_splits;
-  t.split = blockIdx.z % p.num_splits;
+  const int x = static_cast<int>(L % p.tiles_x);
+  const long long yz = L / p.tiles_x;
+  const int y = static_cast<int>(yz % p.tiles_y);
+  const int z = static_cast<int>(yz / p.tiles_y);
+  const int b = z / p.num_splits;
+  t.split = z % p.num_splits;
   if (p.pack_shift > 0) {
-    t.hk = blockIdx.y;
+    t.hk = y;
     t.h = t.hk << p.pack_shift;  // first query head of the group
   } else {
-    t.h = blockIdx.y;
+    t.h = y;
     t.hk = t.h / (p.nheads_q / p.nheads_kv);
   }
   t.rows = C::BM >> p.pack_shift;
@@ -288,7 +318,7 @@ __device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t) {
   t.k0 = p.cu_k[b];
   t.sk = p.cu_k[b + 1] - t.k0;
   // causal: heaviest tiles (bottom of the segment) first
-  const int m_tile = CAUSAL ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
+  const int m_tile = CAUSAL ? (p.tiles_x - 1 - x) : x;
   t.m_base = m_tile * t.rows * C::NQ;
   if (t.m_base >= t.sq) return false;
   // the union of the rows' allowed key ranges
@@ -312,29 +342,54 @@ __device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t) {
   return true;
 }
 
+// Walks the key blocks of this CTA's tiles in order (tiles without blocks are
+// skipped): block j of tile t.  The producer and the MMA warps each keep two,
+// one a block ahead of the other.
+template <int D, bool CAUSAL>
+struct FwdBlocks {
+  const FwdParams& p;
+  FwdTile t;
+  int k = -1;     // position of the tile in this CTA's sequence
+  int j = 0;      // block within the tile
+  bool ok = false;
+  __device__ explicit FwdBlocks(const FwdParams& p_) : p(p_) { next_tile(); }
+  __device__ void next_tile() {
+    while (true) {
+      const long long L = fwd_tile_index(p, ++k);
+      if (L < 0) {
+        ok = false;
+        return;
+      }
+      if (fwd_tile<D, CAUSAL>(p, t, L) && t.n_blocks > 0) break;
+    }
+    j = 0;
+    ok = true;
+  }
+  __device__ void advance() {
+    if (++j >= t.n_blocks) next_tile();
+  }
+  __device__ bool has_rows(int qt) const { return t.m_base + qt * t.rows < t.sq; }
+};
+
 // ---------------------------------------------------------------------------
-// producer warp: Q once, then K/V chunks in MMA consumption order
+// producer warp (one lane): for each of the CTA's tiles its Q tiles, then K/V
+// chunks in MMA consumption order, without a break between tiles.  A tile's Q
+// is loaded once the MMA warp's last S of the previous tile has read the Q
+// buffer (q_empty), so it lands while the previous tile finishes.
 // ---------------------------------------------------------------------------
-template <int D>
-__device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, const FwdSmem& s,
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdSmem& s,
                                          const CUtensorMap* tmQ, const CUtensorMap* tmK,
                                          const CUtensorMap* tmV) {
   using C = FwdCfg<D>;
-  if (t.n_blocks == 0) return;  // nothing to attend to: no copy may outlive the CTA
-  for (int qt = 0; qt < C::NQ; ++qt) {
-    if (t.m_base + qt * t.rows >= t.sq) break;
-    mbar_expect_tx(&s.q_full[qt], C::Q_BYTES);
-    // one box per panel: t.rows query rows x (packed: all G heads) x 64 columns
-    for (int pn = 0; pn < C::PANELS; ++pn)
-      tma_load_3d(s.q + qt * C::Q_BYTES + pn * C::QPANEL, tmQ, &s.q_full[qt], pn * 64, t.h,
-                  t.q0 + t.m_base + qt * t.rows);
-  }
-  uint32_t ring = 0;  // stages issued so far
+  uint32_t ring = 0;             // stages issued so far
+  uint32_t q_loads[C::NQ] = {};  // Q tiles issued so far, per query tile
   // on the way out after a timed-out wait elsewhere: let every copy this CTA
-  // issued land before its shared memory is released
+  // issued land before its shared memory is released (earlier Q copies have
+  // landed: each was read before the next was issued)
   auto drain = [&]() {
     for (int qt = 0; qt < C::NQ; ++qt)
-      if (t.m_base + qt * t.rows < t.sq) mbar_wait_drain(&s.q_full[qt], 0, 100000000ull);
+      if (q_loads[qt] > 0) mbar_wait_drain(&s.q_full[qt], (q_loads[qt] - 1) & 1, 100000000ull);
     const uint32_t first = ring > (uint32_t)C::NSTAGE ? ring - C::NSTAGE : 0u;
     for (uint32_t r = first; r < ring; ++r)
       mbar_wait_drain(&s.kv_full[r % C::NSTAGE], (r / C::NSTAGE) & 1, 100000000ull);
@@ -355,44 +410,80 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdTile& t, c
     ++ring;
     return true;
   };
-  // K block j: one chunk per 64-column panel (BN rows, K-major)
-  auto load_k = [&](uint8_t* dst, uint64_t* full, int j, int c) {
+  // the Q tiles of a tile, once the previous Q in each buffer has been read
+  auto load_q = [&](const FwdTile& t) -> bool {
+    for (int qt = 0; qt < C::NQ; ++qt) {
+      if (t.m_base + qt * t.rows >= t.sq) break;
+      if (q_loads[qt] > 0 &&
+          !mbar_wait(&s.q_empty[qt], (q_loads[qt] - 1) & 1, s.abort, p.err, ERR_FWD_LOAD | 2,
+                     p.timeout_ns)) {
+        drain();
+        return false;
+      }
+      mbar_expect_tx(&s.q_full[qt], C::Q_BYTES);
+      // one box per panel: t.rows query rows x (packed: all G heads) x 64 columns
+      for (int pn = 0; pn < C::PANELS; ++pn)
+        tma_load_3d(s.q + qt * C::Q_BYTES + pn * C::QPANEL, tmQ, &s.q_full[qt], pn * 64, t.h,
+                    t.q0 + t.m_base + qt * t.rows);
+      ++q_loads[qt];
+    }
+    return true;
+  };
+  // K block j of tile t: one chunk per 64-column panel (BN rows, K-major)
+  auto load_k = [&](const FwdTile& t, uint8_t* dst, uint64_t* full, int j, int c) {
     tma_load_3d(dst, tmK, full, c * 64, t.hk, t.k0 + (t.n_lo + j) * C::BN);
   };
   // rows [c*VROWS, (c+1)*VROWS) of V block j: all D columns, panel by panel
-  auto load_v = [&](uint8_t* dst, uint64_t* full, int j, int c) {
+  auto load_v = [&](const FwdTile& t, uint8_t* dst, uint64_t* full, int j, int c) {
     for (int pn = 0; pn < C::PANELS; ++pn)
       tma_load_3d(dst + pn * (C::VROWS * 128), tmV, full, pn * 64, t.hk,
                   t.k0 + (t.n_lo + j) * C::BN + c * C::VROWS);
   };
-  const int n = t.n_blocks;
+  FwdBlocks<D, CAUSAL> kc(p);  // next block whose K is loaded
+  FwdBlocks<D, CAUSAL> vc(p);  // next block whose V is loaded
   uint8_t* base;
   uint64_t* full;
   if constexpr (C::DBUF) {
-    // stage j = (K_j, V_{j-1}); the first holds only K_0, the last only V_{n-1}
-    for (int j = 0; j <= n; ++j) {
-      const uint32_t bytes = ((j < n) ? C::PANELS * C::CHUNK : 0) + ((j > 0) ? C::PANELS * C::CHUNK : 0);
+    // stage = (K of the next block, V of the block before it), exactly what one
+    // MMA iteration consumes; the first holds only K, the last only V
+    bool v_on = false;
+    while (kc.ok || (v_on && vc.ok)) {
+      if (kc.ok && kc.j == 0 && !load_q(kc.t)) return;
+      const bool has_v = v_on && vc.ok;
+      const uint32_t bytes =
+          (kc.ok ? C::PANELS * C::CHUNK : 0) + (has_v ? C::PANELS * C::CHUNK : 0);
       if (!claim(bytes, base, full)) return;
       for (int c = 0; c < C::PANELS; ++c) {
-        if (j < n) load_k(base + c * C::CHUNK, full, j, c);
-        if (j > 0) load_v(base + (C::PANELS + c) * C::CHUNK, full, j - 1, c);
+        if (kc.ok) load_k(kc.t, base + c * C::CHUNK, full, kc.j, c);
+        if (has_v) load_v(vc.t, base + (C::PANELS + c) * C::CHUNK, full, vc.j, c);
       }
+      if (has_v) vc.advance();
+      if (kc.ok) kc.advance();
+      v_on = true;
     }
   } else {
-    // one chunk per stage, in the MMA warp's order: K_0, K_1, then V_j before K_{j+2}
-    auto load_tile = [&](bool is_v, int j) -> bool {
+    // one chunk per stage, in the MMA warp's order: K of blocks 0 and 1, then
+    // V of block g before K of block g + 2
+    auto load_tile = [&](bool is_v, const FwdTile& t, int j) -> bool {
       for (int c = 0; c < C::PANELS; ++c) {
         if (!claim(C::CHUNK, base, full)) return false;
-        if (is_v) load_v(base, full, j, c);
-        else load_k(base, full, j, c);
+        if (is_v) load_v(t, base, full, j, c);
+        else load_k(t, base, full, j, c);
       }
       return true;
     };
-    if (n > 0 && !load_tile(false, 0)) return;
-    if (n > 1 && !load_tile(false, 1)) return;
-    for (int j = 0; j < n; ++j) {
-      if (!load_tile(true, j)) return;
-      if (j + 2 < n && !load_tile(false, j + 2)) return;
+    auto next_k = [&]() -> bool {
+      if (!kc.ok) return true;
+      if (kc.j == 0 && !load_q(kc.t)) return false;
+      if (!load_tile(false, kc.t, kc.j)) return false;
+      kc.advance();
+      return true;
+    };
+    if (!next_k() || !next_k()) return;
+    while (vc.ok) {
+      if (!load_tile(true, vc.t, vc.j)) return;
+      vc.advance();
+      if (!next_k()) return;
     }
   }
 }
@@ -519,90 +610,149 @@ struct FwdMma {
   }
 };
 
-template <int D>
-__device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdTile& t, const FwdSmem& s,
-                                        uint32_t tmem, int qt) {
+// The MMA warp of query tile qt walks the CTA's key blocks across all its
+// tiles in the producer's order.  A tile's first S waits for its Q (q_full),
+// its last S releases the Q buffer (q_empty); its first P.V (which overwrites
+// O) waits until the epilogue of the previous tile has read O (o_empty), its
+// last P.V completes o_final.  Blocks of tiles in which this query tile has
+// no rows are only released.  The S slots and barrier phases run on over the
+// tiles (g_s, g_v count this warp's S and P.V).
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem& s, uint32_t tmem,
+                                        int qt) {
   using C = FwdCfg<D>;
   TRACE_INIT();
   FwdMma<D> m(p, s, tmem);
-  const int n = t.n_blocks;
-  if (n == 0) return;
-  if (!mbar_wait_warp(&s.q_full[qt], 0, s.abort, p.err, ERR_FWD_MMA | 2, p.timeout_ns)) return;
-  tc_fence_after();
+  FwdBlocks<D, CAUSAL> sc(p);  // next block whose S is issued
+  FwdBlocks<D, CAUSAL> vc(p);  // next block whose P.V is issued
+  uint32_t g_s = 0, g_v = 0;   // S and P.V issued by this warp
+  uint32_t q_uses = 0;         // Q tiles read (phases of q_full / q_empty)
+  uint32_t o_tiles = 0;        // tiles whose first P.V was issued (phases of o_empty)
+  auto wait = [&](uint64_t* bar, uint32_t parity, uint32_t code) -> bool {
+    if (!mbar_wait_warp(bar, parity, s.abort, p.err, ERR_FWD_MMA | code, p.timeout_ns))
+      return false;
+    tc_fence_after();
+    return true;
+  };
+  // the P.V of the block at vc into slot `slot`, V in ring chunk ch (DBUF) or
+  // streamed chunk by chunk
+  auto pv = [&](int slot, uint32_t ch) -> bool {
+    if (!wait(&s.p_full[slot], (g_v >> 1) & 1, 3)) return false;
+    if (vc.j == 0) {
+      if (o_tiles > 0 && !wait(&s.o_empty[qt], (o_tiles - 1) & 1, 4)) return false;
+      ++o_tiles;
+    }
+    if constexpr (C::DBUF) {
+      m.issue_pv(qt, slot, ch, vc.j > 0);
+    } else {
+      if (!m.issue_pv_streamed(qt, slot, vc.j > 0)) return false;
+    }
+    mma_commit(&s.o_ready[qt]);
+    if (vc.j == vc.t.n_blocks - 1) mma_commit(&s.o_final[qt]);
+    ++g_v;
+    return true;
+  };
 
   if constexpr (C::DBUF) {
-    // This warp serves query tile qt; the other tile has its own MMA warp, so
-    // one can issue while the other waits on a barrier.  Both read every ring
-    // stage and both release it (the empty barriers count one arrival per
-    // tile).  S of block j lives in slot 2qt + (j & 1); S(j+1) is issued before
-    // P(j).V so the tensor pipe has work while the softmax runs on S(j); the
-    // slot it overwrites held P(j-1), read by the P.V this thread issued one
-    // iteration earlier on the same in-order pipe.  Stage j holds K_j in its
-    // first PANELS chunks and V_{j-1} in the next PANELS.
-    uint32_t ch;
-    if (!m.wait_stages(1, ch)) return;
-    m.issue_s(qt, 2 * qt, ch);
-    mma_commit(&s.s_full[2 * qt]);
-    m.release_stages(1);
-    for (int j = 0; j < n; ++j) {
-      const int b = j & 1;
-      [[maybe_unused]] const int tr = (j < 64) ? 2048 + 16 * j + 8 * qt : -1;
+    // Both MMA warps read every ring stage and both release it (the empty
+    // barriers count one arrival per query tile).  Stage = (K of the next
+    // block, V of the block before it): S of a block is issued before the P.V
+    // of the previous one, so the tensor pipe has work while the softmax runs.
+    // S(g) lives in slot 2qt + (g & 1); the slot it overwrites held P(g - 2),
+    // read by the P.V this thread issued one step earlier on the same in-order
+    // pipe.
+    bool v_on = false;
+    while (sc.ok || (v_on && vc.ok)) {
+      [[maybe_unused]] const int tr = (g_s < 64) ? 2048 + 16 * g_s + 8 * qt : -1;
       TRACE(tr);
+      uint32_t ch;
       if (!m.wait_stages(1, ch)) return;
       TRACE(tr + 1);
-      if (j + 1 < n) {
-        m.issue_s(qt, 2 * qt + (b ^ 1), ch);
-        mma_commit(&s.s_full[2 * qt + (b ^ 1)]);
+      if (sc.ok && sc.has_rows(qt)) {
+        if (sc.j == 0 && !wait(&s.q_full[qt], q_uses & 1, 2)) return;
+        const int slot = 2 * qt + (g_s & 1);
+        m.issue_s(qt, slot, ch);
+        mma_commit(&s.s_full[slot]);
+        if (sc.j == sc.t.n_blocks - 1) {
+          mma_commit(&s.q_empty[qt]);
+          ++q_uses;
+        }
+        ++g_s;
       }
       TRACE(tr + 2);
-      if (!mbar_wait_warp(&s.p_full[2 * qt + b], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
-                     p.timeout_ns))
-        return;
-      tc_fence_after();
-      TRACE(tr + 3);
-      m.issue_pv(qt, 2 * qt + b, ch + C::PANELS, j > 0);
-      mma_commit(&s.o_ready[qt]);
-      m.release_stages(1);
+      if (v_on && vc.ok && vc.has_rows(qt) && !pv(2 * qt + (g_v & 1), ch + C::PANELS)) return;
       TRACE(tr + 4);
+      m.release_stages(1);
+      if (v_on && vc.ok) vc.advance();
+      if (sc.ok) sc.advance();
+      v_on = true;
     }
-    mma_commit(&s.o_final[qt]);
   } else {
-    // one query tile, two S slots alternating over key blocks; one chunk per
-    // stage, each waited for right before its MMAs
-    if (!m.issue_s_streamed(0, 0)) return;
-    mma_commit(&s.s_full[0]);
-    if (n > 1) {
-      if (!m.issue_s_streamed(0, 1)) return;
-      mma_commit(&s.s_full[1]);
-    }
-    for (int j = 0; j < n; ++j) {
-      const int slot = j & 1;
-      [[maybe_unused]] const int tr = (j < 64) ? 2048 + 16 * j : -1;
-      TRACE(tr);
-      if (!mbar_wait_warp(&s.p_full[slot], (j >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
-                     p.timeout_ns))
-        return;
-      tc_fence_after();
-      TRACE(tr + 1);
-      if (!m.issue_pv_streamed(0, slot, j > 0)) return;
-      mma_commit(&s.o_ready[0]);
-      TRACE(tr + 3);
-      if (j + 2 < n) {
-        if (!m.issue_s_streamed(0, slot)) return;
-        mma_commit(&s.s_full[slot]);
-        TRACE(tr + 5);
+    // one query tile, two S slots alternating over the blocks; one chunk per
+    // stage, each waited for right before its MMAs.  Order: S of blocks 0 and
+    // 1, then P.V of block g before S of block g + 2.
+    auto next_s = [&]() -> bool {
+      if (!sc.ok) return true;
+      if (sc.j == 0 && !wait(&s.q_full[0], q_uses & 1, 2)) return false;
+      const int slot = g_s & 1;
+      if (!m.issue_s_streamed(0, slot)) return false;
+      mma_commit(&s.s_full[slot]);
+      if (sc.j == sc.t.n_blocks - 1) {
+        mma_commit(&s.q_empty[0]);
+        ++q_uses;
       }
+      ++g_s;
+      sc.advance();
+      return true;
+    };
+    if (!next_s() || !next_s()) return;
+    while (vc.ok) {
+      [[maybe_unused]] const int tr = (g_v < 64) ? 2048 + 16 * g_v : -1;
+      TRACE(tr);
+      if (!pv(g_v & 1, 0)) return;
+      TRACE(tr + 3);
+      vc.advance();
+      if (!next_s()) return;
+      TRACE(tr + 5);
     }
-    mma_commit(&s.o_final[0]);
+  }
+}
+
+// What a softmax warp carries from tile to tile: the S slots and the
+// o_ready / o_final phases run on over the CTA's tiles.
+struct FwdSoftState {
+  uint32_t g = 0;   // blocks of this query tile processed so far (all tiles)
+  uint32_t nt = 0;  // tiles with blocks finished (phases of o_final / o_empty)
+  bool ok = true;   // false after a timed-out wait: the warp stops
+};
+
+// one tile's epilogue output: 32 columns of a row's O / l as bf16, straight
+// from registers into out[row][head]
+template <int D>
+__device__ __forceinline__ void fwd_store_o32(const FwdParams& p, const FwdTile& t, int row,
+                                              int head, int col0, const uint32_t (&r)[32],
+                                              float inv_l) {
+  uint4* dst = reinterpret_cast<uint4*>(
+      static_cast<uint16_t*>(p.out) +
+      (static_cast<size_t>(t.q0 + row) * p.nheads_q + head) * D + col0);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint4 v;
+    v.x = pack_bf16(__uint_as_float(r[g * 8 + 0]) * inv_l, __uint_as_float(r[g * 8 + 1]) * inv_l);
+    v.y = pack_bf16(__uint_as_float(r[g * 8 + 2]) * inv_l, __uint_as_float(r[g * 8 + 3]) * inv_l);
+    v.z = pack_bf16(__uint_as_float(r[g * 8 + 4]) * inv_l, __uint_as_float(r[g * 8 + 5]) * inv_l);
+    v.w = pack_bf16(__uint_as_float(r[g * 8 + 6]) * inv_l, __uint_as_float(r[g * 8 + 7]) * inv_l);
+    dst[g] = v;
   }
 }
 
 // ---------------------------------------------------------------------------
-// softmax warpgroup: one thread per query row
+// softmax warpgroup: one thread per query row; one tile
 // ---------------------------------------------------------------------------
 template <int D, bool CAUSAL, bool SOFTCAP>
 __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t,
-                                            const FwdSmem& s, uint32_t tmem, int qt) {
+                                            const FwdSmem& s, uint32_t tmem, int qt,
+                                            FwdSoftState& st) {
   using C = FwdCfg<D>;
   const int warp = (threadIdx.x >> 5) & 3;  // warp within the warpgroup = TMEM lane quadrant
   const int lane = lane_id();
@@ -628,8 +778,11 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   // With two query tiles, warp w of each tile shares an SM sub-partition and
   // its special-function unit: their exp phases take turns (tile 0 first in
   // each block) through a pair of named barriers, so one warp's loads, max and
-  // stores overlap the other's exps.  A warp that gives up on a timed-out wait
-  // still plays its remaining turns, so its partner never waits forever.
+  // stores overlap the other's exps.  Every turn of tile 1 ends with an arrive
+  // for tile 0, and tile 0 takes the last one at the end of the tile, so each
+  // barrier sees exactly one arrive and one sync per turn and nothing carries
+  // over into the next tile.  A warp that gives up on a timed-out wait still
+  // plays its remaining turns, so its partner never waits forever.
   const bool pingpong = C::DBUF && C::ROW_SPLIT == 1 && (t.m_base + t.rows < t.sq);
   const int bar_t0 = 3 + 2 * warp, bar_t1 = 4 + 2 * warp;  // "tile 0 / tile 1 may start"
   auto turn_begin = [&](int k) {
@@ -641,7 +794,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   };
   auto turn_end = [&](int k) {
     if (qt == 0) named_bar_arrive(bar_t1, 64);
-    else if (k + 1 < n) named_bar_arrive(bar_t0, 64);
+    else named_bar_arrive(bar_t0, 64);
   };
   int turns_done = 0;
 
@@ -652,8 +805,9 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
 
   constexpr int NCOL = C::BN;  // scores per row and block
   for (int j = 0; j < n; ++j) {
-    const int slot = C::DBUF ? 2 * qt + (j & 1) : (j & 1);
-    const uint32_t parity = (j >> 1) & 1;
+    const uint32_t g = st.g + j;  // this block's index over the CTA's tiles
+    const int slot = C::DBUF ? 2 * qt + (g & 1) : (g & 1);
+    const uint32_t parity = (g >> 1) & 1;
     if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], parity, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 1, p.timeout_ns))) {
       ok = false;
@@ -761,10 +915,10 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
     if (threadIdx.x % 128 == 0 && j < 64) TRACE(1024 * qt + j * 8 + 3);
     if (__any_sync(0xffffffffu, rescale)) {
       // O must not be rescaled while the previous P.V MMA may still write it.
-      // o_ready has completed j-1 or j phases here (S(j), just read, was issued
-      // after P.V(j-2), and P.V(j) needs this block's P), so the parity of
-      // phase j-1 is unambiguous.
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (j - 1) & 1, s.abort, p.err,
+      // Counting over the CTA's tiles, o_ready has completed g-1 or g phases
+      // here (S(g), just read, was issued after P.V(g-2), and P.V(g) needs this
+      // block's P), so the parity of phase g-1 is unambiguous (j > 0 here).
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (g - 1) & 1, s.abort, p.err,
                                              ERR_FWD_SOFTMAX | 2, p.timeout_ns))) {
         ok = false;
         turns_done = j + 1;
@@ -794,19 +948,17 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       turn_end(k);
     }
 
-  // ---- epilogue: O / l -> bf16, staged through this tile's Q buffer ----
+  // ---- epilogue: O / l -> bf16, straight from registers to out ----
   const bool row_valid = row < t.sq;
   const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-  uint8_t* stage = s.q + qt * C::Q_BYTES;
-  constexpr int CPR = D / 8;  // 16-byte chunks per row
-  // Wait for the tile's last P.V on its own single-phase barrier.  A parity
-  // wait on o_ready cannot do it: the last S this warpgroup read was issued
-  // before the second-to-last P.V, so o_ready may be anywhere from two phases
-  // short of the end to already past it, and a parity test cannot tell a phase
-  // two behind from the current one.
+  // Wait for the tile's last P.V on o_final, which completes once per tile
+  // with blocks.  A parity wait on o_ready cannot do it: the last S this
+  // warpgroup read was issued before the second-to-last P.V, so o_ready may be
+  // anywhere from two phases short of the end to already past it, and a
+  // parity test cannot tell a phase two behind from the current one.
   fwd_test_delay(p);
   if (ok && n > 0) {
-    if (!__all_sync(0xffffffffu, mbar_wait(&s.o_final[qt], 0, s.abort, p.err,
+    if (!__all_sync(0xffffffffu, mbar_wait(&s.o_final[qt], st.nt & 1, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 3, p.timeout_ns)))
       ok = false;
   }
@@ -822,49 +974,29 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
 #pragma unroll
         for (int i = 0; i < 32; ++i) r[i] = 0u;
       }
-      if (p.num_splits > 1) {  // SplitKV: fp32 partial, straight from registers
+      if (p.num_splits > 1)  // SplitKV: fp32 partial
         fwd_store_part<D>(p, t, row, head, cc * 32, r, inv_l);
-        continue;
-      }
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {  // 4 chunks of 8 columns
-        uint4 v;
-        v.x = pack_bf16(__uint_as_float(r[g * 8 + 0]) * inv_l, __uint_as_float(r[g * 8 + 1]) * inv_l);
-        v.y = pack_bf16(__uint_as_float(r[g * 8 + 2]) * inv_l, __uint_as_float(r[g * 8 + 3]) * inv_l);
-        v.z = pack_bf16(__uint_as_float(r[g * 8 + 4]) * inv_l, __uint_as_float(r[g * 8 + 5]) * inv_l);
-        v.w = pack_bf16(__uint_as_float(r[g * 8 + 6]) * inv_l, __uint_as_float(r[g * 8 + 7]) * inv_l);
-        const int chunk = cc * 4 + g;
-        *reinterpret_cast<uint4*>(stage + row_in_tile * (D * 2) +
-                                  ((chunk ^ (row_in_tile & 7)) * 16)) = v;
-      }
+      else if (row_valid)
+        fwd_store_o32<D>(p, t, row, head, cc * 32, r, inv_l);
     }
-  }
-  named_bar_sync(1 + qt, 128);
-  if (ok && p.num_splits > 1) {
-    fwd_store_part_lse(p, t, row, head,
-                       (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f
-                                     : -INFINITY);
-  } else if (ok) {
-    const int rows_left = t.sq - tile_row0;
-    uint8_t* out = static_cast<uint8_t*>(p.out);
-    const int tid = threadIdx.x & 127;
-#pragma unroll 4
-    for (int q = tid; q < C::BM * CPR; q += 128) {
-      const int r = q / CPR, ch = q % CPR;
-      if ((r >> p.pack_shift) < rows_left) {
-        const uint4 v =
-            *reinterpret_cast<const uint4*>(stage + r * (D * 2) + ((ch ^ (r & 7)) * 16));
-        const size_t grow = static_cast<size_t>(t.q0 + tile_row0 + (r >> p.pack_shift));
-        const int gh = t.h + (r & ((1 << p.pack_shift) - 1));
-        *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + gh) * D) * 2 + ch * 16) = v;
-      }
+    if (n > 0) {
+      // O is read: the next tile's first P.V may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.o_empty[qt]);
     }
-    if (p.return_lse && row_valid) {
-      const float lse =
-          (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+    const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f
+                                    : -INFINITY;
+    if (p.num_splits > 1)
+      fwd_store_part_lse(p, t, row, head, lse);
+    else if (p.return_lse && row_valid)
       p.lse[static_cast<size_t>(head) * p.total_q + t.q0 + row] = lse;
-    }
   }
+  // tile 0 takes tile 1's arrive from the tile's last turn
+  if (pingpong && qt == 0 && n > 0) named_bar_sync(bar_t0, 64);
+  st.g += n;
+  if (n > 0) ++st.nt;
+  st.ok = ok;
 }
 
 // ---------------------------------------------------------------------------
@@ -881,7 +1013,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
 template <int D, bool CAUSAL, bool SOFTCAP>
 __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const FwdTile& t,
                                                    const FwdSmem& s, uint32_t tmem, int qt,
-                                                   int lh) {
+                                                   int lh, FwdSoftState& st) {
   using C = FwdCfg<D>;
   constexpr int NX = C::BN / 8;  // 8-key groups per block: 12 or 16
   static_assert((C::BN == 96 || C::BN == 128) && D % 64 == 0, "16-row layout");
@@ -912,9 +1044,10 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
   float l_run[2] = {0.f, 0.f};
   bool ok = true;
   for (int j = 0; j < n; ++j) {
-    const int slot = C::DBUF ? 2 * qt + (j & 1) : (j & 1);
+    const uint32_t g = st.g + j;  // this block's index over the CTA's tiles
+    const int slot = C::DBUF ? 2 * qt + (g & 1) : (g & 1);
     [[maybe_unused]] const int tr = (tr_on && j < 64) ? 1024 * qt + j * 8 : -1;
-    if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], (j >> 1) & 1, s.abort, p.err,
+    if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], (g >> 1) & 1, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 1, p.timeout_ns))) {
       ok = false;
       break;
@@ -1024,11 +1157,9 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
     }
     TRACE(tr + 2);
     if (__any_sync(0xffffffffu, rescale)) {
-      // O must not be rescaled while the previous P.V MMA may still write it.
-      // o_ready has completed j-1 or j phases here (S(j), just read, was issued
-      // after P.V(j-2), and P.V(j) needs this block's P), so the parity of
-      // phase j-1 is unambiguous.
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (j - 1) & 1, s.abort, p.err,
+      // O must not be rescaled while the previous P.V MMA may still write it
+      // (the parity of phase g-1 of o_ready is unambiguous, see fwd_softmax)
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.o_ready[qt], (g - 1) & 1, s.abort, p.err,
                                              ERR_FWD_SOFTMAX | 2, p.timeout_ns))) {
         ok = false;
         break;
@@ -1062,12 +1193,10 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
     l_run[r] = l;
     inv_l[r] = (l > 0.f) ? 1.f / l : 0.f;
   }
-  uint8_t* stage = s.q + qt * C::Q_BYTES;
-  constexpr int CPR = D / 8;  // 16-byte chunks per row
-  // the tile's last P.V, on its single-phase barrier (see fwd_softmax)
+  // the tile's last P.V, on o_final (see fwd_softmax)
   fwd_test_delay(p);
   if (ok && n > 0)
-    ok = __all_sync(0xffffffffu, mbar_wait(&s.o_final[qt], 0, s.abort, p.err,
+    ok = __all_sync(0xffffffffu, mbar_wait(&s.o_final[qt], st.nt & 1, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 3, p.timeout_ns));
   if (ok) {
     tc_fence_after();
@@ -1082,62 +1211,52 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
         for (int i = 0; i < 32; ++i) o[i] = 0u;
       }
 #pragma unroll
-      for (int x = 0; x < 8; ++x)
+      for (int r = 0; r < 2; ++r) {
+        if (row[r] >= t.sq) continue;
+        const size_t rh = static_cast<size_t>(t.q0 + row[r]) * p.nheads_q + head[r];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
+        for (int x = 0; x < 8; ++x) {
           const float v0 = __uint_as_float(o[4 * x + 2 * r]) * inv_l[r];
           const float v1 = __uint_as_float(o[4 * x + 2 * r + 1]) * inv_l[r];
           const int col = hc * 64 + 8 * x + 2 * cq;
-          if (p.num_splits > 1) {  // SplitKV: fp32 partial, straight from registers
-            if (row[r] < t.sq)
-              *reinterpret_cast<float2*>(
-                  p.o_part +
-                  ((static_cast<size_t>(t.split) * p.total_q + t.q0 + row[r]) * p.nheads_q +
-                   head[r]) * D + col) = make_float2(v0, v1);
-          } else {
-            // 16-byte chunk 8 hc + x of the row, 4 bytes at 4(t%4), swizzled
-            const int rt = rt0 + 8 * r;
-            *reinterpret_cast<uint32_t*>(stage + rt * (D * 2) +
-                                         (((8 * hc + x) ^ (rt & 7)) * 16) + 4 * cq) =
+          if (p.num_splits > 1)  // SplitKV: fp32 partial
+            *reinterpret_cast<float2*>(
+                p.o_part + (static_cast<size_t>(t.split) * p.total_q * p.nheads_q + rh) * D +
+                col) = make_float2(v0, v1);
+          else  // columns col, col + 1 of the row, as bf16
+            *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + rh * D + col) =
                 pack_bf16(v0, v1);
-          }
         }
-    }
-  }
-  named_bar_sync(1 + qt, 256);  // the whole tile is staged
-  if (ok && p.num_splits > 1) {
-    if (cq == 0)
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-        fwd_store_part_lse(p, t, row[r], head[r],
-                           (l_run[r] > 0.f) ? (m_run[r] + __log2f(l_run[r])) * 0.69314718055994530942f
-                                            : -INFINITY);
-  } else if (ok) {
-    const int rows_left = t.sq - tile_row0;
-    uint8_t* out = static_cast<uint8_t*>(p.out);
-    const int tid = lh * 128 + quad * 32 + lane;
-#pragma unroll 4
-    for (int q = tid; q < C::BM * CPR; q += 256) {
-      const int r = q / CPR, ch = q % CPR;
-      if ((r >> p.pack_shift) < rows_left) {
-        const uint4 v =
-            *reinterpret_cast<const uint4*>(stage + r * (D * 2) + ((ch ^ (r & 7)) * 16));
-        const size_t grow = static_cast<size_t>(t.q0 + tile_row0 + (r >> p.pack_shift));
-        const int gh = t.h + (r & ((1 << p.pack_shift) - 1));
-        *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + gh) * D) * 2 + ch * 16) = v;
       }
     }
-    if (p.return_lse && cq == 0) {
+    if (n > 0) {
+      // O is read: the next tile's first P.V may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.o_empty[qt]);
+    }
+    if (cq == 0) {
 #pragma unroll
-      for (int r = 0; r < 2; ++r)
-        if (row[r] < t.sq)
-          p.lse[static_cast<size_t>(head[r]) * p.total_q + t.q0 + row[r]] =
-              (l_run[r] > 0.f) ? (m_run[r] + __log2f(l_run[r])) * 0.69314718055994530942f
-                               : -INFINITY;
+      for (int r = 0; r < 2; ++r) {
+        const float lse = (l_run[r] > 0.f)
+                              ? (m_run[r] + __log2f(l_run[r])) * 0.69314718055994530942f
+                              : -INFINITY;
+        if (p.num_splits > 1)
+          fwd_store_part_lse(p, t, row[r], head[r], lse);
+        else if (p.return_lse && row[r] < t.sq)
+          p.lse[static_cast<size_t>(head[r]) * p.total_q + t.q0 + row[r]] = lse;
+      }
     }
   }
+  st.g += n;
+  if (n > 0) ++st.nt;
+  st.ok = ok;
 }
 
+// One CTA per SM works through its share of the tiles (fwd_tile_index); every
+// role walks the same sequence, and the barriers' phases carry on from tile to
+// tile, so the next tile's Q and K/V loads and its first S overlap the current
+// tile's last blocks and epilogue.
 template <int D, bool CAUSAL, bool SOFTCAP>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -1147,18 +1266,19 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  FwdTile t;
-  if (!fwd_tile<D, CAUSAL>(p, t)) return;  // uniform across the CTA
   const FwdSmem s = fwd_smem<D>(base);
   const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NQ; ++i) mbar_init(&s.q_full[i], 1);
-    // every MMA warp with a query tile releases each ring stage once
-    const int n_mma = (t.m_base + t.rows < t.sq && C::NQ == 2) ? 2 : 1;
+    for (int i = 0; i < C::NQ; ++i) {
+      mbar_init(&s.q_full[i], 1);
+      mbar_init(&s.q_empty[i], 1);
+    }
+    // every MMA warp releases each ring stage once (one with no rows in a
+    // tile releases that tile's stages without reading them)
     for (int i = 0; i < C::NSTAGE; ++i) {
       mbar_init(&s.kv_full[i], 1);
-      mbar_init(&s.kv_empty[i], n_mma);
+      mbar_init(&s.kv_empty[i], C::NQ);
     }
     for (int i = 0; i < C::NSS; ++i) {
       mbar_init(&s.s_full[i], 1);
@@ -1167,6 +1287,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     for (int i = 0; i < C::NQ; ++i) {
       mbar_init(&s.o_ready[i], 1);
       mbar_init(&s.o_final[i], 1);
+      mbar_init(&s.o_empty[i], 4 * C::ROW_SPLIT);
     }
     *s.abort = 0;
     fence_mbar_init();
@@ -1188,17 +1309,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   if (warp < C::SOFTMAX_WARPS) {
     const int grp = warp / 4;
     const int qt = grp / C::ROW_SPLIT;
-    if (t.m_base + qt * t.rows < t.sq) {
+    FwdSoftState st;
+    for (int k = 0; st.ok; ++k) {
+      const long long L = fwd_tile_index(p, k);
+      if (L < 0) break;
+      FwdTile t;
+      if (!fwd_tile<D, CAUSAL>(p, t, L) || t.m_base + qt * t.rows >= t.sq) continue;
       if constexpr (C::ROW_SPLIT == 2)
-        fwd_softmax_rows16<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt, grp % 2);
+        fwd_softmax_rows16<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt, grp % 2, st);
       else
-        fwd_softmax<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt);
+        fwd_softmax<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt, st);
     }
   } else if (warp == C::LOAD_WARP) {
-    if (lane_id() == 0) fwd_load<D>(p, t, s, &tmQ, &tmK, &tmV);
+    if (lane_id() == 0) fwd_load<D, CAUSAL>(p, s, &tmQ, &tmK, &tmV);
   } else {
-    const int qt = warp - C::MMA_WARP;
-    if (t.m_base + qt * t.rows < t.sq) fwd_mma<D>(p, t, s, tmem, qt);
+    fwd_mma<D, CAUSAL>(p, s, tmem, warp - C::MMA_WARP);
     __syncwarp();
   }
   tc_fence_before();

@@ -40,7 +40,12 @@ enum : uint32_t {
   ERR_FWDP_SOFTMAX = 0x1100,
 };
 
-struct FwdPairCfg {
+template <int D_>
+struct FwdPairCfg;
+
+// head_dim 128: stages of (K half, V half), three S buffers, two issuing warps
+template <>
+struct FwdPairCfg<128> {
   static constexpr int D = 128, BM = 128, BN = 128, PANELS = D / 64;
   static constexpr int QPANEL = BM * 128;            // 16 KB: 128 rows x 64 columns
   static constexpr int Q_BYTES = BM * D * 2;         // 32 KB
@@ -70,6 +75,36 @@ struct FwdPairCfg {
   static constexpr int THREADS = 352;
 };
 
+// head_dim 256: 16 KB chunks in MMA consumption order (K of blocks 0 and 1,
+// then V of block g before K of block g + 2), two S buffers, one issuing warp.
+// Per block and CTA: K half = 2 chunks of 64 keys x 128 columns (two K-major
+// panels), V half = 2 chunks of 64 keys x this CTA's 128 columns (two MN-major
+// panels).  Tensor memory: S x2 (128 columns) + O (256) = 512.
+template <>
+struct FwdPairCfg<256> {
+  static constexpr int D = 256, BM = 128, BN = 128, PANELS = D / 64;
+  static constexpr int QPANEL = BM * 128;            // 16 KB: 128 rows x 64 columns
+  static constexpr int Q_BYTES = BM * D * 2;         // 64 KB
+  static constexpr int CHUNK = 64 * 256;             // 16 KB: 64 rows x two 128-byte panels
+  static constexpr int CPANEL = 64 * 128;            // 8 KB: one panel of a chunk
+  static constexpr int NSTAGE = 9;                   // one chunk per stage
+  static constexpr int STAGE_BYTES = CHUNK;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = OFF_Q + Q_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + NSTAGE * STAGE_BYTES;
+  static constexpr int NS = 2;
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 2 * NS + 2 + 1 + NS;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static constexpr int COL_O = NS * BN;              // S buffers at columns 0, 128
+  static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_S = idesc_bf16(256, BN, false, false);
+  static constexpr uint32_t IDESC_O = idesc_bf16(256, D, false, true);
+  static constexpr int SOFTMAX_WARPS = 8, LOAD_WARP = 8, MMA_WARP = 9;
+  static constexpr int THREADS = 320;
+};
+
 struct FwdPairSmem {
   uint8_t *q, *ring;
   uint64_t *q_full, *kv_full, *kv_empty, *s_full, *p_full, *o_ready, *o_final, *s_free;
@@ -77,8 +112,9 @@ struct FwdPairSmem {
   volatile int* abort;
 };
 
+template <int D>
 __device__ __forceinline__ FwdPairSmem fwd_pair_smem(uint8_t* base) {
-  using C = FwdPairCfg;
+  using C = FwdPairCfg<D>;
   FwdPairSmem s;
   s.q = base + C::OFF_Q;
   s.ring = base + C::OFF_RING;
@@ -98,9 +134,9 @@ __device__ __forceinline__ FwdPairSmem fwd_pair_smem(uint8_t* base) {
 
 // The pair's key-block range covers both CTAs' rows (rows of the pair that do
 // not see a block get P = 0 there); t.m_base is this CTA's first row.
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __device__ __forceinline__ bool fwd_pair_tile(const FwdParams& p, FwdTile& t, uint32_t rank) {
-  using C = FwdPairCfg;
+  using C = FwdPairCfg<D>;
   const int b = blockIdx.z;
   t.split = 0;
   if (p.pack_shift > 0) {
@@ -141,7 +177,7 @@ __device__ __forceinline__ void fwd_pair_load(const FwdParams& p, const FwdTile&
                                               const FwdPairSmem& s, uint32_t rank,
                                               const CUtensorMap* tmQ, const CUtensorMap* tmK,
                                               const CUtensorMap* tmV) {
-  using C = FwdPairCfg;
+  using C = FwdPairCfg<128>;
   const int n = t.n_blocks;
   if (n == 0) return;
   if (rank == 0) mbar_expect_tx(s.q_full, 2 * C::Q_BYTES);
@@ -177,7 +213,7 @@ __device__ __forceinline__ void fwd_pair_load(const FwdParams& p, const FwdTile&
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void fwd_pair_mma(const FwdParams& p, const FwdTile& t,
                                              const FwdPairSmem& s, uint32_t tmem, int role) {
-  using C = FwdPairCfg;
+  using C = FwdPairCfg<128>;
   const int n = t.n_blocks;
   if (n == 0) return;
   constexpr uint16_t kBoth = 0x3;
@@ -247,6 +283,156 @@ __device__ __forceinline__ void fwd_pair_mma(const FwdParams& p, const FwdTile& 
 }
 
 // ---------------------------------------------------------------------------
+// head_dim 256 producer (one lane): this CTA's Q once, then its 16 KB chunks in
+// the MMA warp's order (K of blocks 0 and 1, then V of block j before K of
+// block j + 2); every copy completes on the even CTA's barrier.  The even CTA,
+// whose barriers count both CTAs' bytes, lets every issued copy land before it
+// leaves after a timed-out wait; the cluster barrier at the end holds the odd
+// CTA until then.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fwd_pair256_load(const FwdParams& p, const FwdTile& t,
+                                                 const FwdPairSmem& s, uint32_t rank,
+                                                 const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                                                 const CUtensorMap* tmV) {
+  using C = FwdPairCfg<256>;
+  const int n = t.n_blocks;
+  if (n == 0) return;
+  if (rank == 0) mbar_expect_tx(s.q_full, 2 * C::Q_BYTES);
+  const uint32_t q_bar = mapa_shared(smem_u32(s.q_full), 0);
+  for (int pn = 0; pn < C::PANELS; ++pn)
+    tma_load_3d_pair(s.q + pn * C::QPANEL, tmQ, q_bar, pn * 64, t.h, t.q0 + t.m_base);
+  uint32_t ring = 0;
+  auto drain = [&]() {
+    if (rank != 0) return;
+    mbar_wait_drain(s.q_full, 0, 100000000ull);
+    const uint32_t first = ring > (uint32_t)C::NSTAGE ? ring - C::NSTAGE : 0u;
+    for (uint32_t r = first; r < ring; ++r)
+      mbar_wait_drain(&s.kv_full[r % C::NSTAGE], (r / C::NSTAGE) & 1, 100000000ull);
+  };
+  // chunk c (keys [64c, 64c + 64) for V, columns [128c, 128c + 128) for K) of
+  // block j, as two 64-column panels
+  auto chunk = [&](bool is_v, int j, int c) -> bool {
+    const uint32_t st = ring % C::NSTAGE;
+    if (ring >= (uint32_t)C::NSTAGE &&
+        !mbar_wait_cluster(&s.kv_empty[st], ((ring / C::NSTAGE) - 1) & 1, s.abort, p.err,
+                           ERR_FWDP_LOAD | 1, p.timeout_ns)) {
+      drain();
+      return false;
+    }
+    if (rank == 0) mbar_expect_tx(&s.kv_full[st], 2 * C::CHUNK);
+    const uint32_t bar = mapa_shared(smem_u32(&s.kv_full[st]), 0);
+    uint8_t* dst = s.ring + st * C::CHUNK;
+    const int key0 = t.k0 + (t.n_lo + j) * C::BN;
+    const int r = static_cast<int>(rank);
+    for (int pn = 0; pn < 2; ++pn) {
+      if (is_v)  // this CTA's columns [128 r + 64 pn, +64)
+        tma_load_3d_pair(dst + pn * C::CPANEL, tmV, bar, r * 128 + pn * 64, t.hk, key0 + c * 64);
+      else       // this CTA's keys [64 r, 64 r + 64)
+        tma_load_3d_pair(dst + pn * C::CPANEL, tmK, bar, c * 128 + pn * 64, t.hk, key0 + r * 64);
+    }
+    ++ring;
+    return true;
+  };
+  auto block = [&](bool is_v, int j) { return chunk(is_v, j, 0) && chunk(is_v, j, 1); };
+  if (!block(false, 0)) return;
+  if (n > 1 && !block(false, 1)) return;
+  for (int j = 0; j < n; ++j) {
+    if (!block(true, j)) return;
+    if (j + 2 < n && !block(false, j + 2)) return;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// head_dim 256 MMA warp of the even CTA: S(0), S(1), then P(j).V before
+// S(j + 2), each waiting chunk by chunk; one issuing thread, so S(j + 2)
+// cannot overwrite P(j) before its P.V has read it.
+//   S    M = 256: A = each CTA's Q rows, B = each CTA's 64 keys, 16 k-steps
+//   O   += P V   M = 256, N = 256: A = P in tensor memory, B = each CTA's 128
+//               columns of V (MN-major), 8 k-steps of 16 keys
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fwd_pair256_mma(const FwdParams& p, const FwdTile& t,
+                                                const FwdPairSmem& s, uint32_t tmem) {
+  using C = FwdPairCfg<256>;
+  const int n = t.n_blocks;
+  if (n == 0) return;
+  constexpr uint16_t kBoth = 0x3;
+  uint32_t stage = 0, phase = 0;
+  auto wait = [&](uint64_t* bar, uint32_t parity, uint32_t code) -> bool {
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait_cluster(bar, parity, s.abort, p.err, ERR_FWDP_MMA | code,
+                                      p.timeout_ns)))
+      return false;
+    tc_fence_after();
+    return true;
+  };
+  auto release = [&]() {
+    mma2_commit_to(&s.kv_empty[stage], kBoth);
+    if (++stage == (uint32_t)C::NSTAGE) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  };
+  // descriptors of the Q panel 0 and of ring chunk 0 (K-major K, MN-major V);
+  // byte offsets are added as offset / 16 (the start-address field)
+  const uint64_t qd0 = sdesc_sw128(smem_u32(s.q), 16, 1024);
+  const uint64_t kd0 = sdesc_sw128(smem_u32(s.ring), 16, 1024);
+  const uint64_t vd0 = sdesc_sw128(smem_u32(s.ring), C::CPANEL, 1024);
+  auto issue_s = [&](int slot) -> bool {
+    const uint32_t d = tmem + slot * C::BN;
+    for (int c = 0; c < 2; ++c) {
+      if (!wait(&s.kv_full[stage], phase, 2)) return false;
+      const uint64_t kd = kd0 + ((stage * C::CHUNK) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {  // columns 128c + 16kk
+        const int col = 128 * c + 16 * kk;
+        mma2_ss(d, qd0 + (((col >> 6) * C::QPANEL + (col & 63) * 2) >> 4),
+                kd + (((kk >> 2) * C::CPANEL + (kk & 3) * 32) >> 4), C::IDESC_S,
+                (c | kk) ? 1u : 0u);
+      }
+      release();
+    }
+    return true;
+  };
+  auto issue_pv = [&](int slot, bool acc) -> bool {
+    for (int c = 0; c < 2; ++c) {
+      if (!wait(&s.kv_full[stage], phase, 2)) return false;
+      const uint64_t vd = vd0 + ((stage * C::CHUNK) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {  // keys 64c + 16kk
+        const int ks = 4 * c + kk;
+        mma2_ts(tmem + C::COL_O, tmem + slot * C::BN + ks * 8, vd + ((kk * 16 * 128) >> 4),
+                C::IDESC_O, (acc || ks) ? 1u : 0u);
+      }
+      release();
+    }
+    return true;
+  };
+  TRACE_INIT();
+  if (!wait(s.q_full, 0, 1)) return;
+  if (!issue_s(0)) return;
+  mma2_commit_to(&s.s_full[0], kBoth);
+  if (n > 1) {
+    if (!issue_s(1)) return;
+    mma2_commit_to(&s.s_full[1], kBoth);
+  }
+  for (int j = 0; j < n; ++j) {
+    const int slot = j & 1;
+    [[maybe_unused]] const int tr = (j < 64) ? 2048 + 16 * j : -1;
+    TRACE(tr);
+    if (!wait(&s.p_full[slot], (j >> 1) & 1, 3)) return;
+    TRACE(tr + 1);
+    if (!issue_pv(slot, j > 0)) return;
+    mma2_commit_to(&s.o_ready[j & 1], kBoth);
+    if (j + 2 < n) {
+      if (!issue_s(slot)) return;
+      mma2_commit_to(&s.s_full[slot], kBoth);
+    }
+    TRACE(tr + 2);
+  }
+  mma2_commit_to(s.o_final, kBoth);
+}
+
+// ---------------------------------------------------------------------------
 // softmax: eight warps per CTA.  Warp w serves the 16 tile rows
 // [32 (w & 3) + 16 lh, +16), lh = w >> 2, over all 128 keys of every block,
 // through 16-lane tensor-memory accesses (its lane quadrant is w & 3): thread t
@@ -261,11 +447,11 @@ __device__ __forceinline__ void fwd_pair_mma(const FwdParams& p, const FwdTile& 
 #ifndef ATTN_FWDP_TURNS
 #define ATTN_FWDP_TURNS 1
 #endif
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __device__ __forceinline__ void fwd_pair_softmax(const FwdParams& p, const FwdTile& t,
                                                  const FwdPairSmem& s, uint32_t tmem,
                                                  uint32_t rank, int lh) {
-  using C = FwdPairCfg;
+  using C = FwdPairCfg<D>;
   const int quad = (threadIdx.x >> 5) & 3;
   const int lane = lane_id();
   const int cq = lane & 3;
@@ -435,7 +621,7 @@ __device__ __forceinline__ void fwd_pair_softmax(const FwdParams& p, const FwdTi
       tc_fence_after();
       const uint32_t o_addr = tmem + lane_base + C::COL_O;
 #pragma unroll 1
-      for (int hc = 0; hc < 2; ++hc) {
+      for (int hc = 0; hc < C::D / 64; ++hc) {
         uint32_t o[32];
         tmem_ld16r_x8(o_addr + hc * 64, o);
 #pragma unroll
@@ -480,7 +666,7 @@ __device__ __forceinline__ void fwd_pair_softmax(const FwdParams& p, const FwdTi
     tc_fence_after();
     const uint32_t o_addr = tmem + lane_base + C::COL_O;
 #pragma unroll 1
-    for (int hc = 0; hc < 2; ++hc) {  // columns [64 hc, 64 hc + 64) = Q panel hc
+    for (int hc = 0; hc < C::D / 64; ++hc) {  // columns [64 hc, 64 hc + 64) = Q panel hc
       uint32_t o[32];
       if (n > 0) {
         tmem_ld16r_x8(o_addr + hc * 64, o);
@@ -530,25 +716,25 @@ __device__ __forceinline__ void fwd_pair_softmax(const FwdParams& p, const FwdTi
   }
 }
 
-template <bool CAUSAL>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdPairCfg::THREADS, 1)
+template <int D, bool CAUSAL>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdPairCfg<D>::THREADS, 1)
     attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdPairCfg;
+  using C = FwdPairCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t rank = cluster_ctarank();
   FwdTile t;
-  if (!fwd_pair_tile<CAUSAL>(p, t, rank)) return;  // the same for both CTAs
-  const FwdPairSmem s = fwd_pair_smem(base);
+  if (!fwd_pair_tile<D, CAUSAL>(p, t, rank)) return;  // the same for both CTAs
+  const FwdPairSmem s = fwd_pair_smem<D>(base);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     mbar_init(s.q_full, 1);
     for (int i = 0; i < C::NSTAGE; ++i) {
       mbar_init(&s.kv_full[i], 1);
-      mbar_init(&s.kv_empty[i], 2);  // one release per MMA role
+      mbar_init(&s.kv_empty[i], D == 128 ? 2 : 1);  // one release per MMA role
     }
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(&s.s_full[i], 1);
@@ -576,11 +762,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdPairCfg::THREADS,
   tc_fence_after();
   const uint32_t tmem = *s.tmem_base;
   if (warp < C::SOFTMAX_WARPS) {
-    fwd_pair_softmax<CAUSAL>(p, t, s, tmem, rank, warp >> 2);
+    fwd_pair_softmax<D, CAUSAL>(p, t, s, tmem, rank, warp >> 2);
   } else if (warp == C::LOAD_WARP) {
-    if (lane_id() == 0) fwd_pair_load(p, t, s, rank, &tmQ, &tmK, &tmV);
+    if (lane_id() == 0) {
+      if constexpr (D == 128) fwd_pair_load(p, t, s, rank, &tmQ, &tmK, &tmV);
+      else fwd_pair256_load(p, t, s, rank, &tmQ, &tmK, &tmV);
+    }
   } else if (rank == 0) {
-    fwd_pair_mma(p, t, s, tmem, warp - C::MMA_WARP);
+    if constexpr (D == 128) fwd_pair_mma(p, t, s, tmem, warp - C::MMA_WARP);
+    else fwd_pair256_mma(p, t, s, tmem);
     __syncwarp();
   }
   tc_fence_before();

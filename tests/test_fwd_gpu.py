@@ -197,3 +197,20 @@ def test_large_scores_stay_finite():
     check_o(out.float().cpu().numpy(), ref_o, ref_pabsv, wl.name)
     # |LSE| ~ 100 here: allow the same relative error as at |LSE| ~ 1
     assert lse_err(lse.cpu().numpy(), ref_l) <= LSE_TOL * max(1.0, np.abs(ref_l).max() / 10)
+
+
+# The forward's grid: persistent CTAs (one per SM, each walking a static share
+# of the tiles, the barrier phases running on from tile to tile) for equal
+# segments without key bounds, one CTA per tile otherwise.  Each mode forced on
+# the other's workloads: ragged and empty segments, masks, windows, softcap,
+# SplitKV, and more tiles than CTAs so each CTA walks several.
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("grid", ["persistent", "tiles"])
+def test_grid_modes_forced(d, grid, monkeypatch):
+    monkeypatch.setenv("ATTN_FWD_GRID", grid)
+    check_full(si.Workload(f"grid_{grid}_ragged_d{d}", RAGGED, 4, 2, d, True, seed=90))
+    check_full(si.Workload(f"grid_{grid}_dense_d{d}", [1024] * 6, 8, 8, d, False, seed=91))
+    wl = si.Workload(f"grid_{grid}_window_d{d}", [300, 1, 515, 129, 0, 700], 8, 1, d, True,
+                     lengths_k=[400, 1, 515, 64, 9, 700], seed=92)
+    check_full(wl, window=(100, 37), softcap=20.0)
+    check_full(wl, num_splits=3)
