@@ -232,7 +232,7 @@ bool fwd_use_pair(int d) {
   const char* e = std::getenv("ATTN_FWD_PAIR");
   if (e && e[0] == '1') return true;
   if (e && e[0] == '0') return false;
-  return false;
+  return d == 256;
 }
 
 template <int D, bool CAUSAL>
@@ -271,10 +271,14 @@ attn_status_t launch_fwd_pair(const void* q, const void* k, const void* v, int t
 
 // The forward's grid.  Persistent (one CTA per SM, each walking a static
 // share of the tiles, so a tile's loads and first MMAs overlap the previous
-// tile's epilogue) when every tile has the same work; otherwise one CTA per
-// tile, so the hardware hands tiles of unequal work to whichever SM is free
-// (a static share measured 17% slower on a varlen batch).  ATTN_FWD_GRID=
-// tiles / persistent forces either (read on every call, for tests).
+// tile's epilogue) when every tile has the same, small amount of work
+// (uniform_tiles); otherwise one CTA per tile, so the hardware hands tiles of
+// unequal work to whichever SM is free (a static share measured 17% slower on
+// a varlen batch) and long tiles keep the single-tile epilogue, which stages O
+// through shared memory.  ATTN_FWD_GRID=tiles / persistent forces either (read
+// on every call, for tests).
+constexpr int kPersistMaxBlocks = 4;
+
 bool fwd_grid_persistent(const FwdParams& p) {
   const char* e = std::getenv("ATTN_FWD_GRID");
   if (e && std::strcmp(e, "tiles") == 0) return false;
@@ -553,10 +557,15 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
         bwd_align256(static_cast<size_t>(num_splits) * total_q * nheads_q * head_dim * 4));
   }
   p.pack_shift = pack_gqa_shift(nheads_q / nheads_kv);
-  // equal segments have total = batch x max (no segment is longer than max)
+  // equal segments have total = batch x max (no segment is longer than max);
+  // a persistent grid pays off only for short tiles (set-up and pipeline fill
+  // are then a large share), so tiles of more than kPersistMaxBlocks key
+  // blocks keep one CTA per tile
+  const int block_keys = head_dim == 64 ? 96 : (head_dim == 128 ? 64 : 128);
   p.uniform_tiles = !mk.upper && mk.lo_off >= kNoBound && num_splits == 1 &&
                     static_cast<int64_t>(batch) * max_seqlen_q == total_q &&
-                    static_cast<int64_t>(batch) * max_seqlen_k == total_k;
+                    static_cast<int64_t>(batch) * max_seqlen_k == total_k &&
+                    (max_seqlen_k + block_keys - 1) / block_keys <= kPersistMaxBlocks;
   p.timeout_ns = wait_timeout_ns();
   p.epilogue_delay_ns = test_epilogue_delay_ns();
 

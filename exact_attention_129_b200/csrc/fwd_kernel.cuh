@@ -99,8 +99,9 @@ struct FwdParams {
   int tiles_x;
   int tiles_y;
   long long tiles_total;
-  // host-side only: every tile has the same work (equal segments, no upper or
-  // lower key bound, no split), so a static share per CTA is balanced
+  // host-side only: every tile has the same, small work (equal segments of at
+  // most 4 key blocks, no upper or lower key bound, no split), so a static
+  // share per CTA is balanced and worth its tile-to-tile overlap
   int uniform_tiles;
   uint64_t timeout_ns;
   // test hook (0 in normal use): the softmax warps idle this long before their
@@ -342,40 +343,29 @@ __device__ __forceinline__ bool fwd_tile(const FwdParams& p, FwdTile& t, long lo
   return true;
 }
 
-// Walks the key blocks of this CTA's tiles in order (tiles without blocks are
-// skipped): block j of tile t.  The producer and the MMA warps each keep two,
-// one a block ahead of the other.
-template <int D, bool CAUSAL>
-struct FwdBlocks {
-  const FwdParams& p;
-  FwdTile t;
-  int k = -1;     // position of the tile in this CTA's sequence
-  int j = 0;      // block within the tile
-  bool ok = false;
-  __device__ explicit FwdBlocks(const FwdParams& p_) : p(p_) { next_tile(); }
-  __device__ void next_tile() {
-    while (true) {
-      const long long L = fwd_tile_index(p, ++k);
-      if (L < 0) {
-        ok = false;
-        return;
-      }
-      if (fwd_tile<D, CAUSAL>(p, t, L) && t.n_blocks > 0) break;
-    }
-    j = 0;
-    ok = true;
-  }
-  __device__ void advance() {
-    if (++j >= t.n_blocks) next_tile();
-  }
-  __device__ bool has_rows(int qt) const { return t.m_base + qt * t.rows < t.sq; }
-};
+// A tile's fields taken from lane 0 (for warp-wide callers): every lane holds
+// the same values anyway, but after the shuffles the compiler knows it, so
+// tensor-memory addresses and MMA operands derived from them stay in uniform
+// registers.
+__device__ __forceinline__ void fwd_tile_uniform(FwdTile& t) {
+  t.q0 = __shfl_sync(0xffffffffu, t.q0, 0);
+  t.sq = __shfl_sync(0xffffffffu, t.sq, 0);
+  t.k0 = __shfl_sync(0xffffffffu, t.k0, 0);
+  t.sk = __shfl_sync(0xffffffffu, t.sk, 0);
+  t.m_base = __shfl_sync(0xffffffffu, t.m_base, 0);
+  t.rows = __shfl_sync(0xffffffffu, t.rows, 0);
+  t.n_lo = __shfl_sync(0xffffffffu, t.n_lo, 0);
+  t.n_blocks = __shfl_sync(0xffffffffu, t.n_blocks, 0);
+  t.h = __shfl_sync(0xffffffffu, t.h, 0);
+  t.hk = __shfl_sync(0xffffffffu, t.hk, 0);
+  t.split = __shfl_sync(0xffffffffu, t.split, 0);
+}
 
 // ---------------------------------------------------------------------------
-// producer warp (one lane): for each of the CTA's tiles its Q tiles, then K/V
-// chunks in MMA consumption order, without a break between tiles.  A tile's Q
-// is loaded once the MMA warp's last S of the previous tile has read the Q
-// buffer (q_empty), so it lands while the previous tile finishes.
+// producer warp (one lane): for each of the CTA's tiles, its Q tiles, then K/V
+// chunks in MMA consumption order; the ring runs on from tile to tile.  A
+// tile's Q is loaded once the MMA warp's last S of the previous tile has read
+// the Q buffer (q_empty), so it lands while the previous tile finishes.
 // ---------------------------------------------------------------------------
 template <int D, bool CAUSAL>
 __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdSmem& s,
@@ -410,15 +400,19 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdSmem& s,
     ++ring;
     return true;
   };
-  // the Q tiles of a tile, once the previous Q in each buffer has been read
-  auto load_q = [&](const FwdTile& t) -> bool {
+  for (int k = 0;; ++k) {
+    const long long L = fwd_tile_index(p, k);
+    if (L < 0) return;
+    FwdTile t;
+    if (!fwd_tile<D, CAUSAL>(p, t, L) || t.n_blocks == 0) continue;
+    // the Q tiles, once the previous Q in each buffer has been read
     for (int qt = 0; qt < C::NQ; ++qt) {
       if (t.m_base + qt * t.rows >= t.sq) break;
       if (q_loads[qt] > 0 &&
           !mbar_wait(&s.q_empty[qt], (q_loads[qt] - 1) & 1, s.abort, p.err, ERR_FWD_LOAD | 2,
                      p.timeout_ns)) {
         drain();
-        return false;
+        return;
       }
       mbar_expect_tx(&s.q_full[qt], C::Q_BYTES);
       // one box per panel: t.rows query rows x (packed: all G heads) x 64 columns
@@ -427,63 +421,46 @@ __device__ __forceinline__ void fwd_load(const FwdParams& p, const FwdSmem& s,
                     t.q0 + t.m_base + qt * t.rows);
       ++q_loads[qt];
     }
-    return true;
-  };
-  // K block j of tile t: one chunk per 64-column panel (BN rows, K-major)
-  auto load_k = [&](const FwdTile& t, uint8_t* dst, uint64_t* full, int j, int c) {
-    tma_load_3d(dst, tmK, full, c * 64, t.hk, t.k0 + (t.n_lo + j) * C::BN);
-  };
-  // rows [c*VROWS, (c+1)*VROWS) of V block j: all D columns, panel by panel
-  auto load_v = [&](const FwdTile& t, uint8_t* dst, uint64_t* full, int j, int c) {
-    for (int pn = 0; pn < C::PANELS; ++pn)
-      tma_load_3d(dst + pn * (C::VROWS * 128), tmV, full, pn * 64, t.hk,
-                  t.k0 + (t.n_lo + j) * C::BN + c * C::VROWS);
-  };
-  FwdBlocks<D, CAUSAL> kc(p);  // next block whose K is loaded
-  FwdBlocks<D, CAUSAL> vc(p);  // next block whose V is loaded
-  uint8_t* base;
-  uint64_t* full;
-  if constexpr (C::DBUF) {
-    // stage = (K of the next block, V of the block before it), exactly what one
-    // MMA iteration consumes; the first holds only K, the last only V
-    bool v_on = false;
-    while (kc.ok || (v_on && vc.ok)) {
-      if (kc.ok && kc.j == 0 && !load_q(kc.t)) return;
-      const bool has_v = v_on && vc.ok;
-      const uint32_t bytes =
-          (kc.ok ? C::PANELS * C::CHUNK : 0) + (has_v ? C::PANELS * C::CHUNK : 0);
-      if (!claim(bytes, base, full)) return;
-      for (int c = 0; c < C::PANELS; ++c) {
-        if (kc.ok) load_k(kc.t, base + c * C::CHUNK, full, kc.j, c);
-        if (has_v) load_v(vc.t, base + (C::PANELS + c) * C::CHUNK, full, vc.j, c);
-      }
-      if (has_v) vc.advance();
-      if (kc.ok) kc.advance();
-      v_on = true;
-    }
-  } else {
-    // one chunk per stage, in the MMA warp's order: K of blocks 0 and 1, then
-    // V of block g before K of block g + 2
-    auto load_tile = [&](bool is_v, const FwdTile& t, int j) -> bool {
-      for (int c = 0; c < C::PANELS; ++c) {
-        if (!claim(C::CHUNK, base, full)) return false;
-        if (is_v) load_v(t, base, full, j, c);
-        else load_k(t, base, full, j, c);
-      }
-      return true;
+    // K block j: one chunk per 64-column panel (BN rows, K-major)
+    auto load_k = [&](uint8_t* dst, uint64_t* full, int j, int c) {
+      tma_load_3d(dst, tmK, full, c * 64, t.hk, t.k0 + (t.n_lo + j) * C::BN);
     };
-    auto next_k = [&]() -> bool {
-      if (!kc.ok) return true;
-      if (kc.j == 0 && !load_q(kc.t)) return false;
-      if (!load_tile(false, kc.t, kc.j)) return false;
-      kc.advance();
-      return true;
+    // rows [c*VROWS, (c+1)*VROWS) of V block j: all D columns, panel by panel
+    auto load_v = [&](uint8_t* dst, uint64_t* full, int j, int c) {
+      for (int pn = 0; pn < C::PANELS; ++pn)
+        tma_load_3d(dst + pn * (C::VROWS * 128), tmV, full, pn * 64, t.hk,
+                    t.k0 + (t.n_lo + j) * C::BN + c * C::VROWS);
     };
-    if (!next_k() || !next_k()) return;
-    while (vc.ok) {
-      if (!load_tile(true, vc.t, vc.j)) return;
-      vc.advance();
-      if (!next_k()) return;
+    const int n = t.n_blocks;
+    uint8_t* base;
+    uint64_t* full;
+    if constexpr (C::DBUF) {
+      // stage j = (K_j, V_{j-1}); the first holds only K_0, the last only V_{n-1}
+      for (int j = 0; j <= n; ++j) {
+        const uint32_t bytes =
+            ((j < n) ? C::PANELS * C::CHUNK : 0) + ((j > 0) ? C::PANELS * C::CHUNK : 0);
+        if (!claim(bytes, base, full)) return;
+        for (int c = 0; c < C::PANELS; ++c) {
+          if (j < n) load_k(base + c * C::CHUNK, full, j, c);
+          if (j > 0) load_v(base + (C::PANELS + c) * C::CHUNK, full, j - 1, c);
+        }
+      }
+    } else {
+      // one chunk per stage, in the MMA warp's order: K_0, K_1, then V_j before K_{j+2}
+      auto load_tile = [&](bool is_v, int j) -> bool {
+        for (int c = 0; c < C::PANELS; ++c) {
+          if (!claim(C::CHUNK, base, full)) return false;
+          if (is_v) load_v(base, full, j, c);
+          else load_k(base, full, j, c);
+        }
+        return true;
+      };
+      if (!load_tile(false, 0)) return;
+      if (n > 1 && !load_tile(false, 1)) return;
+      for (int j = 0; j < n; ++j) {
+        if (!load_tile(true, j)) return;
+        if (j + 2 < n && !load_tile(false, j + 2)) return;
+      }
     }
   }
 }
@@ -610,111 +587,122 @@ struct FwdMma {
   }
 };
 
-// The MMA warp of query tile qt walks the CTA's key blocks across all its
-// tiles in the producer's order.  A tile's first S waits for its Q (q_full),
-// its last S releases the Q buffer (q_empty); its first P.V (which overwrites
-// O) waits until the epilogue of the previous tile has read O (o_empty), its
-// last P.V completes o_final.  Blocks of tiles in which this query tile has
-// no rows are only released.  The S slots and barrier phases run on over the
-// tiles (g_s, g_v count this warp's S and P.V).
-template <int D, bool CAUSAL>
-__device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem& s, uint32_t tmem,
-                                        int qt) {
+// The MMA warp of query tile qt, over the CTA's tiles.  A tile's first S waits
+// for its Q (q_full), its last S releases the Q buffer (q_empty); its first
+// P.V (which overwrites O) waits until the epilogue of the previous tile has
+// read O (o_empty), its last P.V completes o_final.  The S slots, ring stages
+// and barrier phases run on over the tiles (g counts this warp's blocks); a
+// tile in which this query tile has no rows only has its stages released.
+// (qt is a template parameter so that every MMA operand and barrier address is
+// a compile-time function of it.)
+template <int D, bool CAUSAL, int qt>
+__device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem& s, uint32_t tmem) {
   using C = FwdCfg<D>;
   TRACE_INIT();
   FwdMma<D> m(p, s, tmem);
-  FwdBlocks<D, CAUSAL> sc(p);  // next block whose S is issued
-  FwdBlocks<D, CAUSAL> vc(p);  // next block whose P.V is issued
-  uint32_t g_s = 0, g_v = 0;   // S and P.V issued by this warp
-  uint32_t q_uses = 0;         // Q tiles read (phases of q_full / q_empty)
-  uint32_t o_tiles = 0;        // tiles whose first P.V was issued (phases of o_empty)
-  auto wait = [&](uint64_t* bar, uint32_t parity, uint32_t code) -> bool {
-    if (!mbar_wait_warp(bar, parity, s.abort, p.err, ERR_FWD_MMA | code, p.timeout_ns))
-      return false;
-    tc_fence_after();
-    return true;
-  };
-  // the P.V of the block at vc into slot `slot`, V in ring chunk ch (DBUF) or
-  // streamed chunk by chunk
-  auto pv = [&](int slot, uint32_t ch) -> bool {
-    if (!wait(&s.p_full[slot], (g_v >> 1) & 1, 3)) return false;
-    if (vc.j == 0) {
-      if (o_tiles > 0 && !wait(&s.o_empty[qt], (o_tiles - 1) & 1, 4)) return false;
-      ++o_tiles;
-    }
-    if constexpr (C::DBUF) {
-      m.issue_pv(qt, slot, ch, vc.j > 0);
-    } else {
-      if (!m.issue_pv_streamed(qt, slot, vc.j > 0)) return false;
-    }
-    mma_commit(&s.o_ready[qt]);
-    if (vc.j == vc.t.n_blocks - 1) mma_commit(&s.o_final[qt]);
-    ++g_v;
-    return true;
-  };
-
-  if constexpr (C::DBUF) {
-    // Both MMA warps read every ring stage and both release it (the empty
-    // barriers count one arrival per query tile).  Stage = (K of the next
-    // block, V of the block before it): S of a block is issued before the P.V
-    // of the previous one, so the tensor pipe has work while the softmax runs.
-    // S(g) lives in slot 2qt + (g & 1); the slot it overwrites held P(g - 2),
-    // read by the P.V this thread issued one step earlier on the same in-order
-    // pipe.
-    bool v_on = false;
-    while (sc.ok || (v_on && vc.ok)) {
-      [[maybe_unused]] const int tr = (g_s < 64) ? 2048 + 16 * g_s + 8 * qt : -1;
-      TRACE(tr);
+  uint32_t g = 0;       // blocks of this query tile so far (S slot and p_full phases)
+  uint32_t tiles = 0;   // tiles with rows for this query tile (q_full / o_empty phases)
+  for (int k = 0;; ++k) {
+    const long long L = fwd_tile_index(p, k);
+    if (L < 0) return;
+    FwdTile t;
+    fwd_tile<D, CAUSAL>(p, t, L);
+    fwd_tile_uniform(t);
+    if (t.m_base >= t.sq || t.n_blocks == 0) continue;  // no rows, or no blocks
+    const int n = t.n_blocks;
+    g = __shfl_sync(0xffffffffu, g, 0);  // warp-uniform, see fwd_softmax
+    if (t.m_base + qt * t.rows >= t.sq) {
+      // no rows for this query tile: release the tile's stages as they fill
       uint32_t ch;
-      if (!m.wait_stages(1, ch)) return;
-      TRACE(tr + 1);
-      if (sc.ok && sc.has_rows(qt)) {
-        if (sc.j == 0 && !wait(&s.q_full[qt], q_uses & 1, 2)) return;
-        const int slot = 2 * qt + (g_s & 1);
-        m.issue_s(qt, slot, ch);
-        mma_commit(&s.s_full[slot]);
-        if (sc.j == sc.t.n_blocks - 1) {
-          mma_commit(&s.q_empty[qt]);
-          ++q_uses;
-        }
-        ++g_s;
+      for (int j = 0; j <= n; ++j) {
+        if (!m.wait_stages(1, ch)) return;
+        m.release_stages(1);
       }
-      TRACE(tr + 2);
-      if (v_on && vc.ok && vc.has_rows(qt) && !pv(2 * qt + (g_v & 1), ch + C::PANELS)) return;
-      TRACE(tr + 4);
-      m.release_stages(1);
-      if (v_on && vc.ok) vc.advance();
-      if (sc.ok) sc.advance();
-      v_on = true;
+      continue;
     }
-  } else {
-    // one query tile, two S slots alternating over the blocks; one chunk per
-    // stage, each waited for right before its MMAs.  Order: S of blocks 0 and
-    // 1, then P.V of block g before S of block g + 2.
-    auto next_s = [&]() -> bool {
-      if (!sc.ok) return true;
-      if (sc.j == 0 && !wait(&s.q_full[0], q_uses & 1, 2)) return false;
-      const int slot = g_s & 1;
-      if (!m.issue_s_streamed(0, slot)) return false;
-      mma_commit(&s.s_full[slot]);
-      if (sc.j == sc.t.n_blocks - 1) {
-        mma_commit(&s.q_empty[0]);
-        ++q_uses;
-      }
-      ++g_s;
-      sc.advance();
+    if (!mbar_wait_warp(&s.q_full[qt], tiles & 1, s.abort, p.err, ERR_FWD_MMA | 2, p.timeout_ns))
+      return;
+    tc_fence_after();
+    // the first P.V of a tile waits for the previous tile's epilogue
+    auto o_free = [&]() -> bool {
+      if (tiles == 0) return true;
+      if (!mbar_wait_warp(&s.o_empty[qt], (tiles - 1) & 1, s.abort, p.err, ERR_FWD_MMA | 4,
+                          p.timeout_ns))
+        return false;
+      tc_fence_after();
       return true;
     };
-    if (!next_s() || !next_s()) return;
-    while (vc.ok) {
-      [[maybe_unused]] const int tr = (g_v < 64) ? 2048 + 16 * g_v : -1;
-      TRACE(tr);
-      if (!pv(g_v & 1, 0)) return;
-      TRACE(tr + 3);
-      vc.advance();
-      if (!next_s()) return;
-      TRACE(tr + 5);
+    if constexpr (C::DBUF) {
+      // S of block j lives in slot 2qt + ((g + j) & 1); S(j+1) is issued
+      // before P(j).V so the tensor pipe has work while the softmax runs on
+      // S(j); the slot it overwrites held P(j-1), read by the P.V this thread
+      // issued one iteration earlier on the same in-order pipe.  Stage j holds
+      // K_j in its first PANELS chunks and V_{j-1} in the next PANELS.
+      uint32_t ch;
+      if (!m.wait_stages(1, ch)) return;
+      m.issue_s(qt, 2 * qt + (g & 1), ch);
+      mma_commit(&s.s_full[2 * qt + (g & 1)]);
+      if (n == 1) mma_commit(&s.q_empty[qt]);
+      m.release_stages(1);
+      for (int j = 0; j < n; ++j) {
+        const uint32_t gj = g + j;
+        const int b = gj & 1;
+        [[maybe_unused]] const int tr = (j < 64) ? 2048 + 16 * j + 8 * qt : -1;
+        TRACE(tr);
+        if (!m.wait_stages(1, ch)) return;
+        TRACE(tr + 1);
+        if (j + 1 < n) {
+          m.issue_s(qt, 2 * qt + (b ^ 1), ch);
+          mma_commit(&s.s_full[2 * qt + (b ^ 1)]);
+          if (j + 2 == n) mma_commit(&s.q_empty[qt]);
+        }
+        TRACE(tr + 2);
+        if (!mbar_wait_warp(&s.p_full[2 * qt + b], (gj >> 1) & 1, s.abort, p.err,
+                            ERR_FWD_MMA | 3, p.timeout_ns))
+          return;
+        tc_fence_after();
+        if (j == 0 && !o_free()) return;
+        TRACE(tr + 3);
+        m.issue_pv(qt, 2 * qt + b, ch + C::PANELS, j > 0);
+        mma_commit(&s.o_ready[qt]);
+        m.release_stages(1);
+        TRACE(tr + 4);
+      }
+    } else {
+      // one query tile, two S slots alternating over key blocks; one chunk per
+      // stage, each waited for right before its MMAs
+      if (!m.issue_s_streamed(0, g & 1)) return;
+      mma_commit(&s.s_full[g & 1]);
+      if (n > 1) {
+        if (!m.issue_s_streamed(0, (g + 1) & 1)) return;
+        mma_commit(&s.s_full[(g + 1) & 1]);
+      }
+      if (n <= 2) mma_commit(&s.q_empty[0]);
+      for (int j = 0; j < n; ++j) {
+        const uint32_t gj = g + j;
+        const int slot = gj & 1;
+        [[maybe_unused]] const int tr = (j < 64) ? 2048 + 16 * j : -1;
+        TRACE(tr);
+        if (!mbar_wait_warp(&s.p_full[slot], (gj >> 1) & 1, s.abort, p.err, ERR_FWD_MMA | 3,
+                            p.timeout_ns))
+          return;
+        tc_fence_after();
+        if (j == 0 && !o_free()) return;
+        TRACE(tr + 1);
+        if (!m.issue_pv_streamed(0, slot, j > 0)) return;
+        mma_commit(&s.o_ready[0]);
+        TRACE(tr + 3);
+        if (j + 2 < n) {
+          if (!m.issue_s_streamed(0, slot)) return;
+          mma_commit(&s.s_full[slot]);
+          if (j + 3 == n) mma_commit(&s.q_empty[0]);
+          TRACE(tr + 5);
+        }
+      }
     }
+    mma_commit(&s.o_final[qt]);
+    g += n;
+    ++tiles;
   }
 }
 
@@ -724,7 +712,31 @@ struct FwdSoftState {
   uint32_t g = 0;   // blocks of this query tile processed so far (all tiles)
   uint32_t nt = 0;  // tiles with blocks finished (phases of o_final / o_empty)
   bool ok = true;   // false after a timed-out wait: the warp stops
+  // the CTA has a single tile: no Q follows, so the epilogue stages O through
+  // the Q buffer and stores whole rows (stores straight from registers write
+  // 16-byte pieces of 32 rows at a time, measured 4.5% slower at head_dim 256)
+  bool single = false;
 };
+
+// Coalesced copy of a staged tile (bf16 rows of D columns, 16-byte chunks
+// XOR-swizzled by row) to out, rows past the segment left out.
+template <int D, int NTHR>
+__device__ __forceinline__ void fwd_copy_out(const FwdParams& p, const FwdTile& t,
+                                             const uint8_t* stage, int tile_row0, int tid) {
+  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  const int rows_left = t.sq - tile_row0;
+  uint8_t* out = static_cast<uint8_t*>(p.out);
+#pragma unroll 4
+  for (int q = tid; q < 128 * CPR; q += NTHR) {
+    const int r = q / CPR, ch = q % CPR;
+    if ((r >> p.pack_shift) < rows_left) {
+      const uint4 v = *reinterpret_cast<const uint4*>(stage + r * (D * 2) + ((ch ^ (r & 7)) * 16));
+      const size_t grow = static_cast<size_t>(t.q0 + tile_row0 + (r >> p.pack_shift));
+      const int gh = t.h + (r & ((1 << p.pack_shift) - 1));
+      *reinterpret_cast<uint4*>(out + ((grow * p.nheads_q + gh) * D) * 2 + ch * 16) = v;
+    }
+  }
+}
 
 // one tile's epilogue output: 32 columns of a row's O / l as bf16, straight
 // from registers into out[row][head]
@@ -762,6 +774,9 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
   const int head = t.h + (row_in_tile & ((1 << p.pack_shift) - 1));
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
   const int n = t.n_blocks;
+  // the block count so far, known to the compiler as warp-uniform, so the S
+  // slot addresses derived from it stay in uniform registers
+  const uint32_t g0 = __shfl_sync(0xffffffffu, st.g, 0);
   // with a softcap the scores are turned into capped log2-domain values first
   const float c = SOFTCAP ? 1.f : p.scale_log2;
   // keys [key_lo, key_lim) are allowed for this row
@@ -805,7 +820,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
 
   constexpr int NCOL = C::BN;  // scores per row and block
   for (int j = 0; j < n; ++j) {
-    const uint32_t g = st.g + j;  // this block's index over the CTA's tiles
+    const uint32_t g = g0 + j;  // this block's index over the CTA's tiles
     const int slot = C::DBUF ? 2 * qt + (g & 1) : (g & 1);
     const uint32_t parity = (g >> 1) & 1;
     if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], parity, s.abort, p.err,
@@ -974,10 +989,23 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
 #pragma unroll
         for (int i = 0; i < 32; ++i) r[i] = 0u;
       }
-      if (p.num_splits > 1)  // SplitKV: fp32 partial
+      if (p.num_splits > 1) {  // SplitKV: fp32 partial
         fwd_store_part<D>(p, t, row, head, cc * 32, r, inv_l);
-      else if (row_valid)
+      } else if (st.single) {  // into the Q buffer, 16-byte chunks swizzled by row
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint4 v;
+          v.x = pack_bf16(__uint_as_float(r[g * 8 + 0]) * inv_l, __uint_as_float(r[g * 8 + 1]) * inv_l);
+          v.y = pack_bf16(__uint_as_float(r[g * 8 + 2]) * inv_l, __uint_as_float(r[g * 8 + 3]) * inv_l);
+          v.z = pack_bf16(__uint_as_float(r[g * 8 + 4]) * inv_l, __uint_as_float(r[g * 8 + 5]) * inv_l);
+          v.w = pack_bf16(__uint_as_float(r[g * 8 + 6]) * inv_l, __uint_as_float(r[g * 8 + 7]) * inv_l);
+          const int chunk = cc * 4 + g;
+          *reinterpret_cast<uint4*>(s.q + qt * C::Q_BYTES + row_in_tile * (D * 2) +
+                                    ((chunk ^ (row_in_tile & 7)) * 16)) = v;
+        }
+      } else if (row_valid) {
         fwd_store_o32<D>(p, t, row, head, cc * 32, r, inv_l);
+      }
     }
     if (n > 0) {
       // O is read: the next tile's first P.V may overwrite it
@@ -991,6 +1019,10 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdTile& t
       fwd_store_part_lse(p, t, row, head, lse);
     else if (p.return_lse && row_valid)
       p.lse[static_cast<size_t>(head) * p.total_q + t.q0 + row] = lse;
+  }
+  if (st.single && p.num_splits == 1) {  // every thread of the tile meets the barrier
+    named_bar_sync(1 + qt, 128);
+    if (ok) fwd_copy_out<D, 128>(p, t, s.q + qt * C::Q_BYTES, tile_row0, threadIdx.x & 127);
   }
   // tile 0 takes tile 1's arrive from the tile's last turn
   if (pingpong && qt == 0 && n > 0) named_bar_sync(bar_t0, 64);
@@ -1034,6 +1066,7 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
   }
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32 + lh * 16) << 16;
   const int n = t.n_blocks;
+  const uint32_t g0 = __shfl_sync(0xffffffffu, st.g, 0);  // see fwd_softmax
   const float c = SOFTCAP ? 1.f : p.scale_log2;
   const int mask_from = CAUSAL ? min(t.sk, tile_row0 + delta + p.hi_off + 1) : t.sk;
   const int lo_until = tile_row0 + (t.rows - 1) + delta - p.lo_off;
@@ -1044,7 +1077,7 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
   float l_run[2] = {0.f, 0.f};
   bool ok = true;
   for (int j = 0; j < n; ++j) {
-    const uint32_t g = st.g + j;  // this block's index over the CTA's tiles
+    const uint32_t g = g0 + j;  // this block's index over the CTA's tiles
     const int slot = C::DBUF ? 2 * qt + (g & 1) : (g & 1);
     [[maybe_unused]] const int tr = (tr_on && j < 64) ? 1024 * qt + j * 8 : -1;
     if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[slot], (g >> 1) & 1, s.abort, p.err,
@@ -1194,10 +1227,13 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
     inv_l[r] = (l > 0.f) ? 1.f / l : 0.f;
   }
   // the tile's last P.V, on o_final (see fwd_softmax)
+  [[maybe_unused]] const int tre = tr_on ? 900 + 4 * qt : -1;
+  TRACE(tre);
   fwd_test_delay(p);
   if (ok && n > 0)
     ok = __all_sync(0xffffffffu, mbar_wait(&s.o_final[qt], st.nt & 1, s.abort, p.err,
                                            ERR_FWD_SOFTMAX | 3, p.timeout_ns));
+  TRACE(tre + 1);
   if (ok) {
     tc_fence_after();
     const uint32_t o_addr = tmem + lane_base + C::O_COL0 + qt * D;
@@ -1223,6 +1259,10 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
             *reinterpret_cast<float2*>(
                 p.o_part + (static_cast<size_t>(t.split) * p.total_q * p.nheads_q + rh) * D +
                 col) = make_float2(v0, v1);
+          else if (st.single)  // into the Q buffer, 16-byte chunk 8 hc + x of the row
+            *reinterpret_cast<uint32_t*>(s.q + qt * C::Q_BYTES + (rt0 + 8 * r) * (D * 2) +
+                                         (((8 * hc + x) ^ ((rt0 + 8 * r) & 7)) * 16) + 4 * cq) =
+                pack_bf16(v0, v1);
           else  // columns col, col + 1 of the row, as bf16
             *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + rh * D + col) =
                 pack_bf16(v0, v1);
@@ -1248,6 +1288,12 @@ __device__ __forceinline__ void fwd_softmax_rows16(const FwdParams& p, const Fwd
       }
     }
   }
+  if (st.single && p.num_splits == 1) {  // every thread of the tile meets the barrier
+    named_bar_sync(1 + qt, 256);
+    if (ok)
+      fwd_copy_out<D, 256>(p, t, s.q + qt * C::Q_BYTES, tile_row0, lh * 128 + quad * 32 + lane);
+  }
+  TRACE(tre + 2);
   st.g += n;
   if (n > 0) ++st.nt;
   st.ok = ok;
@@ -1268,6 +1314,20 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const FwdSmem s = fwd_smem<D>(base);
   const int warp = threadIdx.x >> 5;
+  TRACE_INIT();
+  if (threadIdx.x == 0) TRACE(950);
+  // a CTA whose tiles hold no query row (with one CTA per tile, the grid is
+  // sized by the longest segment) leaves before any set-up
+  {
+    bool work = false;
+    for (int k = 0; !work; ++k) {
+      const long long L = fwd_tile_index(p, k);
+      if (L < 0) break;
+      FwdTile t;
+      work = fwd_tile<D, CAUSAL>(p, t, L);
+    }
+    if (!work) return;
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NQ; ++i) {
@@ -1310,11 +1370,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int grp = warp / 4;
     const int qt = grp / C::ROW_SPLIT;
     FwdSoftState st;
+    st.single = fwd_tile_index(p, 1) < 0;
     for (int k = 0; st.ok; ++k) {
       const long long L = fwd_tile_index(p, k);
       if (L < 0) break;
       FwdTile t;
-      if (!fwd_tile<D, CAUSAL>(p, t, L) || t.m_base + qt * t.rows >= t.sq) continue;
+      fwd_tile<D, CAUSAL>(p, t, L);
+      fwd_tile_uniform(t);
+      if (t.m_base + qt * t.rows >= t.sq) continue;  // no rows for this query tile
       if constexpr (C::ROW_SPLIT == 2)
         fwd_softmax_rows16<D, CAUSAL, SOFTCAP>(p, t, s, tmem, qt, grp % 2, st);
       else
@@ -1323,11 +1386,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   } else if (warp == C::LOAD_WARP) {
     if (lane_id() == 0) fwd_load<D, CAUSAL>(p, s, &tmQ, &tmK, &tmV);
   } else {
-    fwd_mma<D, CAUSAL>(p, s, tmem, warp - C::MMA_WARP);
+    if (warp == C::MMA_WARP) fwd_mma<D, CAUSAL, 0>(p, s, tmem);
+    else if constexpr (C::NQ == 2) fwd_mma<D, CAUSAL, 1>(p, s, tmem);
     __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) TRACE(952);
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);

@@ -214,3 +214,17 @@ def test_grid_modes_forced(d, grid, monkeypatch):
                      lengths_k=[400, 1, 515, 64, 9, 700], seed=92)
     check_full(wl, window=(100, 37), softcap=20.0)
     check_full(wl, num_splits=3)
+
+
+# The two-CTA forward (cta_group::2 MMAs over a CTA pair) is the default at
+# head_dim 256 and opt-in at 128; each head_dim forced both ways on ragged,
+# causal, windowed and packed-GQA workloads
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_cta_pair_forced(d, pair, monkeypatch):
+    monkeypatch.setenv("ATTN_FWD_PAIR", pair)
+    check_full(si.Workload(f"pair{pair}_ragged_d{d}", RAGGED, 4, 2, d, True, seed=95))
+    check_full(si.Workload(f"pair{pair}_mha_d{d}", [777, 300], 3, 3, d, False, seed=96))
+    wl = si.Workload(f"pair{pair}_window_d{d}", [300, 1, 515, 129], 8, 1, d, True,
+                     lengths_k=[400, 1, 515, 64], seed=97)
+    check_full(wl, window=(100, 37))
