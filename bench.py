@@ -108,13 +108,22 @@ def strip_c_comments(text: str) -> str:
     return " ".join("".join(out).split())
 
 
-def library_source_hash():
-    """Hash of the kernel and ABI sources with comments removed: a recorded ncu
-    traffic figure stays valid across comment edits, not across code edits."""
+# the sources each timed kernel is compiled from (the C ABI file launches both)
+KERNEL_SOURCES = {
+    "attn_fwd": ("api.cu", "ptx.cuh", "fwd_kernel.cuh", "fwd_pair_kernel.cuh"),
+    "attn_bwd_main": ("api.cu", "ptx.cuh", "bwd_kernels.cuh", "bwd_pair_kernel.cuh"),
+}
+
+
+def library_source_hash(kernel: str | None = None):
+    """Hash of a kernel's sources (all kernel and ABI sources when kernel is None)
+    with comments removed: a recorded ncu traffic figure stays valid across
+    comment edits and edits of other kernels, not across edits of its own code."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_129_b200", "csrc")
+    names = KERNEL_SOURCES.get(kernel) if kernel else None
     for name in sorted(os.listdir(csrc)):
-        if not name.endswith((".cu", ".cuh", ".h")):
+        if not name.endswith((".cu", ".cuh", ".h")) or (names and name not in names):
             continue
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
@@ -131,7 +140,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(path) as f:
         d = json.load(f)
     e = d.get(f"{kernel}/{workload}")
-    if not e or e.get("source_hash") != library_source_hash():
+    if not e or e.get("source_hash") != library_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 

@@ -440,9 +440,10 @@ __device__ __forceinline__ void fwd_pair256_mma(const FwdParams& p, const FwdTil
 // the two keys 2(t%4) and 2(t%4) + 1 (register 4x + 2r + e is row rt0 + 8r,
 // key 8x + 2(t%4) + e).  The four threads of a row combine its max and sum
 // with two shuffles.  The two warps of a quadrant share no rows, so neither
-// waits for the other's scores.  Their exp phases take turns (lane half 0
-// first in each block), so one warp's loads, max and stores overlap the
-// other's exps (ATTN_FWDP_TURNS=0 lets them run freely: slower).
+// waits for the other's scores.  At head_dim 128 their exp phases take turns
+// (lane half 0 first in each block), so one warp's loads, max and stores
+// overlap the other's exps (ATTN_FWDP_TURNS=0 lets them run freely: slower);
+// at head_dim 256 they run freely.
 // ---------------------------------------------------------------------------
 #ifndef ATTN_FWDP_TURNS
 #define ATTN_FWDP_TURNS 1
@@ -452,6 +453,9 @@ __device__ __forceinline__ void fwd_pair_softmax(const FwdParams& p, const FwdTi
                                                  const FwdPairSmem& s, uint32_t tmem,
                                                  uint32_t rank, int lh) {
   using C = FwdPairCfg<D>;
+  // exp turns at head_dim 128 only: at 256 the softmax is not the limit and the
+  // turns' barriers measured 4% slower
+  constexpr bool TURNS = (D == 128) && (ATTN_FWDP_TURNS != 0);
   const int quad = (threadIdx.x >> 5) & 3;
   const int lane = lane_id();
   const int cq = lane & 3;
@@ -570,7 +574,7 @@ __device__ __forceinline__ void fwd_pair_softmax(const FwdParams& p, const FwdTi
       const float m_sub = (m_run[r] == -INFINITY) ? 0.f : m_run[r];
       mm2[r] = f2_pack(-m_sub, -m_sub);
     }
-    if (ATTN_FWDP_TURNS) turn_begin(j);
+    if (TURNS) turn_begin(j);
     {
       const uint64_t cc2 = f2_pack(c, c);
       uint64_t acc[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
@@ -603,7 +607,7 @@ __device__ __forceinline__ void fwd_pair_softmax(const FwdParams& p, const FwdTi
         l_run[r] += a0 + a1;  // this thread's share; the row's four are summed at the end
       }
     }
-    if (ATTN_FWDP_TURNS) turn_end(j);
+    if (TURNS) turn_end(j);
     turns_done = j + 1;
     TRACE(tr + 2);
     if (__any_sync(0xffffffffu, rescale)) {
@@ -640,7 +644,7 @@ __device__ __forceinline__ void fwd_pair_softmax(const FwdParams& p, const FwdTi
     }
     TRACE(tr + 3);
   }
-  if (ATTN_FWDP_TURNS)
+  if (TURNS)
     for (int k = turns_done; k < n; ++k) {
       turn_begin(k);
       turn_end(k);

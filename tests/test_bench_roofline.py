@@ -53,3 +53,19 @@ def test_source_hash_ignores_comments_only():
     assert bench.strip_c_comments(src) == bench.strip_c_comments(
         src.replace("// note", "// another note"))
     assert bench.strip_c_comments(src) != bench.strip_c_comments(src.replace("a = 1", "a = 2"))
+
+
+def test_kernel_source_sets_cover_their_headers():
+    # every kernel's recorded traffic is tied to the files it is compiled from:
+    # the ABI file, the PTX wrappers and its own kernel headers, and those exist
+    csrc = os.path.join(ROOT, "exact_attention_129_b200", "csrc")
+    for kernel, names in bench.KERNEL_SOURCES.items():
+        assert {"api.cu", "ptx.cuh"} <= set(names), kernel
+        for n in names:
+            assert os.path.exists(os.path.join(csrc, n)), (kernel, n)
+    assert any("fwd" in n for n in bench.KERNEL_SOURCES["attn_fwd"])
+    assert not any("fwd" in n for n in bench.KERNEL_SOURCES["attn_bwd_main"])
+    # a kernel's hash is over its own files only, and the whole-library hash differs
+    assert bench.library_source_hash("attn_fwd") != bench.library_source_hash("attn_bwd_main")
+    assert bench.library_source_hash() not in (bench.library_source_hash("attn_fwd"),
+                                               bench.library_source_hash("attn_bwd_main"))
