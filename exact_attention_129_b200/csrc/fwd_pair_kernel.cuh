@@ -185,13 +185,25 @@ __device__ __forceinline__ void fwd_pair_load(const FwdParams& p, const FwdTile&
   for (int pn = 0; pn < C::PANELS; ++pn)
     tma_load_3d_pair(s.q + pn * C::QPANEL, tmQ, q_bar, pn * 64, t.h, t.q0 + t.m_base);
   uint32_t ring = 0;
+  // after a timed-out wait: the even CTA, whose barriers count both CTAs' bytes,
+  // lets every issued copy land before it leaves (the cluster barrier at the
+  // end holds the odd CTA until then)
+  auto drain = [&]() {
+    if (rank != 0) return;
+    mbar_wait_drain(s.q_full, 0, 100000000ull);
+    const uint32_t first = ring > (uint32_t)C::NSTAGE ? ring - C::NSTAGE : 0u;
+    for (uint32_t r = first; r < ring; ++r)
+      mbar_wait_drain(&s.kv_full[r % C::NSTAGE], (r / C::NSTAGE) & 1, 100000000ull);
+  };
   for (int j = 0; j <= n; ++j) {
     const uint32_t st = ring % C::NSTAGE;
     // the stage's previous use is done once the even CTA's MMAs have read it
     if (ring >= (uint32_t)C::NSTAGE &&
         !mbar_wait_cluster(&s.kv_empty[st], ((ring / C::NSTAGE) - 1) & 1, s.abort, p.err,
-                           ERR_FWDP_LOAD | 1, p.timeout_ns))
+                           ERR_FWDP_LOAD | 1, p.timeout_ns)) {
+      drain();
       return;
+    }
     if (rank == 0)
       mbar_expect_tx(&s.kv_full[st], (j < n ? 2 * C::KH_BYTES : 0) + (j > 0 ? 2 * C::VH_BYTES : 0));
     const uint32_t bar = mapa_shared(smem_u32(&s.kv_full[st]), 0);
