@@ -9,10 +9,14 @@
 // B200 at head_dim^-0.5 scale.  This file is our own design of that loop for one
 // B200 SM:
 //
-//   * One CTA owns NQ query tiles of 128 rows of one (segment, head): NQ = 2
-//     for head_dim 64/128 (both tiles share every K/V tile brought on chip),
-//     NQ = 1 for head_dim 256 (its 128 x 256 fp32 accumulator fills half of
-//     tensor memory).
+//   * A tile is NQ query tiles of 128 rows of one (segment, head): NQ = 2 for
+//     head_dim 64/128 (both share every K/V tile brought on chip), NQ = 1 for
+//     head_dim 256 (its 128 x 256 fp32 accumulator fills half of tensor
+//     memory).  A CTA walks a sequence of tiles (fwd_tile_index): one tile per
+//     CTA, or with a persistent grid a static share, the barrier phases and
+//     ring stages running on from tile to tile.  (The default head_dim-256
+//     forward is the two-CTA kernel of fwd_pair_kernel.cuh; this kernel serves
+//     head_dim 256 with a softcap or SplitKV.)
 //   * Warp roles: softmax warps (head_dim 128: one warpgroup per query tile,
 //     thread i owning row i; head_dim 64 and 256: two warpgroups per tile,
 //     each warp over 16 whole rows with four threads per row), one TMA
