@@ -1,33 +1,34 @@
-// fwd_pair_kernel.cuh -- the head_dim-128 forward on a pair of CTAs that share
-// every tensor-core instruction (tcgen05 cta_group::2).
+// fwd_pair_kernel.cuh -- the forward on a pair of CTAs that share every
+// tensor-core instruction (tcgen05 cta_group::2), for head_dim 128 and 256.
 //
-// The one-CTA head_dim-128 forward uses 64-key blocks (four S buffers and two O
-// tiles fill its tensor memory), and an S MMA of M = 128, N = 64 costs ~56
-// cycles for 32 cycles of work.  Here a cluster of two CTAs works on 256 query
-// rows, 128 per CTA (one query tile each), over 128-key blocks, and the even
-// CTA issues M = 256 MMAs that run on both SMs:
+// A cluster of two CTAs works on 256 query rows, 128 per CTA, over 128-key
+// blocks, and the even CTA issues M = 256 MMAs that run on both SMs:
 //
 //   S = Q K^T   A = each CTA's own 128 Q rows, B = K of the block, 64 keys held
 //               by each CTA; D = each CTA's 128 rows x 128 keys (N = 128)
-//   O += P V    A = each CTA's P in tensor memory, B = V of the block, 64 of the
-//               128 columns held by each CTA; D = each CTA's 128 rows x 128
+//   O += P V    A = each CTA's P in tensor memory, B = V of the block, D/2 of
+//               the columns held by each CTA; D = each CTA's 128 rows x D
 //
-// so every MMA runs at N = 128, and each CTA loads half of every K/V block
-// (32 KB per 128 keys instead of 64).  Per CTA: tensor memory S x3 (128 columns
-// each: S(j + 2) is computed while the softmax works on S(j) and P(j + 1) waits
-// for its P.V) + O (128) = the 512 allocated for the pair; shared memory Q
-// (32 KB) + a ring of (K half of block j, V half of block j - 1) stages (32 KB
-// each).  The loads of both CTAs complete on the
-// even CTA's barriers (TMA with cta_group::2, no multicast); its MMA warp
-// commits each MMA group to the same barrier in both CTAs.  Softmax: eight
-// warps per CTA, each over 16 whole rows (16-lane tensor-memory accesses, four
-// threads per row that combine the row's max and sum by shuffles), so no warp
-// waits for another's scores; P (bf16) goes over the first 64 columns of its S
+// so every MMA has N >= 128 and each SM reads half of every B operand and
+// loads half of every K/V block.  The loads of both CTAs complete on the even
+// CTA's barriers (TMA with cta_group::2, no multicast); its MMA warp commits
+// each MMA group to the same barrier in both CTAs.  Softmax: eight warps per
+// CTA, each over 16 whole rows (16-lane tensor-memory accesses, four threads
+// per row that combine the row's max and sum by shuffles), so no warp waits
+// for another's scores; P (bf16) goes over the first 64 columns of its S
 // buffer, and each softmax warp of either CTA reports its P to the even CTA's
 // barrier, because the P.V MMA reads both CTAs' P.
 //
-// Selected for head_dim 128 without softcap and without SplitKV by
-// ATTN_FWD_PAIR=1; the one-CTA kernel in fwd_kernel.cuh is the default.
+//   head_dim 128: tensor memory S x3 (128 columns each: S(j + 2) is computed
+//     while the softmax works on S(j) and P(j + 1) waits for its P.V) + O (128);
+//     shared memory Q (32 KB) + a ring of (K half of block j, V half of block
+//     j - 1) stages (32 KB each); two issuing warps (S, P.V).  The one-CTA
+//     kernel (an S MMA of N = 64 costs ~56 cycles for 32 of work) stays the
+//     default there: both are bound by the softmax warps' exps; selected by
+//     ATTN_FWD_PAIR=1.
+//   head_dim 256 (the default there, without softcap or SplitKV): S x2 + O
+//     (256); Q (64 KB) + a ring of 16 KB chunks in MMA order; one issuing warp.
+//     The one-CTA kernel is bound by shared-memory reads, which the pair halves.
 #pragma once
 
 #include "fwd_kernel.cuh"
